@@ -1,0 +1,182 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never loads it and
+shares no code with it.
+
+Each function takes CPU tensors (torch bf16, or numpy uint16 bf16 bit
+patterns) and returns float64 numpy arrays.  The C source ``oracle.c`` states
+the definition it follows ("What attention costs", samanvya.dev: softmax of
+scaled scores times V, two-pass; "Flash-Decoding" for the log-sum-exp merge).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+
+from .build import build_oracle
+
+_lib = None
+
+_u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
+_i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
+_f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build_oracle())
+        L.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        L.oracle_max_threads.restype = ctypes.c_int
+        L.oracle_attn.argtypes = [_u16p, _u16p, _u16p] + [ctypes.c_int] * 7 + [
+            ctypes.c_double, _f64p, _f64p]
+        L.oracle_attn.restype = ctypes.c_int
+        L.oracle_attn_varlen_rows.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
+        L.oracle_attn_varlen_rows.restype = ctypes.c_int
+        L.oracle_probs.argtypes = [
+            _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 8 + [ctypes.c_double, _f64p]
+        L.oracle_probs.restype = ctypes.c_int
+        L.oracle_decode_paged.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_int64, ctypes.c_double, _f64p, _f64p]
+        L.oracle_decode_paged.restype = ctypes.c_int
+        L.oracle_lse_combine.argtypes = [_f64p, _f64p, ctypes.c_int, ctypes.c_int64,
+                                         ctypes.c_int, _f64p, _f64p]
+        L.oracle_lse_combine.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 bit patterns (uint16, C-contiguous) of a torch bf16 tensor or array."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("numpy inputs must be uint16 bf16 bit patterns")
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype != torch.bfloat16:
+        raise TypeError("torch inputs must be bfloat16")
+    return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _i32(x) -> np.ndarray:
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: bad arguments (rc={rc})")
+
+
+def set_num_threads(n: int) -> None:
+    lib().oracle_set_num_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+def attn(q, k, v, causal=False, window=0, scale=None):
+    """Dense batch.  q [B,N,Hq,d], k/v [B,N,Hkv,d] -> O [B,N,Hq,d], LSE [B,Hq,N]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((B, N, Hq, d), np.float64)
+    lse = np.empty((B, Hq, N), np.float64)
+    _check(lib().oracle_attn(qb, kb, vb, B, Hq, Hkv, N, d, int(causal), int(window),
+                             float(scale), o, lse), "attn")
+    return o, lse
+
+
+def attn_varlen(q, k, v, cu_seqlens, causal=False, window=0, scale=None, rows=None):
+    """Packed sequences.  q [T,Hq,d], k/v [T,Hkv,d], cu_seqlens [S+1].
+
+    Returns O [T,Hq,d] and LSE [Hq,T]; with ``rows`` (global token indices)
+    only those rows: O [R,Hq,d], LSE [R,Hq].
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        nrows, rp = T, None
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows, rp = r.size, r.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((nrows, Hq, d), np.float64)
+    lse = np.empty((nrows, Hq), np.float64)
+    _check(lib().oracle_attn_varlen_rows(qb, kb, vb, cu, len(cu) - 1, Hq, Hkv, d,
+                                         int(causal), int(window), float(scale),
+                                         rp, nrows, o, lse), "attn_varlen")
+    if rows is None:
+        return o, np.ascontiguousarray(lse.T)
+    return o, lse
+
+
+def attn_rows(q, k, v, rows, causal=False, window=0, scale=None):
+    """Dense batch, only query tokens ``rows`` = list of (b, i).
+
+    Returns O [R,Hq,d] and LSE [R,Hq].
+    """
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, Hq, d = qb.shape
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    flat = [int(b) * N + int(i) for b, i in rows]
+    return attn_varlen(qb.reshape(B * N, Hq, d), kb.reshape(B * N, -1, d),
+                       vb.reshape(B * N, -1, d), cu, causal, window, scale, rows=flat)
+
+
+def probs(q, k, v, cu_seqlens, seq, h, causal=False, window=0, scale=None):
+    """Softmax probability matrix [L, L] of one (sequence, head)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    L = int(cu[seq + 1] - cu[seq])
+    p = np.empty((L, L), np.float64)
+    _check(lib().oracle_probs(qb, kb, vb, cu, len(cu) - 1, int(seq), int(h), Hq, Hkv, d,
+                              int(causal), int(window), float(scale), p), "probs")
+    return p
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None):
+    """q [S,Hq,d], caches [P,ps,Hkv,d] -> O [S,Hq,d], LSE [S,Hq]."""
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    S, Hq, d = qb.shape
+    P, ps, Hkv, _ = kb.shape
+    bt = _i32(block_table)
+    sl = _i32(seq_lens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((S, Hq, d), np.float64)
+    lse = np.empty((S, Hq), np.float64)
+    _check(lib().oracle_decode_paged(qb, kb, vb, bt, sl, S, Hq, Hkv, d, ps,
+                                     bt.shape[1], P, float(scale), o, lse),
+           "decode_paged")
+    return o, lse
+
+
+def lse_combine(o_parts, lse_parts):
+    """Merge partials: o_parts [P,R,d], lse_parts [P,R] -> O [R,d], LSE [R]."""
+    op = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lp = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    P, R, d = op.shape
+    o = np.empty((R, d), np.float64)
+    lse = np.empty((R,), np.float64)
+    _check(lib().oracle_lse_combine(op, lp, P, R, d, o, lse), "lse_combine")
+    return o, lse

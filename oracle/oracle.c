@@ -1,0 +1,341 @@
+/*
+ * oracle.c -- plain, slow fp64 CPU definition of exact attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file; only the tests, the smoke check and the bench's CPU-baseline
+ * leg use it.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes (the definition, not the tiled algorithm):
+ *   "What attention costs" (samanvya.dev, attention optimisation post):
+ *       Attention(Q, K, V) = softmax(Q K^T / sqrt(d)) V
+ *   generalised to a caller-given `scale` in place of 1/sqrt(d) and an
+ *   additive mask that is 0 on the allowed key set A(i) and -inf elsewhere.
+ *   The softmax is taken in the textbook two-pass order the same post lists
+ *   for the naive three-kernel flow: all scores of a row, then their max,
+ *   then the exponentials and their sum, then the weighted sum of V rows.
+ *   The score row is materialised in full, one query row at a time.
+ *
+ *   LSE_i = M_i + log(l_i) in natural log, M_i = max_j S_ij,
+ *   l_i = sum_j exp(S_ij - M_i): the "saved softmax statistics" the same post
+ *   names for the backward pass.
+ *
+ * Allowed key sets A(i) (readings of the pages, each stated once here):
+ *   non-causal : every key of the same sequence;
+ *   causal     : keys j <= i ("every token can see every earlier token",
+ *                "Attending to fewer tokens");
+ *   window W>0 : causal and j > i - W, i.e. the last W tokens including the
+ *                token itself ("Sliding windows and local:global layers");
+ *   decode     : the one query is the sequence's last token and sees all of
+ *                its seq_len keys, gathered page by page through the block
+ *                table ("Paging and prefix sharing").
+ *   A row whose allowed set is empty gets O = 0 and LSE = -inf.
+ *   GQA: query head h reads KV head h / (Hq / Hkv) ("MQA and GQA").
+ *
+ * Split-KV combine ("Flash-Decoding"): partial results over disjoint key
+ * sets are merged with the log-sum-exp rule
+ *   M = max_s lse_s, w_s = exp(lse_s - M), lse = M + log(sum_s w_s),
+ *   O = sum_s w_s O_s / sum_s w_s.
+ *
+ * Inputs are bf16 bit patterns (uint16); each is widened exactly to double.
+ * All sums run in a fixed sequential order, so results do not depend on the
+ * OpenMP thread count.  libm exp/log in double; build without -ffast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 is the upper 16 bits of an IEEE binary32; widening is exact. */
+static double widen(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Is key j (0-based, in the sequence) visible from query i? */
+static int allowed(int64_t i, int64_t j, int causal, int window)
+{
+    if (!causal) return 1;
+    if (j > i) return 0;
+    if (window > 0 && j <= i - window) return 0;
+    return 1;
+}
+
+/*
+ * One output row.  keys[j] / vals[j] point at the d-vector of key / value j;
+ * vis[j] says whether key j is in A(i).  s is scratch of length nkeys.
+ * Writes o[0..d) and *lse; optionally the probability row p[0..nkeys).
+ */
+static void attend_row(const double *q, int d, int64_t nkeys,
+                       const uint16_t *const *keys, const uint16_t *const *vals,
+                       const unsigned char *vis, double scale,
+                       double *s, double *o, double *lse, double *p)
+{
+    int64_t j;
+    int c;
+    double m = -INFINITY, l = 0.0;
+    int any = 0;
+
+    /* 1. scores of the allowed keys */
+    for (j = 0; j < nkeys; ++j) {
+        if (!vis[j]) { s[j] = -INFINITY; continue; }
+        double acc = 0.0;
+        for (c = 0; c < d; ++c) acc += q[c] * widen(keys[j][c]);
+        s[j] = scale * acc;
+        any = 1;
+    }
+    for (c = 0; c < d; ++c) o[c] = 0.0;
+    if (!any) {
+        *lse = -INFINITY;
+        if (p) for (j = 0; j < nkeys; ++j) p[j] = 0.0;
+        return;
+    }
+    /* 2. row max, then the denominator */
+    for (j = 0; j < nkeys; ++j)
+        if (vis[j] && s[j] > m) m = s[j];
+    for (j = 0; j < nkeys; ++j)
+        if (vis[j]) l += exp(s[j] - m);
+    /* 3. probabilities times values */
+    for (j = 0; j < nkeys; ++j) {
+        double pj = vis[j] ? exp(s[j] - m) / l : 0.0;
+        if (p) p[j] = pj;
+        if (!vis[j]) continue;
+        for (c = 0; c < d; ++c) o[c] += pj * widen(vals[j][c]);
+    }
+    /* 4. log-sum-exp */
+    *lse = m + log(l);
+}
+
+/*
+ * Packed-sequence attention, optionally on a subset of query tokens.
+ *   q [total, Hq, d], k/v [total, Hkv, d] (bf16 bits), sequences given by
+ *   cu_seqlens[0..num_seqs] (prefix sums of the lengths).
+ *   rows: global token indices to compute (NULL = all `total` tokens, in order)
+ *   o   [nrows, Hq, d]  lse [nrows, Hq]   (fp64)
+ * Returns 0, or -1 on a bad argument (a row outside every sequence, Hq not a
+ * multiple of Hkv, ...).
+ */
+int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *cu_seqlens, int num_seqs,
+                            int Hq, int Hkv, int d, int causal, int window,
+                            double scale, const int64_t *rows, int64_t nrows,
+                            double *o, double *lse)
+{
+    if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t total = cu_seqlens[num_seqs];
+    if (!rows) nrows = total;
+    int64_t maxlen = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
+        if (L < 0) return -1;
+        if (L > maxlen) maxlen = L;
+    }
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        if (t < 0 || t >= total) return -1;
+    }
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(maxlen > 0 ? maxlen : 1));
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * (size_t)(maxlen > 0 ? maxlen : 1));
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * (size_t)(maxlen > 0 ? maxlen : 1));
+        unsigned char *vis = (unsigned char *)malloc((size_t)(maxlen > 0 ? maxlen : 1));
+        if (!s || !qd || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < nrows * (int64_t)Hq; ++task) {
+                int64_t r = task / Hq;
+                int h = (int)(task % Hq);
+                int64_t t = rows ? rows[r] : r;
+                /* which sequence holds token t */
+                int seq = 0;
+                while (seq < num_seqs && cu_seqlens[seq + 1] <= t) ++seq;
+                int64_t start = cu_seqlens[seq];
+                int64_t L = (int64_t)cu_seqlens[seq + 1] - start;
+                int64_t i = t - start;
+                int g = h / group;
+                for (int c = 0; c < d; ++c)
+                    qd[c] = widen(q[(t * Hq + h) * (int64_t)d + c]);
+                for (int64_t j = 0; j < L; ++j) {
+                    kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
+                    vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
+                    vis[j] = (unsigned char)allowed(i, j, causal, window);
+                }
+                attend_row(qd, d, L, kp, vp, vis, scale, s,
+                           o + (r * Hq + h) * (int64_t)d, lse + r * Hq + h, NULL);
+            }
+        }
+        free(s); free(qd); free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
+
+/* Dense batch: q [B,N,Hq,d], k/v [B,N,Hkv,d]; o [B,N,Hq,d]; lse [B,Hq,N]. */
+int oracle_attn(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                int B, int Hq, int Hkv, int N, int d, int causal, int window,
+                double scale, double *o, double *lse)
+{
+    if (B < 0 || N < 0) return -1;
+    int32_t *cu = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B + 1));
+    double *lse_t = (double *)malloc(sizeof(double) * (size_t)((int64_t)B * N * Hq + 1));
+    if (!cu || !lse_t) { free(cu); free(lse_t); return -2; }
+    for (int b = 0; b <= B; ++b) cu[b] = b * N;
+    int rc = oracle_attn_varlen_rows(q, k, v, cu, B, Hq, Hkv, d, causal, window,
+                                     scale, NULL, 0, o, lse_t);
+    if (rc == 0) {
+        /* token-major [B*N, Hq] -> [B, Hq, N] */
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < Hq; ++h)
+                for (int i = 0; i < N; ++i)
+                    lse[((int64_t)b * Hq + h) * N + i] = lse_t[((int64_t)b * N + i) * Hq + h];
+    }
+    free(cu); free(lse_t);
+    return rc;
+}
+
+/*
+ * The probability matrix of one (sequence, head) -- for invariant checks on
+ * small cases.  p [L, L] for the sequence `seq` of a packed batch.
+ */
+int oracle_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                 const int32_t *cu_seqlens, int num_seqs, int seq, int h,
+                 int Hq, int Hkv, int d, int causal, int window, double scale,
+                 double *p)
+{
+    if (seq < 0 || seq >= num_seqs || h < 0 || h >= Hq || Hq % Hkv) return -1;
+    int64_t start = cu_seqlens[seq], L = (int64_t)cu_seqlens[seq + 1] - start;
+    int g = h / (Hq / Hkv);
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L + 1));
+    double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * (size_t)(L + 1));
+    const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * (size_t)(L + 1));
+    unsigned char *vis = (unsigned char *)malloc((size_t)(L + 1));
+    int rc = (s && qd && o && kp && vp && vis) ? 0 : -2;
+    for (int64_t i = 0; rc == 0 && i < L; ++i) {
+        double lse;
+        for (int c = 0; c < d; ++c) qd[c] = widen(q[((start + i) * Hq + h) * (int64_t)d + c]);
+        for (int64_t j = 0; j < L; ++j) {
+            kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
+            vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
+            vis[j] = (unsigned char)allowed(i, j, causal, window);
+        }
+        attend_row(qd, d, L, kp, vp, vis, scale, s, o, &lse, p + i * L);
+    }
+    free(s); free(qd); free(o); free(kp); free(vp); free(vis);
+    return rc;
+}
+
+/*
+ * Paged decode: one query token per sequence, at position seq_len - 1, seeing
+ * all seq_len cached keys.  Key j of sequence s lives in page
+ * block_table[s * max_pages + j / page_size], slot j % page_size.
+ *   q [S, Hq, d]; k_cache/v_cache [num_pages, page_size, Hkv, d]
+ *   o [S, Hq, d]; lse [S, Hq]
+ */
+int oracle_decode_paged(const uint16_t *q, const uint16_t *k_cache,
+                        const uint16_t *v_cache, const int32_t *block_table,
+                        const int32_t *seq_lens, int S, int Hq, int Hkv, int d,
+                        int page_size, int max_pages, int64_t num_pages,
+                        double scale, double *o, double *lse)
+{
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || page_size <= 0) return -1;
+    int64_t maxlen = 0;
+    for (int s = 0; s < S; ++s) {
+        if (seq_lens[s] < 0 || seq_lens[s] > (int64_t)max_pages * page_size) return -1;
+        if (seq_lens[s] > maxlen) maxlen = seq_lens[s];
+        for (int64_t p = 0; p < ((int64_t)seq_lens[s] + page_size - 1) / page_size; ++p) {
+            int32_t pg = block_table[(int64_t)s * max_pages + p];
+            if (pg < 0 || pg >= num_pages) return -1;
+        }
+    }
+    const int group = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sb = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
+        unsigned char *vis = (unsigned char *)malloc(n);
+        if (!sb || !qd || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < (int64_t)S * Hq; ++task) {
+                int s = (int)(task / Hq), h = (int)(task % Hq), g = h / group;
+                int64_t L = seq_lens[s];
+                for (int c = 0; c < d; ++c) qd[c] = widen(q[((int64_t)s * Hq + h) * d + c]);
+                for (int64_t j = 0; j < L; ++j) {
+                    int64_t pg = block_table[(int64_t)s * max_pages + j / page_size];
+                    int64_t slot = j % page_size;
+                    kp[j] = k_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    vp[j] = v_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    vis[j] = (unsigned char)allowed(L - 1, j, 1, 0);
+                }
+                attend_row(qd, d, L, kp, vp, vis, scale, sb,
+                           o + task * d, lse + task, NULL);
+            }
+        }
+        free(sb); free(qd); free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * Log-sum-exp merge of partial results over disjoint key sets.
+ *   o_parts [nparts, rows, d], lse_parts [nparts, rows] -> o [rows, d], lse [rows]
+ * A part with lse = -inf carries no weight; if every part is -inf the row is
+ * O = 0, LSE = -inf.
+ */
+int oracle_lse_combine(const double *o_parts, const double *lse_parts,
+                       int nparts, int64_t rows, int d, double *o, double *lse)
+{
+    if (nparts < 0 || rows < 0 || d <= 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        double m = -INFINITY, wsum = 0.0;
+        int c, s;
+        for (s = 0; s < nparts; ++s)
+            if (lse_parts[(int64_t)s * rows + r] > m) m = lse_parts[(int64_t)s * rows + r];
+        for (c = 0; c < d; ++c) o[r * d + c] = 0.0;
+        if (m == -INFINITY) { lse[r] = -INFINITY; continue; }
+        for (s = 0; s < nparts; ++s) {
+            double w = exp(lse_parts[(int64_t)s * rows + r] - m);
+            wsum += w;
+            for (c = 0; c < d; ++c) o[r * d + c] += w * o_parts[((int64_t)s * rows + r) * d + c];
+        }
+        for (c = 0; c < d; ++c) o[r * d + c] /= wsum;
+        lse[r] = m + log(wsum);
+    }
+    return 0;
+}
