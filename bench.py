@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * fa_fwd on the 8B-class causal GQA prefill workload (B=1, Hq=32, Hkv=8,
+    N=4096, d=128, bf16, causal) -- the headline metric, attention TFLOP/s
+    with FLOPs = 4*B*Hq*N^2*d / 2 (causal);
+  * fa_decode_paged (split + combine) on 64 sequences with KV lengths
+    uniform in [4096, 32768], 16-token pages under a random permutation --
+    reported beside it as KV GB/s (bytes = sum_s L_s * Hkv * d * 2 B * 2).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Every timed step is preceded by an L2 flush (a 256 MiB write, outside the
+timed events); kernels are timed with CUDA events on the launching stream.
+Under torchrun (N > 1) every rank runs its own independent problem (seed =
+rank): the path shards with no exchange, so the scaling is weak and the
+reported value is the work of all ranks over the slowest rank's time.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+PREFILL = "gqa4k"
+DECODE = "decode64"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "causal bf16 prefill attn TFLOP/s & % tensor peak; decode KV GB/s vs HBM"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    p = dict(FALLBACK_PEAKS)
+    src = "fallback"
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        try:
+            m = json.load(open(path))
+            for k in p:
+                if k in m:
+                    p[k] = float(m[k])
+            src = "measured"
+        except (ValueError, OSError):
+            pass
+    return p, src
+
+
+def prefill_flops(B, Hq, N, d, causal=True, window=0):
+    if window and window < N:
+        pairs = window * (window + 1) // 2 + (N - window) * window
+        return 4.0 * B * Hq * d * pairs
+    return 4.0 * B * Hq * N * N * d / (2.0 if causal else 1.0)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("prefill_sm100.cu", "decode_sm100.cu", "sm100.cuh"):
+        h.update(open(os.path.join(ROOT, "exact_io_aware_75_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, keyed by kernel
+    source hash; None when the kernels changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    want = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[1] == want:
+            out[parts[0]] = float(parts[3])
+    return out
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, interval=0.01):
+        self.index, self.interval = index, interval
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are reported as unknown
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def report(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- CPU oracle leg
+def oracle_sample(inp, target_s, cores):
+    """Time the fp64 oracle on evenly spaced query rows (all heads) of the
+    prefill workload, sized to about target_s seconds.  Returns
+    (TFLOP/s, description, seconds)."""
+    import oracle
+    oracle.set_num_threads(cores)
+    B, N, Hq, d = inp.q.shape
+
+    def run(stride, offset):
+        rows = list(range(offset, N, stride))
+        t0 = time.perf_counter()
+        oracle.attn_rows(inp.q, inp.k, inp.v, [(0, r) for r in rows], True, 0, inp.scale)
+        dt = time.perf_counter() - t0
+        fl = sum(4.0 * Hq * d * (r + 1) for r in rows)
+        return fl, dt, len(rows)
+
+    fl, dt, _ = run(256, 255)                      # probe
+    rate = fl / max(dt, 1e-6)
+    full = prefill_flops(B, Hq, N, d)
+    stride = max(1, int(math.ceil(full / max(rate * target_s, 1.0))))
+    fl, dt, nrows = run(stride, stride - 1)
+    desc = (f"{nrows} query rows (every {stride}th, all {Hq} heads) of the {PREFILL} workload, "
+            f"{fl / 1e9:.1f} GFLOP in {dt:.1f} s")
+    return fl / dt / 1e12, desc, dt
+
+
+# --------------------------------------------------------------------- ours
+def bench_ours(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    import exact_io_aware_75_b200 as fa
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk, pk_src = peaks()
+
+    # ---- inputs (seeded per rank; resident in HBM before timing)
+    cfg = workloads.CONFIGS[PREFILL]
+    pin = workloads.make(PREFILL, seed=args.seed + rank)
+    q, k, v = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev)
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    flops = prefill_flops(B, Hq, N, d, True)
+    din = workloads.make(DECODE, seed=args.seed + rank)
+    dq, dk, dv = din.q.to(dev), din.k_cache.to(dev), din.v_cache.to(dev)
+    dbt, dsl = din.block_table.to(dev), din.seq_lens.to(dev)
+    S, _, Hkv_d, dd = dq.shape[0], None, din.k_cache.shape[2], dq.shape[2]
+    kv_bytes = float(din.seq_lens.sum().item()) * Hkv_d * dd * 2 * 2
+    ws = torch.empty(fa.decode_workspace_bytes(S, dq.shape[1], dd, 16, dbt.shape[1]),
+                     dtype=torch.uint8, device=dev)
+    dout = torch.empty_like(dq)
+    dlse = torch.empty((S, dq.shape[1]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        fa.fwd(q, k, v, True, 0, pin.scale, out=o, lse=lse)
+
+    def decode():
+        fa.decode_paged(dq, dk, dv, dbt, dsl, din.scale, out=dout, lse=dlse, workspace=ws)
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    err = fa.check_device_error()
+    if err:
+        raise RuntimeError(f"device error after warm-up: {fa.status_string(err)}")
+
+    # ---- timed steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            prefill()
+            ev[i][1].record(stream)
+            flush.zero_()
+            ev[i][2].record(stream)
+            decode()
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    p_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    d_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    p_tot, d_tot = sum(p_ms), sum(d_ms)
+    if world > 1:
+        t = torch.tensor([p_tot, d_tot], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        p_tot, d_tot = float(t[0]), float(t[1])
+    err = fa.check_device_error()
+    if err:
+        raise RuntimeError(f"device error in timed region: {fa.status_string(err)}")
+
+    # ---- end to end through the public API with host buffers
+    hq, hk, hv = (t.pin_memory() for t in (pin.q, pin.k, pin.v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq2, dk2, dv2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        dq2.copy_(hq, non_blocking=True)
+        dk2.copy_(hk, non_blocking=True)
+        dv2.copy_(hv, non_blocking=True)
+        fa.fwd(dq2, dk2, dv2, True, 0, pin.scale, out=o, lse=lse)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    # ---- figures
+    K = args.steps
+    p_avg = p_tot / K
+    d_avg = d_tot / K
+    tflops = world * flops / (p_avg * 1e-3) / 1e12
+    kv_gbs = world * kv_bytes / (d_avg * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    ach_tf = flops / (p_avg * 1e-3) / 1e12            # per launch, this rank
+    ach_gb = kv_bytes / (d_avg * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(p_avg + d_avg, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (iid N(0,1) bf16, seeded; no dataset)",
+        "config": {"workload": "gqa4k causal prefill B=1 Hq=32 Hkv=8 N=4096 d=128 + "
+                               "decode64 paged split-KV (64 seqs, KV 4096-32768, 16-token pages)",
+                   "prefill": {"B": B, "Hq": Hq, "Hkv": k.shape[2], "N": N, "d": d,
+                               "causal": True, "flop_per_call": flops},
+                   "decode": {"num_seqs": S, "Hq": dq.shape[1], "Hkv": Hkv_d, "d": dd,
+                              "kv_tokens": int(din.seq_lens.sum()), "kv_bytes": kv_bytes},
+                   "l2": "flushed before every timed kernel (256 MiB write)",
+                   "parallelism": f"{world} independent replica(s), one per GPU"},
+        "roofline": {"bound": "tensor", "achieved": round(ach_tf, 2),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(ach_tf / pk["bf16_tflops"], 4),
+                     "peak_source": f"{pk_src} bf16 burst (cuBLAS)",
+                     "kernel": "prefill_kernel<128>",
+                     "traffic": traffic.get("prefill_gqa4k")},
+        "decode": {"value": round(kv_gbs, 1), "unit": "GB/s", "ms_per_call": round(d_avg, 4),
+                   "roofline": {"bound": "hbm", "achieved": round(ach_gb, 1),
+                                "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                "frac": round(ach_gb / pk["hbm_gbs"], 4),
+                                "peak_source": f"{pk_src} HBM copy",
+                                "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                                "traffic": traffic.get("decode_decode64")}},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4),
+                "what": "fa_fwd through the Python binding: pinned host q,k,v -> device, "
+                        "kernel, O and LSE -> host, per step"},
+        "gpu_launches": 3 * K,
+        "clocks": clk.report(),
+        "wall_s_timed_region": round(t_wall, 3),
+        "kernel_source": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = len(os.sched_getaffinity(0))
+        val, desc, _ = oracle_sample(pin, args.cpu_seconds, cores)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference
+def bench_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    cores = len(os.sched_getaffinity(0))
+    pin = workloads.make(PREFILL, seed=args.seed)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals, descs, secs = [], [], []
+    for i in range(args.warmup + args.steps):
+        val, desc, dt = oracle_sample(pin, per_step, cores)
+        if i >= args.warmup:
+            vals.append(val)
+            descs.append(desc)
+            secs.append(dt)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(secs),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (iid N(0,1) bf16, seeded; no dataset)",
+        "config": {"workload": "gqa4k causal prefill B=1 Hq=32 Hkv=8 N=4096 d=128 "
+                               "(bounded row sample per step)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": descs[-1]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+"""Exact IO-aware attention for B200 (sm_100a): Python binding of libfa_sm100.so.
+
+The binding only marshals arguments: it takes torch CUDA tensors, passes their
+device pointers, sizes and the current CUDA stream to the C ABI declared in
+``include/fa.h``, and raises :class:`FAError` on a non-zero status.  All
+arithmetic runs in the library's kernels.  There is no fallback: if the
+shared library is missing or fails to load, importing this package raises.
+
+Functions mirror the C entry points:
+    fwd            -> fa_fwd            (dense prefill)
+    fwd_varlen     -> fa_fwd_varlen     (packed sequences, cu_seqlens)
+    decode_paged   -> fa_decode_paged   (paged split-KV decode)
+    decode_workspace_bytes, check_device_error, status_string, version
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_sm100.so")
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_ALIGNMENT = -3
+FA_ERR_WORKSPACE = -4
+FA_ERR_CUDA = -5
+FA_ERR_TIMEOUT = -6
+FA_OUT_BF16 = 0
+FA_OUT_FP32 = 1
+
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_workspace_bytes", "fa_decode_paged",
+           "fa_status_string", "fa_check_device_error", "fa_version")
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python exact_io_aware_75_b200/build.py` "
+            "(or __graft_entry__.build()).  There is no fallback path.")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp] + [i] * 7 + [f, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp] + [i] * 8 + [f, i, vp]
+    lib.fa_fwd_varlen.restype = i
+    lib.fa_decode_workspace_bytes.argtypes = [i] * 5
+    lib.fa_decode_workspace_bytes.restype = sz
+    lib.fa_decode_paged.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_decode_paged.restype = i
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_check_device_error.argtypes = [vp]
+    lib.fa_check_device_error.restype = i
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = i
+    return lib
+
+
+_lib = _load()
+
+
+def library():
+    """The loaded ctypes handle (for tests that call the C ABI directly)."""
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.fa_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(_lib.fa_version())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != FA_OK:
+        raise FAError(rc, where)
+
+
+def _need(t, dtype, ndim, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must have {ndim} dims, got {t.dim()}")
+    if not t.is_contiguous():
+        raise FAError(FA_ERR_INVALID_ARG, f"{name} must be contiguous")
+
+
+def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
+        out=None, lse=None, return_lse=True, stream=None):
+    """Dense prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 -> (O [B,N,Hq,d], LSE [B,Hq,N])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, 4, n)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
+        raise FAError(FA_ERR_INVALID_ARG, "k/v shape")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, N, Hq, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    _check(_lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                       int(causal), int(window), float(scale), od, _stream(stream)), "fa_fwd")
+    return out, lse
+
+
+def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=None,
+               out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None):
+    """Packed prefill.  q [T,Hq,d], k/v [T,Hkv,d], cu_seqlens [S+1] int32 (device)
+    -> (O [T,Hq,d], LSE [Hq,T])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, 3, n)
+    _need(cu_seqlens, torch.int32, 1, "cu_seqlens")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    _check(_lib.fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                              _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, int(max_seqlen),
+                              Hq, Hkv, d, int(causal), int(window), float(scale), od,
+                              _stream(stream)), "fa_fwd_varlen")
+    return out, lse
+
+
+def decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq) -> int:
+    return int(_lib.fa_decode_workspace_bytes(int(num_seqs), int(Hq), int(d), int(page_size),
+                                              int(max_pages_per_seq)))
+
+
+def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None, lse=None,
+                 return_lse=True, workspace=None, stream=None):
+    """Paged decode.  q [S,Hq,d], caches [P,ps,Hkv,d], block_table [S,maxp] int32,
+    seq_lens [S] int32 -> (O [S,Hq,d] bf16, LSE [S,Hq])."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    S, Hq, d = q.shape
+    P, ps, Hkv, _ = k_cache.shape
+    maxp = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = decode_workspace_bytes(S, Hq, d, ps, maxp)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(_lib.fa_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                _ptr(seq_lens), _ptr(out), _ptr(lse), S, P, Hq, Hkv, d, ps,
+                                maxp, float(scale), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
+                                _stream(stream)), "fa_decode_paged")
+    return out, lse
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status."""
+    return int(_lib.fa_check_device_error(_stream(stream)))

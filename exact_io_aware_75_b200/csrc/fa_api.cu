@@ -1,0 +1,219 @@
+// fa_api.cu -- the C ABI (include/fa.h): argument checks, launch set-up,
+// status strings and the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+int device_sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    if (dev >= 0 && dev < 64) {
+        int v = cached[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 1;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n < 1) n = 1;
+    if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t dim0,
+                         uint64_t dim1, uint64_t dim2, uint64_t stride1_bytes,
+                         uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
+                         bool swizzle128) {
+    auto fn = encode_fn();
+    if (!fn || elem_bytes != 2) return -1;
+    cuuint64_t dims[3] = {dim0, dim1, dim2};
+    cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    cuuint32_t box[3] = {box0, box1, box2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+}  // namespace fa
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int map_rc(int rc) {
+    switch (rc) {
+    case 0: return FA_OK;
+    case -2: return FA_ERR_UNSUPPORTED;
+    case -4: return FA_ERR_WORKSPACE;
+    default: return FA_ERR_CUDA;
+    }
+}
+
+int check_common(int Hq, int Hkv, int d, int causal, int window, float scale, int o_dtype) {
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (o_dtype != FA_OUT_BF16 && o_dtype != FA_OUT_FP32) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (window > 0 && !causal) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int N, int d, int causal, int window, float scale, int o_dtype,
+           void *stream) {
+    if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
+    if (rc) return rc;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+    if ((long long)B * N > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return FA_ERR_ALIGNMENT;
+    fa::PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.cu_seqlens = nullptr;
+    a.num_seqs = B;
+    a.seqlen = N;
+    a.total_tokens = B * N;
+    a.max_seqlen = N;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.o_fp32 = o_dtype == FA_OUT_FP32;
+    return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
+                  int Hq, int Hkv, int d, int causal, int window, float scale, int o_dtype,
+                  void *stream) {
+    if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
+    if (rc) return rc;
+    if (num_seqs == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
+    if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return FA_ERR_ALIGNMENT;
+    fa::PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.cu_seqlens = cu_seqlens;
+    a.num_seqs = num_seqs;
+    a.seqlen = 0;
+    a.total_tokens = total_tokens;
+    a.max_seqlen = max_seqlen;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.o_fp32 = o_dtype == FA_OUT_FP32;
+    return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size,
+                                 int max_pages_per_seq) {
+    return fa::decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq);
+}
+
+int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
+                    const int *block_table, const int *seq_lens, void *o, float *lse,
+                    int num_seqs, int num_pages, int Hq, int Hkv, int d, int page_size,
+                    int max_pages_per_seq, float scale, void *workspace, size_t workspace_bytes,
+                    void *stream) {
+    if (num_seqs < 0 || num_pages < 0 || max_pages_per_seq <= 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, 0, 0, scale, FA_OUT_BF16);
+    if (rc) return rc;
+    if (page_size != 16) return FA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return FA_OK;
+    if (num_pages == 0) return FA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !o) return FA_ERR_INVALID_ARG;
+    if ((long long)num_pages * page_size > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return FA_ERR_ALIGNMENT;
+    const size_t need = fa::decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq);
+    if (need == 0) return FA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FA_ERR_ALIGNMENT;
+    fa::DecodeArgs a{};
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+    a.block_table = block_table; a.seq_lens = seq_lens;
+    a.o = o; a.lse = lse;
+    a.num_seqs = num_seqs; a.num_pages = num_pages;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d; a.page_size = page_size;
+    a.max_pages = max_pages_per_seq;
+    a.scale = scale;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    return map_rc(fa::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+const char *fa_status_string(int status) {
+    switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_ALIGNMENT: return "pointer not aligned";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA runtime error";
+    case FA_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int fa_check_device_error(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    int word = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, fa::g_device_error, sizeof word) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (word && cudaMemcpyToSymbol(fa::g_device_error, &zero, sizeof zero) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (word == fa::kDevErrTimeout) return FA_ERR_TIMEOUT;
+    if (word == fa::kDevErrInput) return FA_ERR_INVALID_ARG;
+    return word ? FA_ERR_CUDA : FA_OK;
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

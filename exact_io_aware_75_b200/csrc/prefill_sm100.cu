@@ -1,0 +1,547 @@
+// prefill_sm100.cu -- exact attention prefill on the sm_100a tensor core.
+//
+// What it computes: O = softmax(Q K^T * scale + mask) V and the row
+// log-sum-exp, for dense batches and packed sequences, with causal and
+// sliding-window masks and grouped KV heads ("What attention costs",
+// "MQA and GQA", "Sliding windows and local:global layers" in samanvya.dev's
+// "Attention Is the Bottleneck").
+//
+// How (the tiled online softmax of "FlashAttention: same math, different
+// IO", arranged for B200):
+//   * Persistent grid, one CTA per SM.  A work unit is 256 query rows of one
+//     (sequence, query head), split into two 128-row tiles that ping-pong:
+//     while the tensor core runs one tile's GEMMs, the other tile's softmax
+//     warpgroup works ("FlashAttention-3": warp specialisation, ping-pong).
+//     Units run heaviest first (causal: last row blocks first).
+//   * Warp 8 issues TMA loads: the two Q tiles once per unit, then K_j, V_j
+//     tiles (128 keys x d) into a ring of shared-memory slots, 128-byte
+//     swizzled.  Only key blocks that some visible (row, key) pair needs are
+//     loaded: causal and window masks skip whole tiles.
+//   * Warp 9 (one thread) issues tcgen05 MMAs: S_t = Q_t K_j^T into tensor
+//     memory (fp32), then O_t += P_t V_j with P_t read from tensor memory
+//     where the softmax left it (bf16, aliasing S_t) -- "FlashAttention-4":
+//     tensor memory takes operand traffic off shared memory.
+//   * Warps 0-3 / 4-7: one thread per query row.  Each reads its S row from
+//     TMEM, applies scale and mask, updates the running max m and sum l,
+//     writes P = 2^(s*scale*log2e - m) back as bf16, and signals the MMA
+//     warp.  The rescale of O by 2^(m_old - m_new) is skipped unless the max
+//     grew by more than 8 (log2 units) in some row of the warp
+//     ("FlashAttention-4": conditional rescaling); P is then at most 2^8,
+//     and O and l stay consistent because both use the same reference max.
+//   * The epilogue divides O by l once ("FlashAttention-2": delayed
+//     normalisation) and writes O and LSE = ln2 * (m + log2 l).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+namespace prefill_impl {
+
+constexpr int kBlockM = 128;        // rows per tile (TMEM lanes)
+constexpr int kBlockN = 128;        // keys per K/V tile
+constexpr int kThreads = 320;       // 8 softmax warps + TMA warp + MMA warp
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+    static constexpr int kBoxBytes = kBlockM * 64 * 2;             // 128 rows x 64 bf16
+    static constexpr int kTileBytes = kBlockM * D * 2;             // Q tile or K/V tile
+    static constexpr int kStages = (D == 128) ? 5 : 6;             // K/V ring slots
+    static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + 1024;
+    static constexpr uint32_t kColO = 256;                         // O_t at 256 + t*D
+};
+
+struct Params {
+    void *o;
+    float *lse;
+    const int *cu_seqlens;
+    int num_seqs, seqlen, total_tokens, max_seqlen;
+    int Hq, Hkv, group;
+    int causal, window;
+    float scale_log2;
+    int o_fp32;
+    int num_mblocks;   // 256-row blocks per sequence (of max_seqlen)
+    int num_units;
+};
+
+struct Unit {
+    int seq, h, kvh;
+    int tok0;   // packed index of the sequence's first token
+    int L;      // sequence length
+    int q0;     // first query row of the unit, local to the sequence
+    int lo[2], hi[2];  // key-block range per tile, [lo, hi)
+    int lo_all, hi_all;
+};
+
+__device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
+    const int per_mb = p.num_seqs * p.Hq;
+    const int mb = p.num_mblocks - 1 - u / per_mb;
+    const int r = u % per_mb;
+    w.seq = r / p.Hq;
+    w.h = r % p.Hq;
+    w.kvh = w.h / p.group;
+    if (p.cu_seqlens) {
+        w.tok0 = __ldg(p.cu_seqlens + w.seq);
+        w.L = __ldg(p.cu_seqlens + w.seq + 1) - w.tok0;
+    } else {
+        w.tok0 = w.seq * p.seqlen;
+        w.L = p.seqlen;
+    }
+    w.q0 = mb * 2 * kBlockM;
+    if (w.L <= 0 || w.q0 >= w.L) return false;
+    const int nkb = (w.L + kBlockN - 1) / kBlockN;
+    w.lo_all = 1 << 30;
+    w.hi_all = 0;
+    for (int t = 0; t < 2; ++t) {
+        const int r0 = w.q0 + t * kBlockM;
+        if (r0 >= w.L) { w.lo[t] = w.hi[t] = 0; continue; }
+        int lo = 0, hi = nkb;
+        if (p.causal) {
+            const int last = min(r0 + kBlockM - 1, w.L - 1);
+            hi = min(nkb, last / kBlockN + 1);
+            if (p.window > 0) lo = max(0, r0 - p.window + 1) / kBlockN;
+        }
+        w.lo[t] = lo;
+        w.hi[t] = hi;
+        w.lo_all = min(w.lo_all, lo);
+        w.hi_all = max(w.hi_all, hi);
+    }
+    return true;
+}
+
+struct Shared {
+    uint64_t q_full[2], q_empty[2];
+    uint64_t kv_full[8], kv_empty[8];
+    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ------------------------------------------------------------- TMA producer
+template <int D>
+__device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                         const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
+    using C = Cfg<D>;
+    volatile int *abort = &sh.abort;
+    uint32_t q_uses[2] = {0, 0};
+    uint32_t kv_it = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        for (int t = 0; t < 2; ++t) {
+            if (w.lo[t] >= w.hi[t]) continue;
+            if (!mbar_wait(&sh.q_empty[t], (q_uses[t] & 1) ^ 1, abort)) goto out;
+            mbar_arrive_expect_tx(&sh.q_full[t], C::kTileBytes);
+            for (int b = 0; b < D / 64; ++b)
+                tma_load_3d(sQ + t * C::kTileBytes + b * C::kBoxBytes, tmQ, &sh.q_full[t],
+                            b * 64, w.h, w.tok0 + w.q0 + t * kBlockM);
+            ++q_uses[t];
+        }
+        for (int j = w.lo_all; j < w.hi_all; ++j) {
+            for (int kv = 0; kv < 2; ++kv) {
+                const int slot = kv_it % C::kStages;
+                const uint32_t use = kv_it / C::kStages;
+                if (!mbar_wait(&sh.kv_empty[slot], (use & 1) ^ 1, abort)) goto out;
+                mbar_arrive_expect_tx(&sh.kv_full[slot], C::kTileBytes);
+                for (int b = 0; b < D / 64; ++b)
+                    tma_load_3d(sKV + slot * C::kTileBytes + b * C::kBoxBytes, kv ? tmV : tmK,
+                                &sh.kv_full[slot], b * 64, w.kvh, w.tok0 + j * kBlockN);
+                ++kv_it;
+            }
+        }
+    }
+    return;
+out:
+    // Leave no copy in flight: wait for the last load issued into each slot.
+    for (int s = 0; s < C::kStages; ++s) {
+        if (kv_it > (uint32_t)s) {
+            const uint32_t last = (kv_it - 1 - s) / C::kStages;
+            mbar_drain_wait(&sh.kv_full[s], last & 1);
+        }
+    }
+    for (int t = 0; t < 2; ++t)
+        if (q_uses[t]) mbar_drain_wait(&sh.q_full[t], (q_uses[t] - 1) & 1);
+}
+
+// ------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
+    using C = Cfg<D>;
+    volatile int *abort = &sh.abort;
+    const uint32_t tmem = sh.tmem_base;
+    const uint32_t idS = idesc_bf16_f32(kBlockM, kBlockN, false);
+    const uint32_t idPV = idesc_bf16_f32(kBlockM, D, true);
+    const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
+    uint32_t q_uses[2] = {0, 0}, p_cnt[2] = {0, 0}, oe_uses[2] = {0, 0};
+    uint32_t kv_it = 0;
+
+    // S_t = Q_t K^T: d/16 MMAs of K=16; K-major, 128-byte swizzle, atoms of
+    // 8 rows x 128 bytes (SBO 1024), 64 columns per TMA box.
+    auto issue_s = [&](int t, int kslot) {
+        const uint32_t qa = q_addr + t * C::kTileBytes;
+        const uint32_t ka = kv_addr + kslot * C::kTileBytes;
+        #pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * C::kBoxBytes + (ks & 3) * 32;
+            mma_ss(tmem + t * kBlockN, smem_desc_sw128(qa + off, 16, 1024),
+                   smem_desc_sw128(ka + off, 16, 1024), idS, ks > 0);
+        }
+    };
+    // O_t += P_t V: 128/16 MMAs of K=16 keys; V is MN-major (d contiguous):
+    // 16 keys = two 8-row groups (SBO 1024), d split in 64-column boxes (LBO).
+    auto issue_pv = [&](int t, int vslot, bool first) {
+        const uint32_t va = kv_addr + vslot * C::kTileBytes;
+        #pragma unroll
+        for (int ks = 0; ks < kBlockN / 16; ++ks) {
+            mma_ts(tmem + C::kColO + t * D, tmem + t * kBlockN + ks * 8,
+                   smem_desc_sw128(va + ks * 2048, C::kBoxBytes, 1024), idPV,
+                   (ks > 0 || !first) ? 1u : 0u);
+        }
+    };
+
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        bool first_pv[2] = {true, true};
+        for (int t = 0; t < 2; ++t) {
+            if (w.lo[t] >= w.hi[t]) continue;
+            if (!mbar_wait(&sh.q_full[t], q_uses[t] & 1, abort)) goto out;
+            ++q_uses[t];
+        }
+        tc_fence_after();
+        int prev_v = -1;
+        for (int j = w.lo_all; j < w.hi_all; ++j) {
+            const bool in0 = j >= w.lo[0] && j < w.hi[0];
+            const bool in1 = j >= w.lo[1] && j < w.hi[1];
+            const bool prev1 = (j - 1) >= w.lo[1] && (j - 1) < w.hi[1];
+            const int kslot = kv_it % C::kStages;
+            if (!mbar_wait(&sh.kv_full[kslot], (kv_it / C::kStages) & 1, abort)) goto out;
+            ++kv_it;
+            const int vslot = kv_it % C::kStages;
+            const uint32_t vuse = kv_it / C::kStages;
+            ++kv_it;
+            tc_fence_after();
+            if (in0) {
+                issue_s(0, kslot);
+                tc_commit(&sh.s_full[0]);
+            }
+            if (prev1) {
+                if (!mbar_wait(&sh.p_full[1], p_cnt[1] & 1, abort)) goto out;
+                ++p_cnt[1];
+                if (first_pv[1]) {
+                    if (!mbar_wait(&sh.o_empty[1], (oe_uses[1] & 1) ^ 1, abort)) goto out;
+                    ++oe_uses[1];
+                }
+                tc_fence_after();
+                issue_pv(1, prev_v, first_pv[1]);
+                first_pv[1] = false;
+                tc_commit(&sh.o_full[1]);
+                tc_commit(&sh.kv_empty[prev_v]);
+            }
+            if (in1) {
+                issue_s(1, kslot);
+                tc_commit(&sh.s_full[1]);
+            }
+            tc_commit(&sh.kv_empty[kslot]);
+            if (in0 && j == w.hi[0] - 1) tc_commit(&sh.q_empty[0]);
+            if (in1 && j == w.hi[1] - 1) tc_commit(&sh.q_empty[1]);
+            if (!mbar_wait(&sh.kv_full[vslot], vuse & 1, abort)) goto out;
+            tc_fence_after();
+            if (in0) {
+                if (!mbar_wait(&sh.p_full[0], p_cnt[0] & 1, abort)) goto out;
+                ++p_cnt[0];
+                if (first_pv[0]) {
+                    if (!mbar_wait(&sh.o_empty[0], (oe_uses[0] & 1) ^ 1, abort)) goto out;
+                    ++oe_uses[0];
+                }
+                tc_fence_after();
+                issue_pv(0, vslot, first_pv[0]);
+                first_pv[0] = false;
+                tc_commit(&sh.o_full[0]);
+            }
+            if (!in1) tc_commit(&sh.kv_empty[vslot]);
+            prev_v = vslot;
+        }
+        if ((w.hi_all - 1) >= w.lo[1] && (w.hi_all - 1) < w.hi[1]) {
+            if (!mbar_wait(&sh.p_full[1], p_cnt[1] & 1, abort)) goto out;
+            ++p_cnt[1];
+            if (first_pv[1]) {
+                if (!mbar_wait(&sh.o_empty[1], (oe_uses[1] & 1) ^ 1, abort)) goto out;
+                ++oe_uses[1];
+            }
+            tc_fence_after();
+            issue_pv(1, prev_v, first_pv[1]);
+            tc_commit(&sh.o_full[1]);
+            tc_commit(&sh.kv_empty[prev_v]);
+        }
+    }
+out:
+    // Wait for every MMA this thread issued before TMEM is released.
+    tc_commit(&sh.drain);
+    mbar_drain_wait(&sh.drain, 0);
+}
+
+// ---------------------------------------------------------------- softmax
+template <int D>
+__device__ void softmax_wg(const Params &p, Shared &sh) {
+    using C = Cfg<D>;
+    volatile int *abort = &sh.abort;
+    const int warp = warp_id(), lane = lane_id();
+    const int t = warp >> 2;                 // tile of this warpgroup
+    const int r = (warp & 3) * 32 + lane;    // row within the tile
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = sh.tmem_base + lanes + t * kBlockN;
+    const uint32_t tO = sh.tmem_base + lanes + C::kColO + t * D;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, pv_cnt = 0;
+
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        const int lo = w.lo[t], hi = w.hi[t];
+        if (lo >= hi) continue;
+        const int row = w.q0 + t * kBlockM + r;    // row index within the sequence
+        const int rmin = w.q0 + t * kBlockM, rmax = rmin + kBlockM - 1;
+        float m_ref = -INFINITY, l = 0.f;
+        for (int j = lo; j < hi; ++j) {
+            if (!mbar_wait_warp(&sh.s_full[t], s_cnt & 1, abort)) return;
+            ++s_cnt;
+            tc_fence_after();
+            float s[kBlockN];
+            {
+                uint32_t raw[kBlockN];
+                tmem_ld32(tS + 0, raw);
+                tmem_ld32(tS + 32, raw + 32);
+                tmem_ld32(tS + 64, raw + 64);
+                tmem_ld32(tS + 96, raw + 96);
+                tmem_wait_ld();
+                #pragma unroll
+                for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(raw[c]);
+            }
+            const int k0 = j * kBlockN;
+            const bool edge = (k0 + kBlockN > w.L) || (p.causal && k0 + kBlockN - 1 > rmin) ||
+                              (p.window > 0 && k0 <= rmax - p.window);
+            if (edge) {
+                // visible keys of this row in the tile: c in [c_lo, c_hi)
+                int c_hi = w.L - k0;
+                if (p.causal) c_hi = min(c_hi, row + 1 - k0);
+                const int c_lo = (p.window > 0) ? row - p.window + 1 - k0 : 0;
+                #pragma unroll
+                for (int c = 0; c < kBlockN; ++c)
+                    if (c >= c_hi || c < c_lo) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+            #pragma unroll
+            for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_blk = mx * sl2;
+            if (j == lo) {
+                m_ref = m_blk;
+            } else {
+                const bool need = m_blk > m_ref + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = fmaxf(m_ref, m_blk);
+                    const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);
+                    // O_t holds P V of the previous block only once that MMA is done.
+                    if (!mbar_wait_warp(&sh.o_full[t], (pv_cnt - 1) & 1, abort)) return;
+                    tc_fence_after();
+                    // 16 columns at a time: the 128 scores of the row stay live
+                    #pragma unroll 1
+                    for (int c = 0; c < D; c += 16) {
+                        uint32_t ov[16];
+                        tmem_ld16(tO + c, ov);
+                        tmem_wait_ld();
+                        #pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+                        tmem_st16(tO + c, ov);
+                    }
+                    tmem_wait_st();
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+            }
+            const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+            float sum0 = 0.f, sum1 = 0.f;
+            #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+                #pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, -mb));
+                    const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, -mb));
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                tmem_st32(tS + 32 * h, pk);
+            }
+            l += sum0 + sum1;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[t]);
+            ++pv_cnt;
+        }
+        // ---- epilogue: O / l, LSE
+        if (!mbar_wait_warp(&sh.o_full[t], (pv_cnt - 1) & 1, abort)) return;
+        tc_fence_after();
+        const bool valid = row < w.L;
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const size_t orow = ((size_t)(w.tok0 + row) * p.Hq + w.h) * D;
+        #pragma unroll
+        for (int c = 0; c < D; c += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c, ov);
+            tmem_wait_ld();
+            if (valid) {
+                if (p.o_fp32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.o) + orow + c);
+                    #pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 2]) * inv_l,
+                                             __uint_as_float(ov[4 * e + 3]) * inv_l);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.o) + orow + c);
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+                        v.y = pack_bf16(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+                        v.z = pack_bf16(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+                        v.w = pack_bf16(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+                        dst[e] = v;
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.o_empty[t]);
+        if (valid && p.lse) {
+            const float lse2 = (l > 0.f) ? m_ref + __log2f(l) : -INFINITY;
+            size_t idx;
+            if (p.cu_seqlens)
+                idx = (size_t)w.h * p.total_tokens + w.tok0 + row;
+            else
+                idx = ((size_t)w.seq * p.Hq + w.h) * p.seqlen + row;
+            p.lse[idx] = lse2 * 0.69314718055994531f;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Shared sh;
+    const uint32_t base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (base & 1023)) & 1023);
+    uint8_t *sQ = smem;
+    uint8_t *sKV = smem + 2 * C::kTileBytes;
+    const int warp = warp_id();
+
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&sh.q_full[t], 1);
+            mbar_init(&sh.q_empty[t], 1);
+            mbar_init(&sh.s_full[t], 1);
+            mbar_init(&sh.p_full[t], 4);
+            mbar_init(&sh.o_full[t], 1);
+            mbar_init(&sh.o_empty[t], 4);
+        }
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&sh.kv_full[s], 1);
+            mbar_init(&sh.kv_empty[s], 1);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) tmem_alloc(&sh.tmem_base, kTmemCols);
+    if (warp == kWarpTma && lane_id() == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp < 8) {
+        softmax_wg<D>(p, sh);
+    } else if (warp == kWarpTma) {
+        if (lane_id() == 0) producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+    } else {
+        if (lane_id() == 0) mma_issuer<D>(p, sh, sQ, sKV);
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(sh.tmem_base, kTmemCols);
+    }
+}
+
+template <int D>
+int launch_d(const PrefillArgs &a, cudaStream_t stream) {
+    using C = Cfg<D>;
+    alignas(64) CUtensorMap tq, tk, tv;
+    const uint64_t T = (uint64_t)a.total_tokens;
+    if (encode_tensor_map_3d(&tq, a.q, 2, D, a.Hq, T, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2,
+                             64, 1, kBlockM, true) ||
+        encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kBlockN, true) ||
+        encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kBlockN, true))
+        return -5;
+    Params p;
+    p.o = a.o;
+    p.lse = a.lse;
+    p.cu_seqlens = a.cu_seqlens;
+    p.num_seqs = a.num_seqs;
+    p.seqlen = a.seqlen;
+    p.total_tokens = a.total_tokens;
+    p.max_seqlen = a.max_seqlen;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.group = a.Hq / a.Hkv;
+    p.causal = a.causal;
+    p.window = a.causal ? a.window : 0;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.o_fp32 = a.o_fp32;
+    p.num_mblocks = (a.max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM);
+    const long long units = (long long)p.num_mblocks * a.num_seqs * a.Hq;
+    if (units <= 0) return 0;
+    if (units > (1ll << 30)) return -2;
+    p.num_units = (int)units;
+    // Setting the attribute is idempotent and cheap; do it on every call so
+    // that any device the caller switches to is covered.
+    if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+        return -5;
+    const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
+    prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+}  // namespace prefill_impl
+
+int launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
+    if (a.d == 128) return prefill_impl::launch_d<128>(a, stream);
+    if (a.d == 64) return prefill_impl::launch_d<64>(a, stream);
+    return -2;
+}
+
+}  // namespace fa

@@ -1,0 +1,154 @@
+/*
+ * fa.h -- exact IO-aware attention for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Every call computes exact scaled-dot-product attention
+ *
+ *     O = softmax(Q K^T * scale + mask) V ,    LSE = log sum_j exp(s_ij)
+ *
+ * ("What attention costs", samanvya.dev "Attention Is the Bottleneck": the
+ * one-line definition softmax(QK^T/sqrt d)V, with 1/sqrt(d) generalised to
+ * `scale` and an additive mask that is 0 on the allowed keys and -inf
+ * elsewhere), tile by tile with an online softmax so the N x N score matrix
+ * never reaches device memory ("FlashAttention: same math, different IO").
+ * Results equal the plain definition up to floating-point rounding order.
+ *
+ * Conventions shared by every call
+ *   - q, k, v, o, caches: bf16 (o optionally fp32), innermost dimension
+ *     contiguous, token-major:  dense [B, N, H, d], packed [total, H, d],
+ *     cache [num_pages, page_size, Hkv, d].
+ *   - GQA ("MQA and GQA"): query head h reads KV head h / (Hq / Hkv);
+ *     Hq must be a multiple of Hkv; Hkv == 1 is MQA.
+ *   - Masks: causal (key j visible from query i iff j <= i; "every token can
+ *     see every earlier token"), sliding window W > 0 (with causal only: keys
+ *     i-W+1 .. i, i.e. the last W tokens including the query itself;
+ *     "Sliding windows and local:global layers").  window <= 0: no window.
+ *   - LSE is natural-log, in units of scaled scores; a row with no visible
+ *     key (only possible for an empty sequence) has O = 0 and LSE = -inf.
+ *   - head dim d in {64, 128}.
+ *   - Every device pointer must be 16-byte aligned (TMA requirement);
+ *     row strides are implied by the shapes.
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     device memory, keeps no per-call state, and is thread-safe.  All calls
+ *     are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and do not synchronise.
+ *   - Errors: the return value is FA_OK (0) or a negative FA_ERR_* code.  On
+ *     an argument error nothing is launched.  FA_ERR_CUDA reports a launch
+ *     error (cudaGetLastError).  There is no CPU fallback: host pointers are
+ *     not detected and passing them is undefined behaviour.
+ *   - Device-side watchdog: every wait inside a kernel is bounded (about a
+ *     second).  A wait that runs out records an error word and the kernel
+ *     returns early; fa_check_device_error() reads and clears that word.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = -1,  /* null pointer, bad shape, Hq % Hkv != 0, ... */
+    FA_ERR_UNSUPPORTED = -2,  /* valid but not implemented: d, page size, window without causal */
+    FA_ERR_ALIGNMENT = -3,    /* a pointer is not 16-byte aligned */
+    FA_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required */
+    FA_ERR_CUDA = -5,         /* the CUDA runtime reported an error */
+    FA_ERR_TIMEOUT = -6       /* a device-side wait ran out (fa_check_device_error) */
+};
+
+enum fa_out_dtype { FA_OUT_BF16 = 0, FA_OUT_FP32 = 1 };
+
+/*
+ * Dense prefill ("FlashAttention: same math, different IO": a Q tile stays
+ * on chip while K/V tiles stream past it; "FlashAttention-2": parallel over
+ * sequence blocks too, normalise once at the end; "FlashAttention-4":
+ * conditional rescaling, tensor memory).
+ *   q      [B, N, Hq, d]  bf16, device
+ *   k, v   [B, N, Hkv, d] bf16, device
+ *   o      [B, N, Hq, d]  bf16 (o_dtype = FA_OUT_BF16) or fp32, device, written
+ *   lse    [B, Hq, N]     fp32, device, written; may be NULL
+ *   causal 0/1; window as above (requires causal); scale > 0 finite.
+ * N == 0 or B == 0 is a no-op returning FA_OK.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int Hq, int Hkv, int N, int d, int causal, int window,
+           float scale, int o_dtype, void *stream);
+
+/*
+ * Packed variable-length prefill: num_seqs sequences concatenated along the
+ * token axis; each sequence attends only to itself (a document mask,
+ * "FlexAttention" on the Ales Analytics kernels page).
+ *   q          [total_tokens, Hq, d]  bf16, device
+ *   k, v       [total_tokens, Hkv, d] bf16, device
+ *   o          [total_tokens, Hq, d]  bf16 or fp32, device, written
+ *   lse        [Hq, total_tokens]     fp32, device, written; may be NULL
+ *   cu_seqlens [num_seqs + 1] int32, device: 0 = cu[0] <= cu[1] <= ... =
+ *              total_tokens (prefix sums of the lengths).  Empty sequences are
+ *              allowed and write nothing.
+ *   max_seqlen >= every sequence length (sizes the launch).  A longer sequence
+ *              is reported through fa_check_device_error (FA_ERR_INVALID_ARG)
+ *              and its rows past max_seqlen are left unwritten.
+ */
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int num_seqs, int total_tokens,
+                  int max_seqlen, int Hq, int Hkv, int d, int causal, int window,
+                  float scale, int o_dtype, void *stream);
+
+/*
+ * Bytes of workspace fa_decode_paged needs for these sizes (split-KV
+ * partial outputs and their log-sum-exps).  0 for an invalid combination.
+ */
+size_t fa_decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size,
+                                 int max_pages_per_seq);
+
+/*
+ * Paged split-KV decode: one query token per sequence, at position
+ * seq_len - 1, attending to all seq_len cached keys ("Flash-Decoding": split
+ * the cache along the sequence, attend to the chunks in parallel, merge the
+ * partial results with log-sum-exp; "Paging and prefix sharing": the cache
+ * lives in fixed-size pages reached through a block table).
+ *   q           [num_seqs, Hq, d] bf16, device
+ *   k_cache,
+ *   v_cache     [num_pages, page_size, Hkv, d] bf16, device
+ *   block_table [num_seqs, max_pages_per_seq] int32, device; entry p of
+ *               sequence s is the page holding its tokens p*page_size ..
+ *               p*page_size + page_size-1; entries past ceil(seq_len /
+ *               page_size) are never read.  Every read entry must lie in
+ *               [0, num_pages).
+ *   seq_lens    [num_seqs] int32, device; 0 <= seq_len <= max_pages_per_seq *
+ *               page_size.  Cache slots past seq_len are never used in the
+ *               result (they may hold anything, NaN included).
+ *   o           [num_seqs, Hq, d] bf16, device, written
+ *   lse         [num_seqs, Hq] fp32, device, written; may be NULL
+ *   workspace   device scratch of at least fa_decode_workspace_bytes(...)
+ *               bytes, 256-byte aligned; contents on entry do not matter;
+ *               it must not be shared by calls that may overlap on the GPU.
+ *   page_size   16 (others return FA_ERR_UNSUPPORTED).
+ */
+int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
+                    const int *block_table, const int *seq_lens, void *o,
+                    float *lse, int num_seqs, int num_pages, int Hq, int Hkv,
+                    int d, int page_size, int max_pages_per_seq, float scale,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable text of a status code (static storage). */
+const char *fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word that a
+ * kernel sets when one of its bounded waits runs out or it meets an input it
+ * cannot honour.  Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_INVALID_ARG or
+ * FA_ERR_CUDA.
+ */
+int fa_check_device_error(void *stream);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */
