@@ -53,6 +53,13 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    # profiling aids (the default run times both kernels on the named workloads)
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="time one kernel family only (for profiler captures)")
+    ap.add_argument("--prefill-workload", default=PREFILL,
+                    choices=["gqa4k", "long32k", "long32k_w4096"])
+    ap.add_argument("--decode-seqs", type=int, default=64,
+                    help="number of decode sequences (64 = the decode64 workload)")
     return ap.parse_args()
 
 
@@ -62,6 +69,22 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (one all_reduce);
+    identity when torch.distributed is not initialised."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own independent problem."""
+    return int(base) + int(rank)
 
 
 def peaks():
@@ -116,7 +139,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index, interval=0.01):
+    def __init__(self, index, interval=0.002):
         self.index, self.interval = index, interval
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -163,7 +186,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle leg
-def oracle_sample(inp, target_s, cores):
+def oracle_sample(inp, target_s, cores, name=PREFILL):
     """Time the fp64 oracle on evenly spaced query rows (all heads) of the
     prefill workload, sized to about target_s seconds.  Returns
     (TFLOP/s, description, seconds)."""
@@ -174,17 +197,19 @@ def oracle_sample(inp, target_s, cores):
     def run(stride, offset):
         rows = list(range(offset, N, stride))
         t0 = time.perf_counter()
-        oracle.attn_rows(inp.q, inp.k, inp.v, [(0, r) for r in rows], True, 0, inp.scale)
+        oracle.attn_rows(inp.q, inp.k, inp.v, [(0, r) for r in rows], True, inp.window,
+                         inp.scale)
         dt = time.perf_counter() - t0
-        fl = sum(4.0 * Hq * d * (r + 1) for r in rows)
+        W = inp.window if inp.window else N + 1
+        fl = sum(4.0 * Hq * d * min(r + 1, W) for r in rows)
         return fl, dt, len(rows)
 
     fl, dt, _ = run(256, 255)                      # probe
     rate = fl / max(dt, 1e-6)
-    full = prefill_flops(B, Hq, N, d)
+    full = prefill_flops(B, Hq, N, d, True, inp.window)
     stride = max(1, int(math.ceil(full / max(rate * target_s, 1.0))))
     fl, dt, nrows = run(stride, stride - 1)
-    desc = (f"{nrows} query rows (every {stride}th, all {Hq} heads) of the {PREFILL} workload, "
+    desc = (f"{nrows} query rows (every {stride}th, all {Hq} heads) of the {name} workload, "
             f"{fl / 1e9:.1f} GFLOP in {dt:.1f} s")
     return fl / dt / 1e12, desc, dt
 
@@ -205,14 +230,21 @@ def bench_ours(args):
     pk, pk_src = peaks()
 
     # ---- inputs (seeded per rank; resident in HBM before timing)
-    cfg = workloads.CONFIGS[PREFILL]
-    pin = workloads.make(PREFILL, seed=args.seed + rank)
+    do_p = args.only in ("all", "prefill")
+    do_d = args.only in ("all", "decode")
+    pname = args.prefill_workload
+    seed = rank_seed(args.seed, rank)
+    pin = workloads.make(pname, seed=seed)
+    if not do_p:   # keep shapes for reporting, skip the device copies
+        pin = workloads.dense(1, 32, 8, 128, 128, causal=True, seed=seed)
     q, k, v = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev)
     B, N, Hq, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
-    flops = prefill_flops(B, Hq, N, d, True)
-    din = workloads.make(DECODE, seed=args.seed + rank)
+    flops = prefill_flops(B, Hq, N, d, True, pin.window)
+    din = workloads.make(DECODE, seed=seed,
+                         num_seqs=args.decode_seqs if do_d else 1,
+                         **({} if do_d else {"len_lo": 16, "len_hi": 16}))
     dq, dk, dv = din.q.to(dev), din.k_cache.to(dev), din.v_cache.to(dev)
     dbt, dsl = din.block_table.to(dev), din.seq_lens.to(dev)
     S, _, Hkv_d, dd = dq.shape[0], None, din.k_cache.shape[2], dq.shape[2]
@@ -225,10 +257,12 @@ def bench_ours(args):
     stream = torch.cuda.current_stream()
 
     def prefill():
-        fa.fwd(q, k, v, True, 0, pin.scale, out=o, lse=lse)
+        if do_p:
+            fa.fwd(q, k, v, True, pin.window, pin.scale, out=o, lse=lse)
 
     def decode():
-        fa.decode_paged(dq, dk, dv, dbt, dsl, din.scale, out=dout, lse=dlse, workspace=ws)
+        if do_d:
+            fa.decode_paged(dq, dk, dv, dbt, dsl, din.scale, out=dout, lse=dlse, workspace=ws)
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -265,10 +299,7 @@ def bench_ours(args):
     p_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
     d_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
     p_tot, d_tot = sum(p_ms), sum(d_ms)
-    if world > 1:
-        t = torch.tensor([p_tot, d_tot], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        p_tot, d_tot = float(t[0]), float(t[1])
+    p_tot, d_tot = max_over_ranks([p_tot, d_tot], dev)
     err = fa.check_device_error()
     if err:
         raise RuntimeError(f"device error in timed region: {fa.status_string(err)}")
@@ -283,7 +314,7 @@ def bench_ours(args):
         dq2.copy_(hq, non_blocking=True)
         dk2.copy_(hk, non_blocking=True)
         dv2.copy_(hv, non_blocking=True)
-        fa.fwd(dq2, dk2, dv2, True, 0, pin.scale, out=o, lse=lse)
+        fa.fwd(dq2, dk2, dv2, True, pin.window, pin.scale, out=o, lse=lse)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -298,17 +329,14 @@ def bench_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     # ---- figures
     K = args.steps
-    p_avg = p_tot / K
-    d_avg = d_tot / K
+    p_avg = max(p_tot / K, 1e-9)
+    d_avg = max(d_tot / K, 1e-9)
     tflops = world * flops / (p_avg * 1e-3) / 1e12
     kv_gbs = world * kv_bytes / (d_avg * 1e-3) / 1e9
     traffic = recorded_traffic()
@@ -327,8 +355,8 @@ def bench_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (iid N(0,1) bf16, seeded; no dataset)",
-        "config": {"workload": "gqa4k causal prefill B=1 Hq=32 Hkv=8 N=4096 d=128 + "
-                               "decode64 paged split-KV (64 seqs, KV 4096-32768, 16-token pages)",
+        "config": {"workload": f"{pname} causal prefill B={B} Hq={Hq} Hkv={k.shape[2]} N={N} "
+                               f"d={d} + decode{S} paged split-KV (KV 4096-32768, 16-token pages)",
                    "prefill": {"B": B, "Hq": Hq, "Hkv": k.shape[2], "N": N, "d": d,
                                "causal": True, "flop_per_call": flops},
                    "decode": {"num_seqs": S, "Hq": dq.shape[1], "Hkv": Hkv_d, "d": dd,
@@ -353,14 +381,16 @@ def bench_ours(args):
                 "ms_per_step": round(e2e_ms, 4),
                 "what": "fa_fwd through the Python binding: pinned host q,k,v -> device, "
                         "kernel, O and LSE -> host, per step"},
-        "gpu_launches": 3 * K,
+        "gpu_launches": (int(do_p) + 2 * int(do_d)) * K,
         "clocks": clk.report(),
         "wall_s_timed_region": round(t_wall, 3),
         "kernel_source": kernel_source_hash(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.only != "all":
+        line["note"] = f"--only {args.only}: partial run for profiling, not a bench result"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and do_p:
         cores = len(os.sched_getaffinity(0))
-        val, desc, _ = oracle_sample(pin, args.cpu_seconds, cores)
+        val, desc, _ = oracle_sample(pin, args.cpu_seconds, cores, pname)
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
     if world > 1:
