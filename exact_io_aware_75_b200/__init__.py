@@ -34,7 +34,8 @@ FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_workspace_bytes", "fa_decode_paged",
-           "fa_status_string", "fa_check_device_error", "fa_version")
+           "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
+           "fa_version")
 
 
 class FAError(RuntimeError):
@@ -58,6 +59,8 @@ def _load():
     lib.fa_decode_workspace_bytes.restype = sz
     lib.fa_decode_paged.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged.restype = i
+    lib.fa_decode_paged_noalloc.argtypes = [vp] * 7 + [i] * 7 + [f, vp]
+    lib.fa_decode_paged_noalloc.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_check_device_error.argtypes = [vp]
@@ -184,6 +187,33 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=Non
                                 maxp, float(scale), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(),
                                 _stream(stream)), "fa_decode_paged")
+    return out, lse
+
+
+def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None,
+                         lse=None, return_lse=True, stream=None):
+    """Paged decode with the library's fixed device scratch instead of a
+    workspace, for callers that cannot allocate device memory (see
+    fa_decode_paged_noalloc in include/fa.h: 32 MiB limit, first call per
+    device before any stream capture, overlapping calls race)."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    S, Hq, d = q.shape
+    P, ps, Hkv, _ = k_cache.shape
+    maxp = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    _check(_lib.fa_decode_paged_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                                        _ptr(lse), S, P, Hq, Hkv, d, ps, maxp, float(scale),
+                                        _stream(stream)), "fa_decode_paged_noalloc")
     return out, lse
 
 

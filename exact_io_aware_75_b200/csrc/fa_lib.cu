@@ -3,3 +3,4 @@
 #include "fa_api.cu"
 #include "prefill_sm100.cu"
 #include "decode_sm100.cu"
+#include "decode_noalloc.cu"

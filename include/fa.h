@@ -27,10 +27,11 @@
  *   - head dim d in {64, 128}.
  *   - Every device pointer must be 16-byte aligned (TMA requirement);
  *     row strides are implied by the shapes.
- *   - Ownership: the caller owns every buffer.  The library allocates no
- *     device memory, keeps no per-call state, and is thread-safe.  All calls
- *     are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *     stream) and do not synchronise.
+ *   - Ownership: the caller owns every buffer.  No call allocates device
+ *     memory or keeps per-call state, and calls are thread-safe (see
+ *     fa_decode_paged_noalloc for its one fixed, library-owned scratch array).
+ *     All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and do not synchronise.
  *   - Errors: the return value is FA_OK (0) or a negative FA_ERR_* code.  On
  *     an argument error nothing is launched.  FA_ERR_CUDA reports a launch
  *     error (cudaGetLastError).  There is no CPU fallback: host pointers are
@@ -132,6 +133,32 @@ int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
                     float *lse, int num_seqs, int num_pages, int Hq, int Hkv,
                     int d, int page_size, int max_pages_per_seq, float scale,
                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_decode_paged without a workspace argument, for callers that cannot
+ * allocate device memory: code running under a host framework whose memory
+ * pool owns the device and forbids raw cudaMalloc, latency-critical serving
+ * paths where cudaMalloc's implicit synchronisation is not allowed, or
+ * embedded callers with a memory budget fixed at load time.  (The pages have
+ * no counterpart; this is an interface convenience, computing exactly what
+ * fa_decode_paged computes.)
+ *
+ * The split-KV scratch comes from a fixed 32 MiB array in the library's own
+ * device memory, which every GPU that loads the library holds until the
+ * process exits.  Sizes whose workspace (fa_decode_workspace_bytes) exceeds
+ * 32 MiB are refused with FA_ERR_WORKSPACE before any CUDA call.  The first
+ * call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  All calls share
+ * the array and it keeps the last call's contents (nothing in it needs to
+ * start at zero); calls that may overlap on the GPU race on it, so the caller
+ * must order them.  Allocates nothing.  Other arguments, results and errors
+ * as for fa_decode_paged.
+ */
+int fa_decode_paged_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                            const int *block_table, const int *seq_lens, void *o,
+                            float *lse, int num_seqs, int num_pages, int Hq, int Hkv,
+                            int d, int page_size, int max_pages_per_seq, float scale,
+                            void *stream);
 
 /* Human-readable text of a status code (static storage). */
 const char *fa_status_string(int status);
