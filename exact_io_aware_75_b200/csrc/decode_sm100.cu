@@ -88,6 +88,14 @@ struct DecShared {
     int abort;
 };
 
+// Four bf16 pairs (one 16-byte load) to four packed fp32 pairs.
+__device__ __forceinline__ void unpack8x2(uint4 a, uint64_t *f) {
+    f[0] = f2pack(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u));
+    f[1] = f2pack(__uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u));
+    f[2] = f2pack(__uint_as_float(a.z << 16), __uint_as_float(a.z & 0xffff0000u));
+    f[3] = f2pack(__uint_as_float(a.w << 16), __uint_as_float(a.w & 0xffff0000u));
+}
+
 __device__ __forceinline__ void unpack8(uint4 a, float *f) {
     f[0] = __uint_as_float(a.x << 16); f[1] = __uint_as_float(a.x & 0xffff0000u);
     f[2] = __uint_as_float(a.y << 16); f[3] = __uint_as_float(a.y & 0xffff0000u);
@@ -121,8 +129,19 @@ __device__ __forceinline__ void group_transpose_sum(float (&v)[NV], int lane) {
     }
 }
 
+// Block: warps 0-7 compute (the first NW of them work), warp 8 produces,
+// warps 9-11 only complete the third warpgroup.  Registers: launched with
+// 384 x 168; compute warpgroups 216 each, the producer warpgroup 72
+// (2 * 128 * 216 + 128 * 72 = 64,512).
+constexpr int kDecThreads = 384;
+constexpr int kDecWarpProducer = 8;
+constexpr int kDecRegsCompute = 216;
+constexpr int kDecRegsControl = 72;
+static_assert(2 * 128 * kDecRegsCompute + 128 * kDecRegsControl <= kDecThreads * 168,
+              "register split");
+
 template <int D, int QPW>
-__global__ void __launch_bounds__(32 * (kMaxComputeWarps + 1), 1)
+__global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const DecodeParams p) {
     constexpr int DPL = D / 8;          // d values per lane
@@ -144,7 +163,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     __syncthreads();
 
-    if (warp == p.NW) {
+    if (warp >= kMaxComputeWarps) {
+        regs_decrease<kDecRegsControl>();
+        if (warp != kDecWarpProducer) return;
         // ------------------------------------------------------- producer
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
@@ -178,6 +199,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         return;
     }
+    regs_increase<kDecRegsCompute>();
     if (warp >= p.NW) return;
 
     // ------------------------------------------------------------ compute
@@ -191,26 +213,28 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const int kvh = hg * p.HG + hl;
         const int h0 = kvh * p.group + qsub * QPW;   // first query head of this warp
         // q (pre-scaled by scale*log2 e), this lane's d slice
-        float q[QPW][DPL];
+        // fp32 pairs (packed f32x2 arithmetic halves the FMA instructions)
+        uint64_t q2[QPW][DPL / 2];
+        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
         #pragma unroll
         for (int qh = 0; qh < QPW; ++qh) {
             const uint16_t *qp = p.q + ((size_t)seq * p.Hq + h0 + qh) * D + 8 * ds;
             #pragma unroll
             for (int b = 0; b < DPL / 8; ++b) {
                 const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qp + 64 * b));
-                unpack8(raw, &q[qh][8 * b]);
+                unpack8x2(raw, &q2[qh][4 * b]);
             }
             #pragma unroll
-            for (int i = 0; i < DPL; ++i) q[qh][i] *= p.scale_log2;
+            for (int i = 0; i < DPL / 2; ++i) q2[qh][i] = f2mul(q2[qh][i], sc2);
         }
-        float o[QPW][DPL];
+        uint64_t o2[QPW][DPL / 2];
         float m_ref[QPW], l_acc[QPW];
         #pragma unroll
         for (int qh = 0; qh < QPW; ++qh) {
             m_ref[qh] = -INFINITY;
             l_acc[qh] = 0.f;
             #pragma unroll
-            for (int i = 0; i < DPL; ++i) o[qh][i] = 0.f;
+            for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2pack(0.f, 0.f);
         }
         const int pages = (L + kPage - 1) / kPage;
         const int pg0 = chunk * kChunkPages, pg1 = min(pages, pg0 + kChunkPages);
@@ -228,16 +252,23 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 const int t = tg + 4 * k;
                 const uint16_t *kr = reinterpret_cast<const uint16_t *>(sK) +
                                      ((size_t)(t * p.HG + hl) * D + 8 * ds);
-                float kv[DPL];
+                uint64_t kv2[DPL / 2];
                 #pragma unroll
                 for (int b = 0; b < DPL / 8; ++b)
-                    unpack8(*reinterpret_cast<const uint4 *>(kr + 64 * b), &kv[8 * b]);
+                    unpack8x2(*reinterpret_cast<const uint4 *>(kr + 64 * b), &kv2[4 * b]);
                 #pragma unroll
                 for (int qh = 0; qh < QPW; ++qh) {
-                    float acc = 0.f;
+                    uint64_t a0 = f2mul(q2[qh][0], kv2[0]);
+                    uint64_t a1 = f2mul(q2[qh][1], kv2[1]);
                     #pragma unroll
-                    for (int i = 0; i < DPL; ++i) acc = fmaf(q[qh][i], kv[i], acc);
-                    sc[k * QPW + qh] = acc;
+                    for (int i = 2; i < DPL / 2; i += 2) {
+                        a0 = f2fma(q2[qh][i], kv2[i], a0);
+                        a1 = f2fma(q2[qh][i + 1], kv2[i + 1], a1);
+                    }
+                    float x0, x1, y0, y1;
+                    f2unpack(a0, x0, x1);
+                    f2unpack(a1, y0, y1);
+                    sc[k * QPW + qh] = (x0 + x1) + (y0 + y1);
                 }
             }
             group_transpose_sum<NV>(sc, lane);
@@ -280,8 +311,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     const float alpha = (m_ref[qh] == -INFINITY) ? 0.f : ex2(m_ref[qh] - pmax[qh]);
                     m_ref[qh] = pmax[qh];
                     l_acc[qh] *= alpha;
+                    const uint64_t a2 = f2pack(alpha, alpha);
                     #pragma unroll
-                    for (int i = 0; i < DPL; ++i) o[qh][i] *= alpha;
+                    for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2mul(o2[qh][i], a2);
                 }
             }
             // ---- probabilities of the held scores
@@ -315,24 +347,29 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 if (t < nvalid) {   // slots past seq_len may hold anything
                     const uint16_t *vr = reinterpret_cast<const uint16_t *>(sV) +
                                          ((size_t)(t * p.HG + hl) * D + 8 * ds);
-                    float vv[DPL];
+                    uint64_t vv2[DPL / 2];
                     #pragma unroll
                     for (int b = 0; b < DPL / 8; ++b)
-                        unpack8(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv[8 * b]);
+                        unpack8x2(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv2[4 * b]);
                     #pragma unroll
-                    for (int qh = 0; qh < QPW; ++qh)
+                    for (int qh = 0; qh < QPW; ++qh) {
+                        const uint64_t pp = f2pack(pr[k][qh], pr[k][qh]);
                         #pragma unroll
-                        for (int i = 0; i < DPL; ++i) o[qh][i] = fmaf(pr[k][qh], vv[i], o[qh][i]);
+                        for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2fma(pp, vv2[i], o2[qh][i]);
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.empty[st]);
         }
         // ---- merge the four token groups and write this chunk's partial
+        float o[QPW][DPL];
         #pragma unroll
         for (int qh = 0; qh < QPW; ++qh) {
             l_acc[qh] += __shfl_xor_sync(0xffffffffu, l_acc[qh], 8);
             l_acc[qh] += __shfl_xor_sync(0xffffffffu, l_acc[qh], 16);
+            #pragma unroll
+            for (int i = 0; i < DPL / 2; ++i) f2unpack(o2[qh][i], o[qh][2 * i], o[qh][2 * i + 1]);
             #pragma unroll
             for (int i = 0; i < DPL; ++i) {
                 o[qh][i] += __shfl_xor_sync(0xffffffffu, o[qh][i], 8);
@@ -362,17 +399,23 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
 }
 
-// Merge the chunks of each (sequence, head): one warp per row.
+// Merge the chunks of each (sequence, head).  One block of kCombineWarps
+// warps per row: the row's max LSE first, then each warp sums a strided
+// subset of the chunks (several loads in flight), and the warps' partial
+// sums are added in shared memory.
+constexpr int kCombineWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(32 * kCombineWarps)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
                       const int *__restrict__ seq_lens, uint16_t *__restrict__ o,
                       float *__restrict__ lse, int num_seqs, int Hq, int max_pages,
                       int max_chunks) {
     constexpr int PER = D / 32;
-    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= num_seqs * Hq) return;
+    __shared__ float s_acc[kCombineWarps][D];
+    __shared__ float s_w[kCombineWarps];
+    const int row = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int s = row / Hq, h = row % Hq;
     int L = __ldg(seq_lens + s);
     L = max(0, min(L, max_pages * kPage));
@@ -387,22 +430,47 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
     float wsum = 0.f;
     if (m != -INFINITY) {
-        for (int c = 0; c < nc; ++c) {
+        const float *src0 = part_o + ((size_t)s * max_chunks * Hq + h) * D + lane * PER;
+        #pragma unroll 4
+        for (int c = warp; c < nc; c += kCombineWarps) {
             const float w = __expf(lse_p[(size_t)c * Hq] - m);
             wsum += w;
-            const float *src = part_o + (((size_t)s * max_chunks + c) * Hq + h) * D + lane * PER;
-            #pragma unroll
-            for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, src[i], acc[i]);
+            const float4 v = *reinterpret_cast<const float4 *>(src0 + (size_t)c * Hq * D);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
+            if constexpr (PER == 8) {
+                const float4 u = *reinterpret_cast<const float4 *>(src0 + (size_t)c * Hq * D + 4);
+                acc[4] = fmaf(w, u.x, acc[4]);
+                acc[5] = fmaf(w, u.y, acc[5]);
+                acc[6] = fmaf(w, u.z, acc[6]);
+                acc[7] = fmaf(w, u.w, acc[7]);
+            }
         }
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    #pragma unroll
+    for (int i = 0; i < PER; ++i) s_acc[warp][lane * PER + i] = acc[i];
+    if (lane == 0) s_w[warp] = wsum;
+    __syncthreads();
+    if (warp != 0) return;
+    float tw = 0.f;
+    #pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) tw += s_w[w];
+    const float inv = tw > 0.f ? 1.f / tw : 0.f;
+    float r[PER];
+    #pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        float t = 0.f;
+        #pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) t += s_acc[w][lane * PER + i];
+        r[i] = t * inv;
+    }
     uint16_t *dst = o + ((size_t)s * Hq + h) * D + lane * PER;
     #pragma unroll
-    for (int i = 0; i < PER; i += 2) {
-        const uint32_t pk = pack_bf16(acc[i] * inv, acc[i + 1] * inv);
-        *reinterpret_cast<uint32_t *>(dst + i) = pk;
-    }
-    if (lse && lane == 0) lse[(size_t)s * Hq + h] = wsum > 0.f ? m + __logf(wsum) : -INFINITY;
+    for (int i = 0; i < PER; i += 2)
+        *reinterpret_cast<uint32_t *>(dst + i) = pack_bf16(r[i], r[i + 1]);
+    if (lse && lane == 0) lse[(size_t)s * Hq + h] = tw > 0.f ? m + __logf(tw) : -INFINITY;
 }
 
 struct Plan {
@@ -440,7 +508,7 @@ int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParam
     if (cudaFuncSetAttribute(decode_split_kernel<D, QPW>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return -5;
-    decode_split_kernel<D, QPW><<<device_sm_count(), 32 * (p.NW + 1), smem, stream>>>(tk, tv, p);
+    decode_split_kernel<D, QPW><<<device_sm_count(), kDecThreads, smem, stream>>>(tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 
@@ -501,14 +569,13 @@ int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
            : pl.QPW == 2 ? launch_split<64, 2>(tk, tv, p, stream)
                          : launch_split<64, 1>(tk, tv, p, stream);
     if (rc) return rc;
-    const int rows_out = a.num_seqs * a.Hq;
-    const int blocks = (rows_out + 3) / 4;
+    const int blocks = a.num_seqs * a.Hq;
     if (a.d == 128)
-        decode_combine_kernel<128><<<blocks, 128, 0, stream>>>(
+        decode_combine_kernel<128><<<blocks, 32 * kCombineWarps, 0, stream>>>(
             p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.num_seqs,
             a.Hq, a.max_pages, pl.max_chunks);
     else
-        decode_combine_kernel<64><<<blocks, 128, 0, stream>>>(
+        decode_combine_kernel<64><<<blocks, 32 * kCombineWarps, 0, stream>>>(
             p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.num_seqs,
             a.Hq, a.max_pages, pl.max_chunks);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;

@@ -42,10 +42,21 @@ namespace prefill_impl {
 
 constexpr int kBlockM = 128;        // rows per tile (TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
-constexpr int kThreads = 320;       // 8 softmax warps + TMA warp + MMA warp
+constexpr int kThreads = 384;       // 2 softmax warpgroups + 1 warpgroup for TMA / MMA
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
+// Register split: launched with 384 x 168 = 64,512 registers; the softmax
+// warpgroups take 216 each, the TMA/MMA warpgroup 72:
+// 2 * 128 * 216 + 128 * 72 = 64,512.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsControl = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * 168, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+#ifndef FA_POLY_PERIOD
+#define FA_POLY_PERIOD 8
+#endif
+// One score pair in kPolyPeriod takes the FMA-pipe exponential (0 = none).
+constexpr int kPolyPeriod = FA_POLY_PERIOD;
 constexpr uint32_t kTmemCols = 512;
 
 template <int D>
@@ -115,6 +126,18 @@ __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     return true;
 }
 
+// Unit `it` of this CTA: rows of G = gridDim.x units are walked in
+// alternating directions (snake order), so with units sorted by decreasing
+// cost every CTA gets a similar total.
+__device__ __forceinline__ int sched_unit(int it) {
+    const int G = gridDim.x, b = blockIdx.x;
+    return (it & 1) ? (it + 1) * G - 1 - b : it * G + b;
+}
+
+#define FOR_EACH_UNIT(u)                                                  \
+    for (int it_ = 0, u = 0; it_ * (int)gridDim.x < p.num_units; ++it_)   \
+        if ((u = sched_unit(it_)) < p.num_units)
+
 struct Shared {
     uint64_t q_full[2], q_empty[2];
     uint64_t kv_full[8], kv_empty[8];
@@ -132,7 +155,7 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
     volatile int *abort = &sh.abort;
     uint32_t q_uses[2] = {0, 0};
     uint32_t kv_it = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FOR_EACH_UNIT(u) {
         Unit w;
         if (!get_unit(u, p, w)) continue;
         for (int t = 0; t < 2; ++t) {
@@ -206,7 +229,7 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
         }
     };
 
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FOR_EACH_UNIT(u) {
         Unit w;
         if (!get_unit(u, p, w)) continue;
         bool first_pv[2] = {true, true};
@@ -302,7 +325,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
     const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, pv_cnt = 0;
 
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    FOR_EACH_UNIT(u) {
         Unit w;
         if (!get_unit(u, p, w)) continue;
         const int lo = w.lo[t], hi = w.hi[t];
@@ -337,9 +360,17 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
                 for (int c = 0; c < kBlockN; ++c)
                     if (c >= c_hi || c < c_lo) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max: eight independent chains of 3-input max, then combine
+            float mq[8];
             #pragma unroll
-            for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+            for (int i = 0; i < 8; ++i) {
+                float a = fmax3(s[i], s[8 + i], s[16 + i]);
+                #pragma unroll
+                for (int b = 24; b + 8 < kBlockN; b += 16) a = fmax3(a, s[b + i], s[b + 8 + i]);
+                mq[i] = fmaxf(a, s[kBlockN - 8 + i]);
+            }
+            const float mx = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]),
+                                   fmaxf(mq[6], mq[7]));
             const float m_blk = mx * sl2;
             if (j == lo) {
                 m_ref = m_blk;
@@ -368,21 +399,35 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
                 }
             }
             const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-            float sum0 = 0.f, sum1 = 0.f;
+            // P = 2^(s*scale*log2e - m): MUFU ex2 for most pairs, the FMA-pipe
+            // polynomial for one pair in kPolyPeriod ("software exponentials")
+            const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-mb, -mb);
+            uint64_t acc[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
             #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
                 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, -mb));
-                    const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, -mb));
-                    sum0 += p0;
-                    sum1 += p1;
+                    const uint64_t x = f2fma(f2pack(s[64 * h + 2 * c], s[64 * h + 2 * c + 1]), c2, nm2);
+                    float x0, x1, p0, p1;
+                    f2unpack(x, x0, x1);
+                    if (kPolyPeriod > 0 && (c % kPolyPeriod) == kPolyPeriod - 1) {
+                        exp2_poly_pair(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    }
+                    acc[c & 1] = f2add(acc[c & 1], f2pack(p0, p1));
                     pk[c] = pack_bf16(p0, p1);
                 }
                 tmem_st32(tS + 32 * h, pk);
             }
-            l += sum0 + sum1;
+            {
+                float a0, a1, b0, b1;
+                f2unpack(acc[0], a0, a1);
+                f2unpack(acc[1], b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -479,11 +524,15 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_after();
 
     if (warp < 8) {
+        regs_increase<kRegsSoftmax>();
         softmax_wg<D>(p, sh);
-    } else if (warp == kWarpTma) {
-        if (lane_id() == 0) producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
     } else {
-        if (lane_id() == 0) mma_issuer<D>(p, sh, sQ, sKV);
+        regs_decrease<kRegsControl>();
+        if (warp == kWarpTma) {
+            if (lane_id() == 0) producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+        } else if (warp == kWarpMma) {
+            if (lane_id() == 0) mma_issuer<D>(p, sh, sQ, sKV);
+        }
     }
     __syncwarp();
     tc_fence_before();

@@ -251,12 +251,84 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Per-warpgroup register budget (all four warps of the warpgroup execute it).
+// The sum over warpgroups must stay within the registers the block was
+// launched with, or the increase waits forever.
+template <int N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------- arithmetic
 // Hardware base-2 exponential (MUFU), flushes subnormals; ex2(-inf) = +0.
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Maximum of three floats (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Packed fp32 pairs (sm_100 executes f32x2 add/mul/fma as one instruction).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2add_rm(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x on the FMA pipe for a pair, x <= 2^7 (larger negative x, -inf
+// included, is clamped to -127, where the result is below 2^-126).
+// x = j + f with j = floor(x) taken by a round-down add of 1.5*2^23 (the
+// integer lands in the low mantissa bits), f = x - j in [0, 1); 2^f is a cubic
+// with p(0) = 1 fitted for minimax relative error on [0, 1] (8.6e-5, see
+// fit_exp2_poly.py); 2^j is added into the exponent field as an integer.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &r0, float &r1) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c1 = 6.951166391e-01f, c2 = 2.276449800e-01f, c3 = 7.706724107e-02f;
+    const uint64_t x = f2pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t y = f2add_rm(x, f2pack(kShift, kShift));
+    const uint64_t j = f2add(y, f2pack(-kShift, -kShift));
+    const uint64_t f = f2fma(j, f2pack(-1.f, -1.f), x);
+    uint64_t p = f2fma(f, f2pack(c3, c3), f2pack(c2, c2));
+    p = f2fma(p, f, f2pack(c1, c1));
+    p = f2fma(p, f, f2pack(1.f, 1.f));
+    float p0, p1, y0, y1;
+    f2unpack(p, p0, p1);
+    f2unpack(y, y0, y1);
+    r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
+    r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
 }
 
 // Two fp32 values to a packed bf16 pair, round to nearest even; `lo` goes to
