@@ -42,18 +42,24 @@ namespace prefill_impl {
 
 constexpr int kBlockM = 128;        // rows per tile (TMEM lanes)
 constexpr int kBlockN = 128;        // keys per K/V tile
-constexpr int kThreads = 384;       // 2 softmax warpgroups + 1 warpgroup for TMA / MMA
+constexpr int kHalf = 64;           // P is published to the MMA warp in halves
+// 2 softmax warpgroups (one per Q tile, one thread per row) + 1 warpgroup
+// for TMA / MMA.
+constexpr int kThreads = 384;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 // Register split: launched with 384 x 168 = 64,512 registers; the softmax
 // warpgroups take 216 each, the TMA/MMA warpgroup 72:
 // 2 * 128 * 216 + 128 * 72 = 64,512.
+constexpr int kLaunchRegs = 168;
 constexpr int kRegsSoftmax = 216;
 constexpr int kRegsControl = 72;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * 168, "register split");
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
+              "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #ifndef FA_POLY_PERIOD
-#define FA_POLY_PERIOD 8
+#define FA_POLY_PERIOD 0
 #endif
 // One score pair in kPolyPeriod takes the FMA-pipe exponential (0 = none).
 constexpr int kPolyPeriod = FA_POLY_PERIOD;
@@ -141,7 +147,7 @@ __device__ __forceinline__ int sched_unit(int it) {
 struct Shared {
     uint64_t q_full[2], q_empty[2];
     uint64_t kv_full[8], kv_empty[8];
-    uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+    uint64_t s_full[2], p_lo[2], p_hi[2], o_full[2], o_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -206,27 +212,51 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
     uint32_t kv_it = 0;
 
     // S_t = Q_t K^T: d/16 MMAs of K=16; K-major, 128-byte swizzle, atoms of
-    // 8 rows x 128 bytes (SBO 1024), 64 columns per TMA box.
+    // 8 rows x 128 bytes (SBO 1024), 64 columns per TMA box.  Descriptors
+    // are precomputed; a k-step adds its byte offset >> 4 to the low half.
+    const uint32_t q_lo = desc_lo(q_addr, 16), kv_lo = desc_lo(kv_addr, 16);
+    const uint32_t v_lo = desc_lo(kv_addr, C::kBoxBytes);
+    constexpr uint32_t kTileStep = C::kTileBytes >> 4;
     auto issue_s = [&](int t, int kslot) {
-        const uint32_t qa = q_addr + t * C::kTileBytes;
-        const uint32_t ka = kv_addr + kslot * C::kTileBytes;
+        const uint32_t qa = q_lo + t * kTileStep;
+        const uint32_t ka = kv_lo + kslot * kTileStep;
+        const uint32_t dt = tmem + t * kBlockN;
         #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * C::kBoxBytes + (ks & 3) * 32;
-            mma_ss(tmem + t * kBlockN, smem_desc_sw128(qa + off, 16, 1024),
-                   smem_desc_sw128(ka + off, 16, 1024), idS, ks > 0);
+            const uint32_t off = ((ks >> 2) * C::kBoxBytes + (ks & 3) * 32) >> 4;
+            mma_ss_lo(dt, qa + off, ka + off, idS, ks > 0 ? 1u : 0u);
         }
     };
     // O_t += P_t V: 128/16 MMAs of K=16 keys; V is MN-major (d contiguous):
     // 16 keys = two 8-row groups (SBO 1024), d split in 64-column boxes (LBO).
-    auto issue_pv = [&](int t, int vslot, bool first) {
-        const uint32_t va = kv_addr + vslot * C::kTileBytes;
+    auto issue_pv_half = [&](int t, int vslot, bool first, int half) {
+        const uint32_t va = v_lo + vslot * kTileStep;
+        const uint32_t dt = tmem + C::kColO + t * D;
+        const uint32_t pa = tmem + t * kBlockN;
         #pragma unroll
-        for (int ks = 0; ks < kBlockN / 16; ++ks) {
-            mma_ts(tmem + C::kColO + t * D, tmem + t * kBlockN + ks * 8,
-                   smem_desc_sw128(va + ks * 2048, C::kBoxBytes, 1024), idPV,
-                   (ks > 0 || !first) ? 1u : 0u);
+        for (int k = 0; k < 4; ++k) {
+            const int ks = half * 4 + k;
+            mma_ts_lo(dt, pa + half * kHalf + k * 8, va + ((ks * 2048) >> 4), idPV,
+                      (ks > 0 || !first) ? 1u : 0u);
         }
+    };
+    // P_t V in two halves of 64 keys, each issued as soon as the softmax
+    // warpgroup has published that half of P.
+    auto issue_pv = [&](int t, int vslot, bool &first) -> bool {
+        if (!mbar_wait(&sh.p_lo[t], p_cnt[t] & 1, abort)) return false;
+        if (first) {
+            if (!mbar_wait(&sh.o_empty[t], (oe_uses[t] & 1) ^ 1, abort)) return false;
+            ++oe_uses[t];
+        }
+        tc_fence_after();
+        issue_pv_half(t, vslot, first, 0);
+        if (!mbar_wait(&sh.p_hi[t], p_cnt[t] & 1, abort)) return false;
+        tc_fence_after();
+        issue_pv_half(t, vslot, false, 1);
+        ++p_cnt[t];
+        first = false;
+        tc_commit(&sh.o_full[t]);
+        return true;
     };
 
     FOR_EACH_UNIT(u) {
@@ -256,16 +286,7 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
                 tc_commit(&sh.s_full[0]);
             }
             if (prev1) {
-                if (!mbar_wait(&sh.p_full[1], p_cnt[1] & 1, abort)) goto out;
-                ++p_cnt[1];
-                if (first_pv[1]) {
-                    if (!mbar_wait(&sh.o_empty[1], (oe_uses[1] & 1) ^ 1, abort)) goto out;
-                    ++oe_uses[1];
-                }
-                tc_fence_after();
-                issue_pv(1, prev_v, first_pv[1]);
-                first_pv[1] = false;
-                tc_commit(&sh.o_full[1]);
+                if (!issue_pv(1, prev_v, first_pv[1])) goto out;
                 tc_commit(&sh.kv_empty[prev_v]);
             }
             if (in1) {
@@ -278,30 +299,13 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
             if (!mbar_wait(&sh.kv_full[vslot], vuse & 1, abort)) goto out;
             tc_fence_after();
             if (in0) {
-                if (!mbar_wait(&sh.p_full[0], p_cnt[0] & 1, abort)) goto out;
-                ++p_cnt[0];
-                if (first_pv[0]) {
-                    if (!mbar_wait(&sh.o_empty[0], (oe_uses[0] & 1) ^ 1, abort)) goto out;
-                    ++oe_uses[0];
-                }
-                tc_fence_after();
-                issue_pv(0, vslot, first_pv[0]);
-                first_pv[0] = false;
-                tc_commit(&sh.o_full[0]);
+                if (!issue_pv(0, vslot, first_pv[0])) goto out;
             }
             if (!in1) tc_commit(&sh.kv_empty[vslot]);
             prev_v = vslot;
         }
         if ((w.hi_all - 1) >= w.lo[1] && (w.hi_all - 1) < w.hi[1]) {
-            if (!mbar_wait(&sh.p_full[1], p_cnt[1] & 1, abort)) goto out;
-            ++p_cnt[1];
-            if (first_pv[1]) {
-                if (!mbar_wait(&sh.o_empty[1], (oe_uses[1] & 1) ^ 1, abort)) goto out;
-                ++oe_uses[1];
-            }
-            tc_fence_after();
-            issue_pv(1, prev_v, first_pv[1]);
-            tc_commit(&sh.o_full[1]);
+            if (!issue_pv(1, prev_v, first_pv[1])) goto out;
             tc_commit(&sh.kv_empty[prev_v]);
         }
     }
@@ -309,6 +313,43 @@ out:
     // Wait for every MMA this thread issued before TMEM is released.
     tc_commit(&sh.drain);
     mbar_drain_wait(&sh.drain, 0);
+}
+
+// Maximum of 64 scores: eight chains of 3-input max, then a combine.
+__device__ __forceinline__ float row_max64(const float (&v)[kHalf]) {
+    float mq[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float a = fmax3(v[i], v[8 + i], v[16 + i]);
+        a = fmax3(a, v[24 + i], v[32 + i]);
+        a = fmax3(a, v[40 + i], v[48 + i]);
+        mq[i] = fmaxf(a, v[56 + i]);
+    }
+    return fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
+}
+
+// P = 2^(s*scale*log2e - m) for 64 scores, packed to bf16 pairs, with the
+// running fp32 sum.  MUFU ex2 for most pairs, the FMA-pipe polynomial for one
+// pair in kPolyPeriod ("software exponentials").
+__device__ __forceinline__ void exp_half(const float (&v)[kHalf], float sl2, float mb,
+                                         uint32_t (&pk)[kHalf / 2], uint64_t &acc) {
+    const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-mb, -mb);
+    uint64_t a2[2] = {acc, f2pack(0.f, 0.f)};
+    #pragma unroll
+    for (int c = 0; c < kHalf / 2; ++c) {
+        const uint64_t x = f2fma(f2pack(v[2 * c], v[2 * c + 1]), c2, nm2);
+        float x0, x1, p0, p1;
+        f2unpack(x, x0, x1);
+        if (kPolyPeriod > 0 && (c % kPolyPeriod) == kPolyPeriod - 1) {
+            exp2_poly_pair(x0, x1, p0, p1);
+        } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+        }
+        a2[c & 1] = f2add(a2[c & 1], f2pack(p0, p1));
+        pk[c] = pack_bf16(p0, p1);
+    }
+    acc = f2add(a2[0], a2[1]);
 }
 
 // ---------------------------------------------------------------- softmax
@@ -337,42 +378,52 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
             if (!mbar_wait_warp(&sh.s_full[t], s_cnt & 1, abort)) return;
             ++s_cnt;
             tc_fence_after();
-            float s[kBlockN];
-            {
-                uint32_t raw[kBlockN];
-                tmem_ld32(tS + 0, raw);
-                tmem_ld32(tS + 32, raw + 32);
-                tmem_ld32(tS + 64, raw + 64);
-                tmem_ld32(tS + 96, raw + 96);
-                tmem_wait_ld();
-                #pragma unroll
-                for (int c = 0; c < kBlockN; ++c) s[c] = __uint_as_float(raw[c]);
-            }
+            const bool first = (j == lo);
             const int k0 = j * kBlockN;
             const bool edge = (k0 + kBlockN > w.L) || (p.causal && k0 + kBlockN - 1 > rmin) ||
                               (p.window > 0 && k0 <= rmax - p.window);
+            // visible keys of this row in the tile: c in [c_lo, c_hi)
+            int c_hi = w.L - k0;
+            if (p.causal) c_hi = min(c_hi, row + 1 - k0);
+            const int c_lo = (p.window > 0) ? row - p.window + 1 - k0 : 0;
+            // Scores in two halves of 64 keys: the second half's TMEM load is
+            // in flight while the first half is masked and reduced.
+            float sA[kHalf], sB[kHalf];
+            {
+                uint32_t raw[kHalf];
+                tmem_ld32(tS + 0, raw);
+                tmem_ld32(tS + 32, raw + 32);
+                tmem_wait_ld();
+                #pragma unroll
+                for (int c = 0; c < kHalf; ++c) sA[c] = __uint_as_float(raw[c]);
+            }
+            uint32_t rawB[kHalf];
+            tmem_ld32(tS + 64, rawB);
+            tmem_ld32(tS + 96, rawB + 32);
             if (edge) {
-                // visible keys of this row in the tile: c in [c_lo, c_hi)
-                int c_hi = w.L - k0;
-                if (p.causal) c_hi = min(c_hi, row + 1 - k0);
-                const int c_lo = (p.window > 0) ? row - p.window + 1 - k0 : 0;
                 #pragma unroll
-                for (int c = 0; c < kBlockN; ++c)
-                    if (c >= c_hi || c < c_lo) s[c] = -INFINITY;
+                for (int c = 0; c < kHalf; ++c)
+                    if (c >= c_hi || c < c_lo) sA[c] = -INFINITY;
             }
-            // row max: eight independent chains of 3-input max, then combine
-            float mq[8];
+            const float mA = row_max64(sA);
+            // With the reference max unchanged (the common case under the
+            // conditional rescale) the first half's P needs no block max:
+            // start its exponentials while the block max is still unknown.
+            float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+            uint32_t pkA[kHalf / 2];
+            uint64_t accA = f2pack(0.f, 0.f);
+            if (!first) exp_half(sA, sl2, mb, pkA, accA);
+            tmem_wait_ld();
             #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float a = fmax3(s[i], s[8 + i], s[16 + i]);
+            for (int c = 0; c < kHalf; ++c) sB[c] = __uint_as_float(rawB[c]);
+            if (edge) {
                 #pragma unroll
-                for (int b = 24; b + 8 < kBlockN; b += 16) a = fmax3(a, s[b + i], s[b + 8 + i]);
-                mq[i] = fmaxf(a, s[kBlockN - 8 + i]);
+                for (int c = 0; c < kHalf; ++c)
+                    if (c + kHalf >= c_hi || c + kHalf < c_lo) sB[c] = -INFINITY;
             }
-            const float mx = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]),
-                                   fmaxf(mq[6], mq[7]));
-            const float m_blk = mx * sl2;
-            if (j == lo) {
+            const float m_blk = fmaxf(mA, row_max64(sB)) * sl2;
+            bool redo = first;
+            if (first) {
                 m_ref = m_blk;
             } else {
                 const bool need = m_blk > m_ref + kRescaleThreshold;
@@ -382,7 +433,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
                     // O_t holds P V of the previous block only once that MMA is done.
                     if (!mbar_wait_warp(&sh.o_full[t], (pv_cnt - 1) & 1, abort)) return;
                     tc_fence_after();
-                    // 16 columns at a time: the 128 scores of the row stay live
+                    // 16 columns at a time: the row's scores stay live
                     #pragma unroll 1
                     for (int c = 0; c < D; c += 16) {
                         uint32_t ov[16];
@@ -396,42 +447,36 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
                     tmem_wait_st();
                     l *= alpha;
                     m_ref = m_new;
+                    redo = true;
                 }
             }
-            const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-            // P = 2^(s*scale*log2e - m): MUFU ex2 for most pairs, the FMA-pipe
-            // polynomial for one pair in kPolyPeriod ("software exponentials")
-            const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-mb, -mb);
-            uint64_t acc[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
-            #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-                #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const uint64_t x = f2fma(f2pack(s[64 * h + 2 * c], s[64 * h + 2 * c + 1]), c2, nm2);
-                    float x0, x1, p0, p1;
-                    f2unpack(x, x0, x1);
-                    if (kPolyPeriod > 0 && (c % kPolyPeriod) == kPolyPeriod - 1) {
-                        exp2_poly_pair(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2(x0);
-                        p1 = ex2(x1);
-                    }
-                    acc[c & 1] = f2add(acc[c & 1], f2pack(p0, p1));
-                    pk[c] = pack_bf16(p0, p1);
-                }
-                tmem_st32(tS + 32 * h, pk);
+            if (redo) {
+                mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+                accA = f2pack(0.f, 0.f);
+                exp_half(sA, sl2, mb, pkA, accA);
             }
-            {
-                float a0, a1, b0, b1;
-                f2unpack(acc[0], a0, a1);
-                f2unpack(acc[1], b0, b1);
-                l += (a0 + a1) + (b0 + b1);
-            }
+            // publish P for keys 0-63 (bf16 pairs in S columns 0-31): the MMA
+            // warp starts that half of P V
+            tmem_st32(tS + 0, pkA);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.p_full[t]);
+            if (lane == 0) mbar_arrive(&sh.p_lo[t]);
+            // keys 64-127 (S columns 64-95)
+            uint32_t pkB[kHalf / 2];
+            uint64_t accB = f2pack(0.f, 0.f);
+            exp_half(sB, sl2, mb, pkB, accB);
+            tmem_st32(tS + kHalf, pkB);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_hi[t]);
+            {
+                float a0, a1, b0, b1;
+                f2unpack(accA, a0, a1);
+                f2unpack(accB, b0, b1);
+                l += (a0 + a1) + (b0 + b1);
+            }
             ++pv_cnt;
         }
         // ---- epilogue: O / l, LSE
@@ -501,7 +546,8 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mbar_init(&sh.q_full[t], 1);
             mbar_init(&sh.q_empty[t], 1);
             mbar_init(&sh.s_full[t], 1);
-            mbar_init(&sh.p_full[t], 4);
+            mbar_init(&sh.p_lo[t], 4);
+            mbar_init(&sh.p_hi[t], 4);
             mbar_init(&sh.o_full[t], 1);
             mbar_init(&sh.o_empty[t], 4);
         }
@@ -523,7 +569,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
 
-    if (warp < 8) {
+    if (warp < kSoftmaxWarps) {
         regs_increase<kRegsSoftmax>();
         softmax_wg<D>(p, sh);
     } else {
@@ -542,6 +588,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tmem_dealloc(sh.tmem_base, kTmemCols);
     }
 }
+
+// Shared memory per CTA: static (barriers, exchange buffers) + dynamic
+// (Q tiles, K/V ring, 1 KiB alignment slack) within the 227 KiB opt-in limit.
+static_assert(Cfg<128>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
+static_assert(Cfg<64>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 
 template <int D>
 int launch_d(const PrefillArgs &a, cudaStream_t stream) {
