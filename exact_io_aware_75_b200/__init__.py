@@ -35,7 +35,7 @@ FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_workspace_bytes", "fa_decode_paged",
            "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
-           "fa_version")
+           "fa_selftest_watchdog", "fa_version")
 
 
 class FAError(RuntimeError):
@@ -65,6 +65,8 @@ def _load():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_check_device_error.argtypes = [vp]
     lib.fa_check_device_error.restype = i
+    lib.fa_selftest_watchdog.argtypes = [vp]
+    lib.fa_selftest_watchdog.restype = i
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i
     return lib
@@ -215,6 +217,12 @@ def decode_paged_noalloc(q, k_cache, v_cache, block_table, seq_lens, scale=None,
                                         _ptr(lse), S, P, Hq, Hkv, d, ps, maxp, float(scale),
                                         _stream(stream)), "fa_decode_paged_noalloc")
     return out, lse
+
+
+def selftest_watchdog(stream=None) -> int:
+    """Launch the watchdog diagnostic (a wait that must time out); read the
+    result with check_device_error()."""
+    return int(_lib.fa_selftest_watchdog(_stream(stream)))
 
 
 def check_device_error(stream=None) -> int:

@@ -62,6 +62,21 @@ int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t d
     return r == CUDA_SUCCESS ? 0 : -1;
 }
 
+// Diagnostic kernel for the watchdog: waits on a barrier that nothing ever
+// arrives on.  The bounded wait gives up after ~1 s, records the timeout in
+// the device error word and the kernel returns normally.
+__global__ void watchdog_probe_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);
+}
+
 }  // namespace fa
 
 namespace {
@@ -212,6 +227,11 @@ int fa_check_device_error(void *stream) {
     if (word == fa::kDevErrTimeout) return FA_ERR_TIMEOUT;
     if (word == fa::kDevErrInput) return FA_ERR_INVALID_ARG;
     return word ? FA_ERR_CUDA : FA_OK;
+}
+
+int fa_selftest_watchdog(void *stream) {
+    fa::watchdog_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_version(void) { return 100; }

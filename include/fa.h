@@ -171,6 +171,15 @@ const char *fa_status_string(int status);
  */
 int fa_check_device_error(void *stream);
 
+/*
+ * Diagnostic: launches a one-warp kernel whose wait on a barrier never
+ * completes, so the device-side watchdog must end it: after about a second
+ * the wait gives up, the error word is set and the kernel returns.  A later
+ * fa_check_device_error() then reports FA_ERR_TIMEOUT and the CUDA context
+ * stays usable.  Returns FA_OK once launched (asynchronous on `stream`).
+ */
+int fa_selftest_watchdog(void *stream);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int fa_version(void);
 
