@@ -50,6 +50,10 @@ def lib():
         L.oracle_lse_combine.argtypes = [_f64p, _f64p, ctypes.c_int, ctypes.c_int64,
                                          ctypes.c_int, _f64p, _f64p]
         L.oracle_lse_combine.restype = ctypes.c_int
+        L.oracle_attn_bwd_varlen.argtypes = [
+            _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, _f64p, _f64p, _f64p]
+        L.oracle_attn_bwd_varlen.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -180,3 +184,34 @@ def lse_combine(o_parts, lse_parts):
     lse = np.empty((R,), np.float64)
     _check(lib().oracle_lse_combine(op, lp, P, R, d, o, lse), "lse_combine")
     return o, lse
+
+
+def attn_bwd_varlen(q, k, v, dout, cu_seqlens, causal=False, window=0, scale=None):
+    """Gradients of packed attention for upstream dO.  q/dout [T,Hq,d],
+    k/v [T,Hkv,d], cu_seqlens [S+1] -> dQ [T,Hq,d], dK [T,Hkv,d], dV [T,Hkv,d]."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.empty((T, Hq, d), np.float64)
+    dk = np.empty((T, Hkv, d), np.float64)
+    dv = np.empty((T, Hkv, d), np.float64)
+    _check(lib().oracle_attn_bwd_varlen(qb, kb, vb, db, cu, len(cu) - 1, Hq, Hkv, d,
+                                        int(causal), int(window), float(scale), dq, dk, dv),
+           "attn_bwd_varlen")
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, dout, causal=False, window=0, scale=None):
+    """Dense batch gradients.  q/dout [B,N,Hq,d], k/v [B,N,Hkv,d]
+    -> dQ [B,N,Hq,d], dK [B,N,Hkv,d], dV [B,N,Hkv,d]."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    dq, dk, dv = attn_bwd_varlen(qb.reshape(B * N, Hq, d), kb.reshape(B * N, Hkv, d),
+                                 vb.reshape(B * N, Hkv, d), db.reshape(B * N, Hq, d), cu,
+                                 causal, window, scale)
+    return (dq.reshape(B, N, Hq, d), dk.reshape(B, N, Hkv, d), dv.reshape(B, N, Hkv, d))

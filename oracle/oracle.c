@@ -339,3 +339,105 @@ int oracle_lse_combine(const double *o_parts, const double *lse_parts,
     }
     return 0;
 }
+
+/*
+ * Backward of packed-sequence attention (the gradients the backward pass
+ * recomputes from Q, K, V and the saved statistics; "What attention costs",
+ * the FlashAttention paragraph on not storing the attention matrix).  The
+ * pages give no formulas; these are the chain rule through the definition
+ * above, with the upstream gradient dO = dLoss/dO:
+ *   P_ij  = softmax_j(S_ij) over A(i)           (two-pass, as attend_row)
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = dO_i . V_j
+ *   D_i   = sum_j P_ij dP_ij                    (softmax Jacobian term)
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij K_j
+ *   dK_j  = scale sum_i dS_ij Q_i
+ * With GQA, dK and dV of KV head g sum over the query heads that read g.
+ *   q, dout [total, Hq, d]; k, v [total, Hkv, d] (bf16 bits)
+ *   dq [total, Hq, d]; dk, dv [total, Hkv, d] (fp64)
+ * Each (sequence, KV head) is one task that owns its dK/dV rows; sums run in
+ * a fixed order (query head, then row, ascending), independent of threads.
+ */
+int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                           int Hq, int Hkv, int d, int causal, int window, double scale,
+                           double *dq, double *dk, double *dv)
+{
+    if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
+    const int group = Hq / Hkv;
+    int64_t maxlen = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
+        if (L < 0) return -1;
+        if (L > maxlen) maxlen = L;
+    }
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sc = (double *)malloc(sizeof(double) * n);
+        double *p = (double *)malloc(sizeof(double) * n);
+        double *dp = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dod = (double *)malloc(sizeof(double) * (size_t)d);
+        double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
+        unsigned char *vis = (unsigned char *)malloc(n);
+        if (!sc || !p || !dp || !qd || !dod || !orow || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < (int64_t)num_seqs * Hkv; ++task) {
+                int seq = (int)(task / Hkv), g = (int)(task % Hkv);
+                int64_t start = cu_seqlens[seq];
+                int64_t L = (int64_t)cu_seqlens[seq + 1] - start;
+                for (int64_t j = 0; j < L; ++j) {
+                    kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
+                    vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
+                    for (int c = 0; c < d; ++c) {
+                        dk[((start + j) * Hkv + g) * (int64_t)d + c] = 0.0;
+                        dv[((start + j) * Hkv + g) * (int64_t)d + c] = 0.0;
+                    }
+                }
+                for (int h = g * group; h < (g + 1) * group; ++h) {
+                    for (int64_t i = 0; i < L; ++i) {
+                        const int64_t row = ((start + i) * Hq + h) * (int64_t)d;
+                        double lse_i, D = 0.0;
+                        for (int c = 0; c < d; ++c) {
+                            qd[c] = widen(q[row + c]);
+                            dod[c] = widen(dout[row + c]);
+                        }
+                        for (int64_t j = 0; j < L; ++j)
+                            vis[j] = (unsigned char)allowed(i, j, causal, window);
+                        attend_row(qd, d, L, kp, vp, vis, scale, sc, orow, &lse_i, p);
+                        /* dP and the Jacobian term D_i */
+                        for (int64_t j = 0; j < L; ++j) {
+                            dp[j] = 0.0;
+                            if (!vis[j]) continue;
+                            for (int c = 0; c < d; ++c) dp[j] += dod[c] * widen(vp[j][c]);
+                            D += p[j] * dp[j];
+                        }
+                        for (int c = 0; c < d; ++c) dq[row + c] = 0.0;
+                        for (int64_t j = 0; j < L; ++j) {
+                            if (!vis[j]) continue;
+                            const double ds = p[j] * (dp[j] - D);
+                            double *dkj = dk + ((start + j) * Hkv + g) * (int64_t)d;
+                            double *dvj = dv + ((start + j) * Hkv + g) * (int64_t)d;
+                            for (int c = 0; c < d; ++c) {
+                                dq[row + c] += scale * ds * widen(kp[j][c]);
+                                dkj[c] += scale * ds * qd[c];
+                                dvj[c] += p[j] * dod[c];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        free(sc); free(p); free(dp); free(qd); free(dod); free(orow);
+        free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
