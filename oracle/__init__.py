@@ -50,10 +50,23 @@ def lib():
         L.oracle_lse_combine.argtypes = [_f64p, _f64p, ctypes.c_int, ctypes.c_int64,
                                          ctypes.c_int, _f64p, _f64p]
         L.oracle_lse_combine.restype = ctypes.c_int
+        L.oracle_attn_varlen_rows_sinks.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _f64p,
+            ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
+        L.oracle_attn_varlen_rows_sinks.restype = ctypes.c_int
+        L.oracle_decode_paged_sinks.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_int64, ctypes.c_double, _f64p, _f64p, _f64p]
+        L.oracle_decode_paged_sinks.restype = ctypes.c_int
         L.oracle_attn_bwd_varlen.argtypes = [
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _f64p, _f64p, _f64p]
         L.oracle_attn_bwd_varlen.restype = ctypes.c_int
+        L.oracle_attn_bwd_dq_rows.argtypes = [
+            _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
+        L.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -215,3 +228,74 @@ def attn_bwd(q, k, v, dout, causal=False, window=0, scale=None):
                                  vb.reshape(B * N, Hkv, d), db.reshape(B * N, Hq, d), cu,
                                  causal, window, scale)
     return (dq.reshape(B, N, Hq, d), dk.reshape(B, N, Hkv, d), dv.reshape(B, N, Hkv, d))
+
+
+def attn_bwd_dq_rows(q, k, v, dout, cu_seqlens, rows, causal=False, window=0, scale=None):
+    """dQ of the packed tokens ``rows`` only (all query heads) -> [R, Hq, d]."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.empty((r.size, Hq, d), np.float64)
+    _check(lib().oracle_attn_bwd_dq_rows(qb, kb, vb, db, cu, len(cu) - 1, Hq, Hkv, d,
+                                         int(causal), int(window), float(scale), r, r.size, dq),
+           "attn_bwd_dq_rows")
+    return dq
+
+
+def attn_varlen_sinks(q, k, v, cu_seqlens, sinks, causal=False, window=0, scale=None, rows=None):
+    """attn_varlen with a learned sink logit per query head (``sinks`` [Hq],
+    in units of scaled scores): the sink joins each row's softmax denominator
+    as one extra key with a zero value.  Returns O and LSE as attn_varlen."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(Hq))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        nrows, rp = T, None
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows, rp = r.size, r.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((nrows, Hq, d), np.float64)
+    lse = np.empty((nrows, Hq), np.float64)
+    _check(lib().oracle_attn_varlen_rows_sinks(qb, kb, vb, cu, len(cu) - 1, Hq, Hkv, d,
+                                               int(causal), int(window), float(scale), sk,
+                                               rp, nrows, o, lse), "attn_varlen_sinks")
+    if rows is None:
+        return o, np.ascontiguousarray(lse.T)
+    return o, lse
+
+
+def attn_sinks(q, k, v, sinks, causal=False, window=0, scale=None):
+    """Dense batch with sinks -> O [B,N,Hq,d], LSE [B,Hq,N]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    o, lse = attn_varlen_sinks(qb.reshape(B * N, Hq, d), kb.reshape(B * N, Hkv, d),
+                               vb.reshape(B * N, Hkv, d), cu, sinks, causal, window, scale)
+    return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(Hq, B, N).transpose(1, 0, 2))
+
+
+def decode_paged_sinks(q, k_cache, v_cache, block_table, seq_lens, sinks, scale=None):
+    """decode_paged with a learned sink logit per query head."""
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    S, Hq, d = qb.shape
+    P, ps, Hkv, _ = kb.shape
+    bt = _i32(block_table)
+    sl = _i32(seq_lens)
+    sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(Hq))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((S, Hq, d), np.float64)
+    lse = np.empty((S, Hq), np.float64)
+    _check(lib().oracle_decode_paged_sinks(qb, kb, vb, bt, sl, S, Hq, Hkv, d, ps,
+                                           bt.shape[1], P, float(scale), sk, o, lse),
+           "decode_paged_sinks")
+    return o, lse

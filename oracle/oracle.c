@@ -87,12 +87,14 @@ static int allowed(int64_t i, int64_t j, int causal, int window)
 /*
  * One output row.  keys[j] / vals[j] point at the d-vector of key / value j;
  * vis[j] says whether key j is in A(i).  s is scratch of length nkeys.
+ * `sink` is a per-head logit that joins the softmax denominator as the score
+ * of one extra key whose value is zero (-INFINITY: no sink).
  * Writes o[0..d) and *lse; optionally the probability row p[0..nkeys).
  */
-static void attend_row(const double *q, int d, int64_t nkeys,
-                       const uint16_t *const *keys, const uint16_t *const *vals,
-                       const unsigned char *vis, double scale,
-                       double *s, double *o, double *lse, double *p)
+static void attend_row_sink(const double *q, int d, int64_t nkeys,
+                            const uint16_t *const *keys, const uint16_t *const *vals,
+                            const unsigned char *vis, double scale, double sink,
+                            double *s, double *o, double *lse, double *p)
 {
     int64_t j;
     int c;
@@ -108,17 +110,19 @@ static void attend_row(const double *q, int d, int64_t nkeys,
         any = 1;
     }
     for (c = 0; c < d; ++c) o[c] = 0.0;
-    if (!any) {
+    if (!any && sink == -INFINITY) {
         *lse = -INFINITY;
         if (p) for (j = 0; j < nkeys; ++j) p[j] = 0.0;
         return;
     }
-    /* 2. row max, then the denominator */
+    /* 2. row max (the sink counts as a score), then the denominator */
     for (j = 0; j < nkeys; ++j)
         if (vis[j] && s[j] > m) m = s[j];
+    if (sink > m) m = sink;
     for (j = 0; j < nkeys; ++j)
         if (vis[j]) l += exp(s[j] - m);
-    /* 3. probabilities times values */
+    if (sink != -INFINITY) l += exp(sink - m);
+    /* 3. probabilities times values (the sink's value is zero) */
     for (j = 0; j < nkeys; ++j) {
         double pj = vis[j] ? exp(s[j] - m) / l : 0.0;
         if (p) p[j] = pj;
@@ -127,6 +131,14 @@ static void attend_row(const double *q, int d, int64_t nkeys,
     }
     /* 4. log-sum-exp */
     *lse = m + log(l);
+}
+
+static void attend_row(const double *q, int d, int64_t nkeys,
+                       const uint16_t *const *keys, const uint16_t *const *vals,
+                       const unsigned char *vis, double scale,
+                       double *s, double *o, double *lse, double *p)
+{
+    attend_row_sink(q, d, nkeys, keys, vals, vis, scale, -INFINITY, s, o, lse, p);
 }
 
 /*
@@ -138,11 +150,11 @@ static void attend_row(const double *q, int d, int64_t nkeys,
  * Returns 0, or -1 on a bad argument (a row outside every sequence, Hq not a
  * multiple of Hkv, ...).
  */
-int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                            const int32_t *cu_seqlens, int num_seqs,
-                            int Hq, int Hkv, int d, int causal, int window,
-                            double scale, const int64_t *rows, int64_t nrows,
-                            double *o, double *lse)
+static int attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  const int32_t *cu_seqlens, int num_seqs,
+                                  int Hq, int Hkv, int d, int causal, int window,
+                                  double scale, const double *sinks, const int64_t *rows,
+                                  int64_t nrows, double *o, double *lse)
 {
     if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
     const int group = Hq / Hkv;
@@ -189,13 +201,40 @@ int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t
                     vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
                     vis[j] = (unsigned char)allowed(i, j, causal, window);
                 }
-                attend_row(qd, d, L, kp, vp, vis, scale, s,
-                           o + (r * Hq + h) * (int64_t)d, lse + r * Hq + h, NULL);
+                attend_row_sink(qd, d, L, kp, vp, vis, scale, sinks ? sinks[h] : -INFINITY, s,
+                                o + (r * Hq + h) * (int64_t)d, lse + r * Hq + h, NULL);
             }
         }
         free(s); free(qd); free(kp); free(vp); free(vis);
     }
     return bad ? -2 : 0;
+}
+
+int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *cu_seqlens, int num_seqs,
+                            int Hq, int Hkv, int d, int causal, int window,
+                            double scale, const int64_t *rows, int64_t nrows,
+                            double *o, double *lse)
+{
+    return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
+                                  scale, NULL, rows, nrows, o, lse);
+}
+
+/*
+ * The same with a learned sink logit per query head, sinks[Hq] (in units of
+ * scaled scores), joining every row's softmax denominator as the score of
+ * one extra key with a zero value ("Sliding windows and local:global
+ * layers": gpt-oss's learned sink per head).  LSE includes the sink's term.
+ */
+int oracle_attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  const int32_t *cu_seqlens, int num_seqs,
+                                  int Hq, int Hkv, int d, int causal, int window,
+                                  double scale, const double *sinks, const int64_t *rows,
+                                  int64_t nrows, double *o, double *lse)
+{
+    if (!sinks) return -1;
+    return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
+                                  scale, sinks, rows, nrows, o, lse);
 }
 
 /* Dense batch: q [B,N,Hq,d], k/v [B,N,Hkv,d]; o [B,N,Hq,d]; lse [B,Hq,N]. */
@@ -261,11 +300,11 @@ int oracle_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  *   q [S, Hq, d]; k_cache/v_cache [num_pages, page_size, Hkv, d]
  *   o [S, Hq, d]; lse [S, Hq]
  */
-int oracle_decode_paged(const uint16_t *q, const uint16_t *k_cache,
-                        const uint16_t *v_cache, const int32_t *block_table,
-                        const int32_t *seq_lens, int S, int Hq, int Hkv, int d,
-                        int page_size, int max_pages, int64_t num_pages,
-                        double scale, double *o, double *lse)
+static int decode_paged_sinks(const uint16_t *q, const uint16_t *k_cache,
+                              const uint16_t *v_cache, const int32_t *block_table,
+                              const int32_t *seq_lens, int S, int Hq, int Hkv, int d,
+                              int page_size, int max_pages, int64_t num_pages,
+                              double scale, const double *sinks, double *o, double *lse)
 {
     if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || page_size <= 0) return -1;
     int64_t maxlen = 0;
@@ -303,13 +342,35 @@ int oracle_decode_paged(const uint16_t *q, const uint16_t *k_cache,
                     vp[j] = v_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
                     vis[j] = (unsigned char)allowed(L - 1, j, 1, 0);
                 }
-                attend_row(qd, d, L, kp, vp, vis, scale, sb,
-                           o + task * d, lse + task, NULL);
+                attend_row_sink(qd, d, L, kp, vp, vis, scale, sinks ? sinks[h] : -INFINITY,
+                                sb, o + task * d, lse + task, NULL);
             }
         }
         free(sb); free(qd); free(kp); free(vp); free(vis);
     }
     return bad ? -2 : 0;
+}
+
+int oracle_decode_paged(const uint16_t *q, const uint16_t *k_cache,
+                        const uint16_t *v_cache, const int32_t *block_table,
+                        const int32_t *seq_lens, int S, int Hq, int Hkv, int d,
+                        int page_size, int max_pages, int64_t num_pages,
+                        double scale, double *o, double *lse)
+{
+    return decode_paged_sinks(q, k_cache, v_cache, block_table, seq_lens, S, Hq, Hkv, d,
+                              page_size, max_pages, num_pages, scale, NULL, o, lse);
+}
+
+/* Paged decode with a learned sink logit per query head (sinks[Hq]). */
+int oracle_decode_paged_sinks(const uint16_t *q, const uint16_t *k_cache,
+                              const uint16_t *v_cache, const int32_t *block_table,
+                              const int32_t *seq_lens, int S, int Hq, int Hkv, int d,
+                              int page_size, int max_pages, int64_t num_pages,
+                              double scale, const double *sinks, double *o, double *lse)
+{
+    if (!sinks) return -1;
+    return decode_paged_sinks(q, k_cache, v_cache, block_table, seq_lens, S, Hq, Hkv, d,
+                              page_size, max_pages, num_pages, scale, sinks, o, lse);
 }
 
 /*
@@ -359,6 +420,33 @@ int oracle_lse_combine(const double *o_parts, const double *lse_parts,
  * Each (sequence, KV head) is one task that owns its dK/dV rows; sums run in
  * a fixed order (query head, then row, ascending), independent of threads.
  */
+/*
+ * One query row of the backward: given q_i, dO_i and the key/value rows of
+ * its sequence, fills p[j] = P_ij and ds[j] = dS_ij (0 outside A(i)) and
+ * dq[c] = scale sum_j dS_ij K_j[c].  Scratch: sc, dp (length nkeys), orow (d).
+ */
+static void bwd_row(const double *qd, const double *dod, int d, int64_t nkeys,
+                    const uint16_t *const *kp, const uint16_t *const *vp,
+                    const unsigned char *vis, double scale, double *sc, double *p,
+                    double *dp, double *ds, double *orow, double *dq)
+{
+    double lse_i, D = 0.0;
+    attend_row(qd, d, nkeys, kp, vp, vis, scale, sc, orow, &lse_i, p);
+    /* dP and the Jacobian term D_i */
+    for (int64_t j = 0; j < nkeys; ++j) {
+        dp[j] = 0.0;
+        if (!vis[j]) continue;
+        for (int c = 0; c < d; ++c) dp[j] += dod[c] * widen(vp[j][c]);
+        D += p[j] * dp[j];
+    }
+    for (int c = 0; c < d; ++c) dq[c] = 0.0;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        ds[j] = vis[j] ? p[j] * (dp[j] - D) : 0.0;
+        if (!vis[j]) continue;
+        for (int c = 0; c < d; ++c) dq[c] += scale * ds[j] * widen(kp[j][c]);
+    }
+}
+
 int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                            const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
                            int Hq, int Hkv, int d, int causal, int window, double scale,
@@ -379,13 +467,14 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
         double *sc = (double *)malloc(sizeof(double) * n);
         double *p = (double *)malloc(sizeof(double) * n);
         double *dp = (double *)malloc(sizeof(double) * n);
+        double *ds = (double *)malloc(sizeof(double) * n);
         double *qd = (double *)malloc(sizeof(double) * (size_t)d);
         double *dod = (double *)malloc(sizeof(double) * (size_t)d);
         double *orow = (double *)malloc(sizeof(double) * (size_t)d);
         const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
         const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
         unsigned char *vis = (unsigned char *)malloc(n);
-        if (!sc || !p || !dp || !qd || !dod || !orow || !kp || !vp || !vis) {
+        if (!sc || !p || !dp || !ds || !qd || !dod || !orow || !kp || !vp || !vis) {
 #pragma omp atomic write
             bad = 1;
         } else {
@@ -405,30 +494,20 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
                 for (int h = g * group; h < (g + 1) * group; ++h) {
                     for (int64_t i = 0; i < L; ++i) {
                         const int64_t row = ((start + i) * Hq + h) * (int64_t)d;
-                        double lse_i, D = 0.0;
                         for (int c = 0; c < d; ++c) {
                             qd[c] = widen(q[row + c]);
                             dod[c] = widen(dout[row + c]);
                         }
                         for (int64_t j = 0; j < L; ++j)
                             vis[j] = (unsigned char)allowed(i, j, causal, window);
-                        attend_row(qd, d, L, kp, vp, vis, scale, sc, orow, &lse_i, p);
-                        /* dP and the Jacobian term D_i */
-                        for (int64_t j = 0; j < L; ++j) {
-                            dp[j] = 0.0;
-                            if (!vis[j]) continue;
-                            for (int c = 0; c < d; ++c) dp[j] += dod[c] * widen(vp[j][c]);
-                            D += p[j] * dp[j];
-                        }
-                        for (int c = 0; c < d; ++c) dq[row + c] = 0.0;
+                        bwd_row(qd, dod, d, L, kp, vp, vis, scale, sc, p, dp, ds, orow,
+                                dq + row);
                         for (int64_t j = 0; j < L; ++j) {
                             if (!vis[j]) continue;
-                            const double ds = p[j] * (dp[j] - D);
                             double *dkj = dk + ((start + j) * Hkv + g) * (int64_t)d;
                             double *dvj = dv + ((start + j) * Hkv + g) * (int64_t)d;
                             for (int c = 0; c < d; ++c) {
-                                dq[row + c] += scale * ds * widen(kp[j][c]);
-                                dkj[c] += scale * ds * qd[c];
+                                dkj[c] += scale * ds[j] * qd[c];
                                 dvj[c] += p[j] * dod[c];
                             }
                         }
@@ -436,7 +515,74 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
                 }
             }
         }
-        free(sc); free(p); free(dp); free(qd); free(dod); free(orow);
+        free(sc); free(p); free(dp); free(ds); free(qd); free(dod); free(orow);
+        free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * dQ of selected query tokens only (every query head): rows[r] is a packed
+ * token index; dq [nrows, Hq, d].  Each row needs only its own row of P, so
+ * this stays cheap at any sequence length.
+ */
+int oracle_attn_bwd_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                            int Hq, int Hkv, int d, int causal, int window, double scale,
+                            const int64_t *rows, int64_t nrows, double *dq)
+{
+    if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0 || nrows < 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t total = cu_seqlens[num_seqs];
+    int64_t maxlen = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
+        if (L < 0) return -1;
+        if (L > maxlen) maxlen = L;
+    }
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sc = (double *)malloc(sizeof(double) * n);
+        double *p = (double *)malloc(sizeof(double) * n);
+        double *dp = (double *)malloc(sizeof(double) * n);
+        double *ds = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dod = (double *)malloc(sizeof(double) * (size_t)d);
+        double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
+        unsigned char *vis = (unsigned char *)malloc(n);
+        if (!sc || !p || !dp || !ds || !qd || !dod || !orow || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < nrows * (int64_t)Hq; ++task) {
+                int64_t r = task / Hq, t = rows[r];
+                int h = (int)(task % Hq), g = h / group;
+                int seq = 0;
+                while (seq < num_seqs && cu_seqlens[seq + 1] <= t) ++seq;
+                int64_t start = cu_seqlens[seq];
+                int64_t L = (int64_t)cu_seqlens[seq + 1] - start, i = t - start;
+                const int64_t row = (t * Hq + h) * (int64_t)d;
+                for (int c = 0; c < d; ++c) {
+                    qd[c] = widen(q[row + c]);
+                    dod[c] = widen(dout[row + c]);
+                }
+                for (int64_t j = 0; j < L; ++j) {
+                    kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
+                    vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
+                    vis[j] = (unsigned char)allowed(i, j, causal, window);
+                }
+                bwd_row(qd, dod, d, L, kp, vp, vis, scale, sc, p, dp, ds, orow,
+                        dq + (r * Hq + h) * (int64_t)d);
+            }
+        }
+        free(sc); free(p); free(dp); free(ds); free(qd); free(dod); free(orow);
         free(kp); free(vp); free(vis);
     }
     return bad ? -2 : 0;

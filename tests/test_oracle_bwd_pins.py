@@ -145,3 +145,17 @@ def test_backward_thread_count_does_not_change_bits():
         oracle.set_num_threads(n0)
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
+
+
+def test_dq_rows_match_full_backward():
+    """The row-sampled dQ equals the pinned full backward on the same rows."""
+    lens = [40, 0, 77]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv, d = int(cu[-1]), 4, 2, 32
+    q, k, v = rnd((T, Hq, d), 41), rnd((T, Hkv, d), 42), rnd((T, Hkv, d), 43)
+    do = rnd((T, Hq, d), 44)
+    for causal, window in ((0, 0), (1, 0), (1, 9)):
+        dq, _, _ = oracle.attn_bwd_varlen(q, k, v, do, cu, causal, window, 0.3)
+        rows = [0, 5, 39, 40, 41, 100, 116]
+        got = oracle.attn_bwd_dq_rows(q, k, v, do, cu, rows, causal, window, 0.3)
+        assert np.array_equal(got, dq[rows])
