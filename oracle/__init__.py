@@ -59,6 +59,14 @@ def lib():
             _u16p, _u16p, _u16p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_int64, ctypes.c_double, _f64p, _f64p, _f64p]
         L.oracle_decode_paged_sinks.restype = ctypes.c_int
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        _u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+        _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+        L.oracle_decode_paged_fp8.argtypes = [
+            _u16p, _u8p, _u8p, _f32p, _f32p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, _f64p, _f64p]
+        L.oracle_decode_paged_fp8.restype = ctypes.c_int
         L.oracle_attn_bwd_varlen.argtypes = [
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _f64p, _f64p, _f64p]
@@ -298,4 +306,45 @@ def decode_paged_sinks(q, k_cache, v_cache, block_table, seq_lens, sinks, scale=
     _check(lib().oracle_decode_paged_sinks(qb, kb, vb, bt, sl, S, Hq, Hkv, d, ps,
                                            bt.shape[1], P, float(scale), sk, o, lse),
            "decode_paged_sinks")
+    return o, lse
+
+
+def e4m3_value(code: int) -> float:
+    """The real value of one FP8 E4M3 ("fn") code."""
+    return float(lib().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def _u8(x) -> np.ndarray:
+    if not isinstance(x, np.ndarray):
+        import torch
+        x = x.detach().cpu().contiguous()
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    return np.ascontiguousarray(x, dtype=np.uint8)
+
+
+def decode_paged_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                     sinks=None):
+    """Paged decode over an FP8 (E4M3) cache.  k_codes/v_codes [P,ps,Hkv,d] uint8 codes
+    (or torch float8_e4m3fn), k_scale/v_scale [P,Hkv] fp32 -> O [S,Hq,d], LSE [S,Hq]."""
+    qb = _bits(q)
+    kc, vc = _u8(k_codes), _u8(v_codes)
+    S, Hq, d = qb.shape
+    P, ps, Hkv, _ = kc.shape
+    ks = np.ascontiguousarray(np.asarray(k_scale, dtype=np.float32).reshape(P, Hkv))
+    vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float32).reshape(P, Hkv))
+    bt = _i32(block_table)
+    sl = _i32(seq_lens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    sp = None
+    if sinks is not None:
+        sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(Hq))
+        sp = sk.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((S, Hq, d), np.float64)
+    lse = np.empty((S, Hq), np.float64)
+    _check(lib().oracle_decode_paged_fp8(qb, kc, vc, ks, vs, bt, sl, S, Hq, Hkv, d, ps,
+                                         bt.shape[1], P, float(scale), sp, o, lse),
+           "decode_paged_fp8")
     return o, lse

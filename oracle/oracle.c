@@ -587,3 +587,114 @@ int oracle_attn_bwd_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t
     }
     return bad ? -2 : 0;
 }
+
+/*
+ * FP8 KV cache ("FP8 KV cache is a routine flag": the "Paging and prefix
+ * sharing" neighbourhood of the same post stores the cache in fewer bits).
+ * Codes are OCP FP8 E4M3 in its "fn" form (no infinities): sign bit, 4
+ * exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ * subnormals m/8 * 2^-6; S.1111.111 is NaN.  A cached value is
+ * e4m3(code) * scale, with one fp32 scale per (page, KV head).
+ */
+double oracle_e4m3_value(uint8_t code)
+{
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/*
+ * One row over FP8 keys and values: keys[j]/vals[j] point at d codes,
+ * ks[j]/vs[j] are their dequantisation scales.  Same steps as
+ * attend_row_sink with K_j = e4m3(code) * ks[j], V_j = e4m3(code) * vs[j].
+ */
+static void attend_row_fp8(const double *q, int d, int64_t nkeys,
+                           const uint8_t *const *keys, const uint8_t *const *vals,
+                           const double *ks, const double *vs, double scale, double sink,
+                           double *s, double *o, double *lse)
+{
+    int64_t j;
+    int c;
+    double m = -INFINITY, l = 0.0;
+    for (c = 0; c < d; ++c) o[c] = 0.0;
+    for (j = 0; j < nkeys; ++j) {
+        double acc = 0.0;
+        for (c = 0; c < d; ++c) acc += q[c] * (oracle_e4m3_value(keys[j][c]) * ks[j]);
+        s[j] = scale * acc;
+    }
+    if (nkeys == 0 && sink == -INFINITY) { *lse = -INFINITY; return; }
+    for (j = 0; j < nkeys; ++j)
+        if (s[j] > m) m = s[j];
+    if (sink > m) m = sink;
+    for (j = 0; j < nkeys; ++j) l += exp(s[j] - m);
+    if (sink != -INFINITY) l += exp(sink - m);
+    for (j = 0; j < nkeys; ++j) {
+        const double pj = exp(s[j] - m) / l;
+        for (c = 0; c < d; ++c) o[c] += pj * (oracle_e4m3_value(vals[j][c]) * vs[j]);
+    }
+    *lse = m + log(l);
+}
+
+/*
+ * Paged decode over an FP8 cache: k_cache/v_cache [num_pages, page_size,
+ * Hkv, d] E4M3 codes; k_scale/v_scale [num_pages, Hkv] fp32; sinks [Hq] or
+ * NULL.  Otherwise as oracle_decode_paged.
+ */
+int oracle_decode_paged_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                            const float *k_scale, const float *v_scale,
+                            const int32_t *block_table, const int32_t *seq_lens, int S,
+                            int Hq, int Hkv, int d, int page_size, int max_pages,
+                            int64_t num_pages, double scale, const double *sinks, double *o,
+                            double *lse)
+{
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || page_size <= 0) return -1;
+    int64_t maxlen = 0;
+    for (int s = 0; s < S; ++s) {
+        if (seq_lens[s] < 0 || seq_lens[s] > (int64_t)max_pages * page_size) return -1;
+        if (seq_lens[s] > maxlen) maxlen = seq_lens[s];
+        for (int64_t p = 0; p < ((int64_t)seq_lens[s] + page_size - 1) / page_size; ++p) {
+            int32_t pg = block_table[(int64_t)s * max_pages + p];
+            if (pg < 0 || pg >= num_pages) return -1;
+        }
+    }
+    const int group = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sb = (double *)malloc(sizeof(double) * n);
+        double *ksr = (double *)malloc(sizeof(double) * n);
+        double *vsr = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint8_t **kp = (const uint8_t **)malloc(sizeof(void *) * n);
+        const uint8_t **vp = (const uint8_t **)malloc(sizeof(void *) * n);
+        if (!sb || !ksr || !vsr || !qd || !kp || !vp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < (int64_t)S * Hq; ++task) {
+                int s = (int)(task / Hq), h = (int)(task % Hq), g = h / group;
+                int64_t L = seq_lens[s];
+                for (int c = 0; c < d; ++c) qd[c] = widen(q[((int64_t)s * Hq + h) * d + c]);
+                for (int64_t j = 0; j < L; ++j) {
+                    int64_t pg = block_table[(int64_t)s * max_pages + j / page_size];
+                    int64_t slot = j % page_size;
+                    kp[j] = k_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    vp[j] = v_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    ksr[j] = (double)k_scale[pg * Hkv + g];
+                    vsr[j] = (double)v_scale[pg * Hkv + g];
+                }
+                attend_row_fp8(qd, d, L, kp, vp, ksr, vsr, scale,
+                               sinks ? sinks[h] : -INFINITY, sb, o + task * d, lse + task);
+            }
+        }
+        free(sb); free(ksr); free(vsr); free(qd); free(kp); free(vp);
+    }
+    return bad ? -2 : 0;
+}

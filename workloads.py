@@ -176,6 +176,44 @@ def paged(lens=None, num_seqs=64, len_lo=4096, len_hi=32768, Hq=32, Hkv=8,
                  pages_used=used)
 
 
+@dataclass
+class PagedFP8:
+    q: torch.Tensor            # [S, Hq, d] bf16
+    k_codes: torch.Tensor      # [num_pages, page_size, Hkv, d] uint8 (FP8 E4M3 codes)
+    v_codes: torch.Tensor
+    k_scale: torch.Tensor      # [num_pages, Hkv] fp32
+    v_scale: torch.Tensor
+    block_table: torch.Tensor
+    seq_lens: torch.Tensor
+    page_size: int
+    scale: float
+    pages_used: int = 0
+
+
+def _quantize_e4m3(x: torch.Tensor, pow2: bool):
+    """Per-(page, KV head) scale = amax / 448 (rounded up to a power of two
+    with ``pow2``), codes = the round-to-nearest-even E4M3 of x / scale
+    (torch's float8_e4m3fn conversion).  NaN inputs stay NaN codes."""
+    xf = x.float()
+    amax = torch.nan_to_num(xf.abs(), nan=0.0).amax(dim=(1, 3))          # [P, Hkv]
+    sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    if pow2:
+        sc = torch.exp2(torch.ceil(torch.log2(sc)))
+    codes = (xf / sc[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, sc.to(torch.float32).contiguous()
+
+
+def paged_fp8(pow2_scales=False, **kw) -> PagedFP8:
+    """The paged workload of ``paged(**kw)`` with its cache stored as FP8
+    E4M3 codes and one fp32 scale per (page, KV head): the same draws, then
+    quantised (a storage format of the input, not attention arithmetic)."""
+    b = paged(**kw)
+    kc, ks = _quantize_e4m3(b.k_cache, pow2_scales)
+    vc, vs = _quantize_e4m3(b.v_cache, pow2_scales)
+    return PagedFP8(b.q, kc, vc, ks, vs, b.block_table, b.seq_lens, b.page_size, b.scale,
+                    b.pages_used)
+
+
 def make(name: str, seed: int = 0, **over):
     """Inputs of one named workload (CPU tensors)."""
     cfg = dict(CONFIGS[name])
@@ -189,6 +227,14 @@ def make(name: str, seed: int = 0, **over):
     if kind == "decode":
         return paged(seed=seed, **cfg)
     raise ValueError(kind)
+
+
+def grad_out(shape, seed=0) -> torch.Tensor:
+    """The upstream gradient dO of a backward workload: iid N(0,1) in bf16
+    from a generator of its own, seeded with ``seed + 1`` (so the forward
+    inputs drawn with ``seed`` are unchanged)."""
+    g = torch.Generator("cpu").manual_seed(seed + 1)
+    return randn_bf16(tuple(shape), g)
 
 
 def bf16_bits(t: torch.Tensor):
