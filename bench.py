@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     # profiling aids (the default run times both kernels on the named workloads)
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the extension rows (backward, FP8-cache decode)")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one kernel family only (for profiler captures)")
     ap.add_argument("--prefill-workload", default=PREFILL,
@@ -304,6 +306,14 @@ def bench_ours(args):
     if err:
         raise RuntimeError(f"device error in timed region: {fa.status_string(err)}")
 
+    # ---- extension rows, timed on their own after the step (same inputs):
+    # the backward of the prefill and the decode over an FP8 copy of the cache
+    nxt = {}
+    if not args.no_next and args.only == "all":
+        nxt = bench_next(fa, args, dev, stream, flush, pk, traffic_all=recorded_traffic(),
+                         pin=pin, q=q, k=k, v=v, o=o, lse=lse, flops=flops, din=din,
+                         dq=dq, dk=dk, dv=dv, dbt=dbt, dsl=dsl, ws=ws, dout=dout, dlse=dlse)
+
     # ---- end to end through the public API with host buffers
     hq, hk, hv = (t.pin_memory() for t in (pin.q, pin.k, pin.v))
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -382,6 +392,7 @@ def bench_ours(args):
                 "what": "fa_fwd through the Python binding: pinned host q,k,v -> device, "
                         "kernel, O and LSE -> host, per step"},
         "gpu_launches": (int(do_p) + 2 * int(do_d)) * K,
+        "next": nxt,
         "clocks": clk.report(),
         "wall_s_timed_region": round(t_wall, 3),
         "kernel_source": kernel_source_hash(),
@@ -397,6 +408,85 @@ def bench_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, lse, flops,
+               din, dq, dk, dv, dbt, dsl, ws, dout, dlse):
+    """The rows built beyond the headline path, each timed with CUDA events
+    over K calls (L2 flushed before each), with its own roofline:
+      bwd        -- fa_bwd on the prefill workload: FLOPs = 2.5 x the forward's
+                    (five GEMMs of the forward's size per tile against two);
+      decode_fp8 -- fa_decode_paged_fp8 over the decode workload's cache stored
+                    as FP8 E4M3 with a scale per (page, KV head): KV bytes halve.
+    """
+    K = args.steps
+    out = {}
+
+    def timed(fn):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks([sum(a.elapsed_time(b) for a, b in evs)], dev)[0] / K
+
+    # backward: O and LSE from the forward, a seeded upstream gradient
+    fa.fwd(q, k, v, True, pin.window, pin.scale, out=o, lse=lse)
+    g = workloads.grad_out(tuple(q.shape), seed=args.seed).to(dev)
+    gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    B, N, Hq, d = q.shape
+    wsb = torch.empty(fa.bwd_workspace_bytes(B * N, Hq, d), dtype=torch.uint8, device=dev)
+    ms = timed(lambda: fa.bwd(q, k, v, o, g, lse, True, pin.window, pin.scale, gq, gk, gv, wsb))
+    bflops = 2.5 * flops
+    ach = bflops / (ms * 1e-3) / 1e12
+    out["bwd"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+                  "flop_per_call": bflops, "launches_per_call": 3,
+                  "workload": "backward of the prefill workload (dQ, dK, dV), causal",
+                  "roofline": {"bound": "tensor", "achieved": round(ach, 2),
+                               "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                               "frac": round(ach / pk["bf16_tflops"], 4),
+                               "kernel": "bwd_kernel (+ bwd_prep_kernel, bwd_convert_kernel)",
+                               "traffic": traffic_all.get("bwd_gqa4k")}}
+    del g, gq, gk, gv, wsb
+
+    # FP8 cache: quantised on the device from the bf16 cache (input preparation)
+    def quant(x):
+        amax = x.float().abs().amax(dim=(1, 3))
+        sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).float().contiguous()
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+        step = 4096
+        for i in range(0, x.shape[0], step):
+            codes[i:i + step] = (x[i:i + step].float() / sc[i:i + step, None, :, None]).to(
+                torch.float8_e4m3fn).view(torch.uint8)
+        return codes, sc
+    kc8, ks8 = quant(dk)
+    vc8, vs8 = quant(dv)
+    ms = timed(lambda: fa.decode_paged_fp8(dq, kc8, vc8, ks8, vs8, dbt, dsl, din.scale,
+                                           out=dout, lse=dlse, workspace=ws))
+    tokens = float(din.seq_lens.sum().item())
+    kv8 = tokens * dk.shape[2] * dk.shape[3] * 1 * 2
+    ach = kv8 / (ms * 1e-3) / 1e9
+    out["decode_fp8"] = {"value": round(ach, 1), "unit": "GB/s", "ms_per_call": round(ms, 4),
+                         "kv_bytes": kv8, "tokens_per_s": round(tokens / (ms * 1e-3), 1),
+                         "launches_per_call": 2,
+                         "workload": "decode workload with its cache as FP8 E4M3 + scales",
+                         "roofline": {"bound": "hbm", "achieved": round(ach, 1),
+                                      "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                      "frac": round(ach / pk["hbm_gbs"], 4),
+                                      "kernel": "decode_split_kernel<128,4,fp8> + combine",
+                                      "traffic": traffic_all.get("decode_fp8_decode64")}}
+    del kc8, vc8, ks8, vs8
+    err = fa.check_device_error()
+    if err:
+        raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
+    return out
 
 
 # ---------------------------------------------------------------- reference

@@ -9,8 +9,11 @@ shared library is missing or fails to load, importing this package raises.
 Functions mirror the C entry points:
     fwd            -> fa_fwd            (dense prefill)
     fwd_varlen     -> fa_fwd_varlen     (packed sequences, cu_seqlens)
+    bwd            -> fa_bwd            (dense backward: dQ, dK, dV)
+    bwd_varlen     -> fa_bwd_varlen     (packed-sequence backward)
     decode_paged   -> fa_decode_paged   (paged split-KV decode)
-    decode_workspace_bytes, check_device_error, status_string, version
+    decode_paged_noalloc, decode_workspace_bytes, bwd_workspace_bytes,
+    check_device_error, selftest_watchdog, status_string, version
 """
 from __future__ import annotations
 
@@ -33,7 +36,10 @@ FA_ERR_TIMEOUT = -6
 FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
-EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_decode_workspace_bytes", "fa_decode_paged",
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks",
+           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen",
+           "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
+           "fa_decode_paged_fp8",
            "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
            "fa_selftest_watchdog", "fa_version")
 
@@ -55,6 +61,20 @@ def _load():
     lib.fa_fwd.restype = i
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp] + [i] * 8 + [f, i, vp]
     lib.fa_fwd_varlen.restype = i
+    lib.fa_fwd_sinks.argtypes = [vp] * 6 + [i] * 7 + [f, i, vp]
+    lib.fa_fwd_sinks.restype = i
+    lib.fa_fwd_varlen_sinks.argtypes = [vp] * 7 + [i] * 8 + [f, i, vp]
+    lib.fa_fwd_varlen_sinks.restype = i
+    lib.fa_decode_paged_sinks.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_decode_paged_sinks.restype = i
+    lib.fa_decode_paged_fp8.argtypes = [vp] * 10 + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_decode_paged_fp8.restype = i
+    lib.fa_bwd_workspace_bytes.argtypes = [i] * 3
+    lib.fa_bwd_workspace_bytes.restype = sz
+    lib.fa_bwd.argtypes = [vp] * 9 + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_varlen.argtypes = [vp] * 10 + [i] * 8 + [f, vp, sz, vp]
+    lib.fa_bwd_varlen.restype = i
     lib.fa_decode_workspace_bytes.argtypes = [i] * 5
     lib.fa_decode_workspace_bytes.restype = sz
     lib.fa_decode_paged.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
@@ -115,8 +135,9 @@ def _need(t, dtype, ndim, name):
 
 
 def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
-        out=None, lse=None, return_lse=True, stream=None):
-    """Dense prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 -> (O [B,N,Hq,d], LSE [B,Hq,N])."""
+        out=None, lse=None, return_lse=True, stream=None, sinks=None):
+    """Dense prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 -> (O [B,N,Hq,d], LSE [B,Hq,N]).
+    ``sinks`` (fp32 [Hq], device) selects fa_fwd_sinks."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, 4, n)
     B, N, Hq, d = q.shape
@@ -130,13 +151,20 @@ def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+        _check(_lib.fa_fwd_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(sinks),
+                                 B, Hq, Hkv, N, d, int(causal), int(window), float(scale), od,
+                                 _stream(stream)), "fa_fwd_sinks")
+        return out, lse
     _check(_lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
                        int(causal), int(window), float(scale), od, _stream(stream)), "fa_fwd")
     return out, lse
 
 
 def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=None,
-               out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None):
+               out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None,
+               sinks=None):
     """Packed prefill.  q [T,Hq,d], k/v [T,Hkv,d], cu_seqlens [S+1] int32 (device)
     -> (O [T,Hq,d], LSE [Hq,T])."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -151,11 +179,77 @@ def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=No
     if lse is None and return_lse:
         lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
     od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+        _check(_lib.fa_fwd_varlen_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                        _ptr(sinks), _ptr(cu_seqlens), cu_seqlens.numel() - 1,
+                                        T, int(max_seqlen), Hq, Hkv, d, int(causal),
+                                        int(window), float(scale), od, _stream(stream)),
+               "fa_fwd_varlen_sinks")
+        return out, lse
     _check(_lib.fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                               _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, int(max_seqlen),
                               Hq, Hkv, d, int(causal), int(window), float(scale), od,
                               _stream(stream)), "fa_fwd_varlen")
     return out, lse
+
+
+def bwd_workspace_bytes(total_tokens, Hq, d) -> int:
+    return int(_lib.fa_bwd_workspace_bytes(int(total_tokens), int(Hq), int(d)))
+
+
+def bwd(q, k, v, o, dout, lse, causal=False, window=0, scale=None, dq=None, dk=None, dv=None,
+        workspace=None, stream=None):
+    """Dense backward.  q/o/dout [B,N,Hq,d], k/v [B,N,Hkv,d] bf16, lse [B,Hq,N] fp32
+    (from fwd) -> (dQ, dK, dV) bf16."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, torch.bfloat16, 4, n)
+    _need(lse, torch.float32, 3, "lse")
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if (tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d)
+            or tuple(o.shape) != (B, N, Hq, d) or tuple(dout.shape) != (B, N, Hq, d)
+            or tuple(lse.shape) != (B, Hq, N)):
+        raise FAError(FA_ERR_INVALID_ARG, "bwd shapes")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(B * N, Hq, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                       _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, int(causal), int(window),
+                       float(scale), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_varlen(q, k, v, o, dout, lse, cu_seqlens, max_seqlen, causal=False, window=0,
+               scale=None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Packed backward.  q/o/dout [T,Hq,d], k/v [T,Hkv,d], lse [Hq,T], cu_seqlens [S+1]
+    -> (dQ, dK, dV) bf16."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, torch.bfloat16, 3, n)
+    _need(lse, torch.float32, 2, "lse")
+    _need(cu_seqlens, torch.int32, 1, "cu_seqlens")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(T, Hq, d), 1), dtype=torch.uint8,
+                                device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(_lib.fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens),
+                              cu_seqlens.numel() - 1, T, int(max_seqlen), Hq, Hkv, d,
+                              int(causal), int(window), float(scale), _ptr(workspace),
+                              workspace.numel(), _stream(stream)), "fa_bwd_varlen")
+    return dq, dk, dv
 
 
 def decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq) -> int:
@@ -164,7 +258,7 @@ def decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq) -> int
 
 
 def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=None, lse=None,
-                 return_lse=True, workspace=None, stream=None):
+                 return_lse=True, workspace=None, stream=None, sinks=None):
     """Paged decode.  q [S,Hq,d], caches [P,ps,Hkv,d], block_table [S,maxp] int32,
     seq_lens [S] int32 -> (O [S,Hq,d] bf16, LSE [S,Hq])."""
     _need(q, torch.bfloat16, 3, "q")
@@ -184,11 +278,57 @@ def decode_paged(q, k_cache, v_cache, block_table, seq_lens, scale=None, out=Non
         out = torch.empty((S, Hq, d), dtype=torch.bfloat16, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+        _check(_lib.fa_decode_paged_sinks(_ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                                          _ptr(lse), _ptr(sinks), S, P, Hq, Hkv, d, ps, maxp,
+                                          float(scale), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)), "fa_decode_paged_sinks")
+        return out, lse
     _check(_lib.fa_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                 _ptr(seq_lens), _ptr(out), _ptr(lse), S, P, Hq, Hkv, d, ps,
                                 maxp, float(scale), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(),
                                 _stream(stream)), "fa_decode_paged")
+    return out, lse
+
+
+def decode_paged_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_lens, scale=None,
+                     sinks=None, out=None, lse=None, return_lse=True, workspace=None,
+                     stream=None):
+    """Paged decode over an FP8 E4M3 cache.  k_codes/v_codes [P,ps,Hkv,d] uint8 (or
+    float8_e4m3fn), k_scale/v_scale [P,Hkv] fp32 -> (O [S,Hq,d] bf16, LSE [S,Hq])."""
+    _need(q, torch.bfloat16, 3, "q")
+    if k_codes.dtype == torch.float8_e4m3fn:
+        k_codes, v_codes = k_codes.view(torch.uint8), v_codes.view(torch.uint8)
+    _need(k_codes, torch.uint8, 4, "k_codes")
+    _need(v_codes, torch.uint8, 4, "v_codes")
+    _need(k_scale, torch.float32, 2, "k_scale")
+    _need(v_scale, torch.float32, 2, "v_scale")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(seq_lens, torch.int32, 1, "seq_lens")
+    S, Hq, d = q.shape
+    P, ps, Hkv, _ = k_codes.shape
+    maxp = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = decode_workspace_bytes(S, Hq, d, ps, maxp)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((S, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+    _check(_lib.fa_decode_paged_fp8(_ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_scale),
+                                    _ptr(v_scale), _ptr(block_table), _ptr(seq_lens), _ptr(out),
+                                    _ptr(lse), _ptr(sinks), S, P, Hq, Hkv, d, ps, maxp,
+                                    float(scale), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    _stream(stream)), "fa_decode_paged_fp8")
     return out, lse
 
 

@@ -1,0 +1,641 @@
+// bwd_sm100.cu -- exact attention backward (dQ, dK, dV) on the sm_100a tensor
+// core.
+//
+// What it computes: for O = softmax(Q K^T * scale + mask) V and an upstream
+// gradient dO, the gradients of sum(dO * O) with respect to Q, K and V.  The
+// attention matrix is never stored: it is recomputed from Q, K and the row
+// log-sum-exp the forward saved ("FlashAttention: same math, different IO" in
+// samanvya.dev's "Attention Is the Bottleneck": the backward pass recomputes
+// the matrix from Q, K, V and the saved softmax statistics).  With
+// D_i = dO_i . O_i, for each visible (query i, key j):
+//     P_ij  = 2^(S_ij * scale * log2e - LSE_i * log2e)
+//     dS_ij = P_ij (dO_i . V_j - D_i)
+//     dV_j += P_ij dO_i,   dK_j += scale dS_ij Q_i,   dQ_i += scale dS_ij K_j
+// and grouped query heads add into their shared KV head's dK, dV.
+//
+// How (B200 design):
+//   * bwd_prep_kernel: D = rowsum(O * dO) per (token, head), and zeroes the
+//     fp32 dQ accumulator.
+//   * bwd_kernel, persistent, one CTA per SM.  A work unit is one KV head's
+//     block of 128 keys; K_j and V_j stay in shared memory while the unit walks
+//     every (query head of the group, 64-row query tile) that sees the block.
+//     dK_j and dV_j accumulate in tensor memory for the whole unit, so the GQA
+//     sum over query heads costs nothing and each unit writes its rows once.
+//   * Per tile, five tcgen05 GEMMs, all with the 128 keys on the TMEM lanes:
+//       S^T  = K_j Q_t^T        (128 x 64, K = d)
+//       dP^T = V_j dO_t^T       (128 x 64, K = d)
+//       dV  += P^T dO_t         (128 x d,  K = 64; P^T read from TMEM)
+//       dK  += dS^T Q_t         (128 x d,  K = 64; dS^T from shared memory)
+//       dQ^T = K_j^T dS^T       (d x 64,   K = 128; lands on dP^T's columns)
+//     S^T and dP^T are double-buffered in TMEM (2 x 2 x 64 columns) and dK, dV
+//     take 2 x 128: the 512 columns of the SM.  Two softmax warpgroups take
+//     alternate tiles, so one tile's elementwise work overlaps the next tile's
+//     GEMMs.
+//   * Warps 8-11 drain dQ^T from TMEM, stage it transposed in shared memory
+//     and add it into the fp32 accumulator with TMA reduce-adds (the adds
+//     happen in L2, 16 KB per operation); bwd_convert_kernel rounds the
+//     accumulator to bf16 at the end.
+//   * Warp 12 loads K_j, V_j once per unit and Q_t, dO_t per tile by TMA into
+//     a 3-slot ring, with the tile's LSE (in log2 units) and D beside them;
+//     warp 13 (one thread) issues every MMA and owns the TMEM allocation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+namespace bwd_impl {
+
+constexpr int kD = 128;
+constexpr int kBlockK = 128;   // keys per unit
+constexpr int kBlockQ = 64;    // queries per tile
+constexpr int kThreads = 512;
+constexpr int kWarpDrain = 8;  // warps 8..11
+constexpr int kWarpTma = 12;
+constexpr int kWarpMma = 13;
+constexpr int kStages = 3;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;     // S^T of buffer b at b * 64 (P^T overwrites its first 32)
+constexpr uint32_t kColDP = 128;  // dP^T of buffer b at 128 + b * 64, then the tile's dQ^T
+constexpr uint32_t kColDV = 256;
+constexpr uint32_t kColDK = 384;
+
+constexpr int kKVBox = kBlockK * 64 * 2;         // 128 rows x 64 bf16 (16 KB)
+constexpr int kKVTile = kBlockK * kD * 2;        // 32 KB
+constexpr int kQBox = kBlockQ * 64 * 2;          // 64 rows x 64 bf16 (8 KB)
+constexpr int kQTile = kBlockQ * kD * 2;         // 16 KB
+constexpr int kDSBytes = kBlockK * kBlockQ * 2;  // 16 KB
+constexpr int kOffK = 0;
+constexpr int kOffV = kKVTile;
+constexpr int kOffStage = 2 * kKVTile;           // stage s: Q_t then dO_t
+constexpr int kStageBytes = 2 * kQTile;
+constexpr int kOffDS = kOffStage + kStages * kStageBytes;
+constexpr int kDQHalf = 32;                      // dQ rows per reduce-add
+constexpr int kDQBytes = kDQHalf * kD * 4;       // 16 KB staging buffer
+constexpr int kOffDQ = kOffDS + 2 * kDSBytes;    // two staging buffers
+constexpr int kOffRows = kOffDQ + 2 * kDQBytes;  // stage s: lse2[64], D[64] (fp32)
+constexpr int kSmemBytes = kOffRows + kStages * 2 * kBlockQ * 4 + 1024;
+static_assert(kSmemBytes + 256 <= 232448, "shared memory");
+constexpr int kBarDrain = 1;                     // named barrier of the dQ warps
+
+struct Params {
+    const float *lse;   // saved row log-sum-exp (natural log)
+    const float *dd;    // D = rowsum(O * dO), same layout as lse
+    float *dq_acc;      // [total, Hq, d] fp32
+    void *dk, *dv;      // [total, Hkv, d] bf16
+    const int *cu_seqlens;
+    int num_seqs, seqlen, total_tokens;
+    int Hq, Hkv, group;
+    int causal, window;
+    float scale, scale_log2;
+    int num_kblocks, num_units;
+};
+
+struct Unit {
+    int seq, kvh, tok0, L;
+    int j0, jl;        // first and last key of the block (local to the sequence)
+    int t_lo, nt;      // query tiles [t_lo, t_lo + nt) of each query head
+    int ntiles;        // group * nt
+};
+
+__device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
+    const int per = p.num_seqs * p.Hkv;
+    const int jb = u / per;           // causal: low key blocks are the heaviest
+    const int r = u % per;
+    w.seq = r / p.Hkv;
+    w.kvh = r % p.Hkv;
+    if (p.cu_seqlens) {
+        w.tok0 = __ldg(p.cu_seqlens + w.seq);
+        w.L = __ldg(p.cu_seqlens + w.seq + 1) - w.tok0;
+    } else {
+        w.tok0 = w.seq * p.seqlen;
+        w.L = p.seqlen;
+    }
+    w.j0 = jb * kBlockK;
+    if (w.L <= 0 || w.j0 >= w.L) return false;
+    w.jl = min(w.L, w.j0 + kBlockK) - 1;
+    const int nq = (w.L + kBlockQ - 1) / kBlockQ;
+    int lo = 0, hi = nq;
+    if (p.causal) {
+        lo = w.j0 / kBlockQ;                        // queries i >= j0
+        if (p.window > 0) hi = min(nq, (w.jl + p.window - 1) / kBlockQ + 1);  // i < jl + W
+    }
+    w.t_lo = lo;
+    w.nt = hi - lo;
+    w.ntiles = p.group * w.nt;
+    return w.nt > 0;
+}
+
+__device__ __forceinline__ void tile_of(const Unit &w, const Params &p, int k, int &h, int &q0) {
+    h = w.kvh * p.group + k / w.nt;
+    q0 = (w.t_lo + k % w.nt) * kBlockQ;
+}
+
+__device__ __forceinline__ size_t row_index(const Params &p, const Unit &w, int h, int i) {
+    return p.cu_seqlens ? (size_t)h * p.total_tokens + w.tok0 + i
+                        : ((size_t)w.seq * p.Hq + h) * p.seqlen + i;
+}
+
+__device__ __forceinline__ int sched_unit(int it) {
+    const int G = gridDim.x, b = blockIdx.x;
+    return (it & 1) ? (it + 1) * G - 1 - b : it * G + b;
+}
+
+#define FOR_EACH_UNIT(u)                                                  \
+    for (int it_ = 0, u = 0; it_ * (int)gridDim.x < p.num_units; ++it_)   \
+        if ((u = sched_unit(it_)) < p.num_units)
+
+struct Shared {
+    uint64_t kv_full, kv_empty;
+    uint64_t qd_full[kStages], qd_empty[kStages];
+    uint64_t s_full[2], p_full[2], dq_full[2], dq_free[2];
+    uint64_t acc_full, acc_free;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ------------------------------------------------------------- TMA producer
+__device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                         const CUtensorMap *tmdO, const Params &p, Shared &sh, uint8_t *smem) {
+    volatile int *abort = &sh.abort;
+    const int lane = lane_id();
+    float *rows = reinterpret_cast<float *>(smem + kOffRows);
+    uint32_t uc = 0, n = 0;
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        if (!mbar_wait_warp(&sh.kv_empty, (uc & 1) ^ 1, abort)) goto out;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&sh.kv_full, 2 * kKVTile);
+            for (int b = 0; b < kD / 64; ++b) {
+                tma_load_3d(smem + kOffK + b * kKVBox, tmK, &sh.kv_full, b * 64, w.kvh, w.tok0 + w.j0);
+                tma_load_3d(smem + kOffV + b * kKVBox, tmV, &sh.kv_full, b * 64, w.kvh, w.tok0 + w.j0);
+            }
+        }
+        ++uc;
+        for (int k = 0; k < w.ntiles; ++k, ++n) {
+            const int s = n % kStages;
+            if (!mbar_wait_warp(&sh.qd_empty[s], ((n / kStages) & 1) ^ 1, abort)) goto out;
+            int h, q0;
+            tile_of(w, p, k, h, q0);
+            if (lane == 0) {
+                uint8_t *st = smem + kOffStage + s * kStageBytes;
+                mbar_arrive_expect_tx(&sh.qd_full[s], 2 * kQTile);
+                for (int b = 0; b < kD / 64; ++b) {
+                    tma_load_3d(st + b * kQBox, tmQ, &sh.qd_full[s], b * 64, h, w.tok0 + q0);
+                    tma_load_3d(st + kQTile + b * kQBox, tmdO, &sh.qd_full[s], b * 64, h, w.tok0 + q0);
+                }
+            }
+            // The tile's LSE (log2 units) and D; rows past the sequence get
+            // LSE = +inf, so their P is exactly 0.
+            float *rs = rows + s * 2 * kBlockQ;
+            #pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int rr = lane + 32 * e, i = q0 + rr;
+                float l2 = INFINITY, dv = 0.f;
+                if (i < w.L) {
+                    const size_t idx = row_index(p, w, h, i);
+                    l2 = __ldg(p.lse + idx) * 1.4426950408889634f;
+                    dv = __ldg(p.dd + idx);
+                }
+                rs[rr] = l2;
+                rs[kBlockQ + rr] = dv;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.qd_full[s]);
+        }
+    }
+    return;
+out:
+    if (lane == 0) {
+        if (uc) mbar_drain_wait(&sh.kv_full, (uc - 1) & 1);
+        for (int s = 0; s < kStages; ++s)
+            if (n > (uint32_t)s) mbar_drain_wait(&sh.qd_full[s], ((n - 1 - s) / kStages) & 1);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+__device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
+    volatile int *abort = &sh.abort;
+    const uint32_t tmem = sh.tmem_base;
+    const uint32_t idS = idesc_bf16_f32_ab(kBlockK, kBlockQ, false, false);
+    const uint32_t idAcc = idesc_bf16_f32_ab(kBlockK, kD, false, true);
+    const uint32_t idDQ = idesc_bf16_f32_ab(kD, kBlockQ, true, true);
+    const uint32_t aK = smem_u32(smem + kOffK), aV = smem_u32(smem + kOffV);
+    const uint32_t aStage = smem_u32(smem + kOffStage), aDS = smem_u32(smem + kOffDS);
+    uint32_t uc = 0, n = 0;
+
+    // S^T(b) = K Q^T and dP^T(b) = V dO^T: K-major operands, d/16 steps; a
+    // step moves 32 bytes inside a 64-column box, 4 steps cross to the next box.
+    auto issue_s_dp = [&](int b, int s) {
+        const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+        #pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
+            const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
+            mma_ss(tmem + kColS + b * kBlockQ, smem_desc_sw128(aK + okv, 16, 1024),
+                   smem_desc_sw128(q + oq, 16, 1024), idS, ks > 0);
+        }
+        #pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
+            const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
+            mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aV + okv, 16, 1024),
+                   smem_desc_sw128(dO + oq, 16, 1024), idS, ks > 0);
+        }
+    };
+    // dV += P^T dO, dK += dS^T Q (K = 64 queries), then dQ^T = K^T dS^T (K = 128 keys).
+    // dO and Q are MN-major B operands (d contiguous; 16 query rows per step,
+    // boxes of 64 columns LBO apart); dS^T sits in shared memory as 128 key rows
+    // of 64 queries, 128-byte swizzled: K-major A for dK, MN-major B for dQ^T.
+    auto issue_grads = [&](int m, bool first) -> bool {
+        const int b = m & 1, s = m % kStages;
+        if (!mbar_wait(&sh.p_full[b], (m >> 1) & 1, abort)) return false;
+        if (first && uc > 1)
+            if (!mbar_wait(&sh.acc_free, (uc - 2) & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+        const uint32_t ds = aDS + b * kDSBytes;
+        #pragma unroll
+        for (int ks = 0; ks < kBlockQ / 16; ++ks)
+            mma_ts(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
+                   smem_desc_sw128(dO + ks * 2048, kQBox, 1024), idAcc, (ks > 0 || !first) ? 1u : 0u);
+        #pragma unroll
+        for (int ks = 0; ks < kBlockQ / 16; ++ks)
+            mma_ss(tmem + kColDK, smem_desc_sw128(ds + ks * 32, 16, 1024),
+                   smem_desc_sw128(q + ks * 2048, kQBox, 1024), idAcc, (ks > 0 || !first) ? 1u : 0u);
+        tc_commit(&sh.qd_empty[s]);
+        #pragma unroll
+        for (int ks = 0; ks < kBlockK / 16; ++ks)
+            mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aK + ks * 2048, kKVBox, 1024),
+                   smem_desc_sw128(ds + ks * 2048, kDSBytes, 1024), idDQ, ks > 0);
+        tc_commit(&sh.dq_full[b]);
+        return true;
+    };
+
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        if (!mbar_wait(&sh.kv_full, uc & 1, abort)) goto out;
+        ++uc;
+        for (int k = 0; k < w.ntiles; ++k, ++n) {
+            const int b = n & 1, s = n % kStages;
+            if (!mbar_wait(&sh.qd_full[s], (n / kStages) & 1, abort)) goto out;
+            if (n >= 2 && !mbar_wait(&sh.dq_free[b], ((n - 2) >> 1) & 1, abort)) goto out;
+            tc_fence_after();
+            issue_s_dp(b, s);
+            tc_commit(&sh.s_full[b]);
+            if (k > 0 && !issue_grads(n - 1, k == 1)) goto out;
+        }
+        if (!issue_grads(n - 1, w.ntiles == 1)) goto out;
+        tc_commit(&sh.kv_empty);
+        tc_commit(&sh.acc_full);
+    }
+out:
+    tc_commit(&sh.drain);
+    mbar_drain_wait(&sh.drain, 0);
+}
+
+// ---------------------------------------------------- softmax-gradient warps
+__device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
+    volatile int *abort = &sh.abort;
+    const int warp = warp_id(), lane = lane_id();
+    const int wg = warp >> 2;                  // takes tiles n with n % 2 == wg
+    const int r = (warp & 3) * 32 + lane;      // key row of the block
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = sh.tmem_base + lanes + kColS + wg * kBlockQ;
+    const uint32_t tdP = sh.tmem_base + lanes + kColDP + wg * kBlockQ;
+    const float *rows = reinterpret_cast<const float *>(smem + kOffRows);
+    uint8_t *dsb = smem + kOffDS + wg * kDSBytes + r * 128;
+    const float sl2 = p.scale_log2;
+    uint32_t n = 0, uc = 0;
+
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        const int kj = w.j0 + r;                  // this thread's key
+        const bool key_ok = kj < w.L;
+        for (int k = 0; k < w.ntiles; ++k, ++n) {
+            if ((int)(n & 1) != wg) continue;
+            const int s = n % kStages;
+            if (!mbar_wait_warp(&sh.s_full[wg], (n >> 1) & 1, abort)) return;
+            if (!mbar_wait_warp(&sh.qd_full[s], (n / kStages) & 1, abort)) return;
+            tc_fence_after();
+            int h, q0;
+            tile_of(w, p, k, h, q0);
+            (void)h;
+            const float *l2 = rows + s * 2 * kBlockQ;
+            const float *dd = l2 + kBlockQ;
+            const int qmax = min(q0 + kBlockQ, w.L) - 1;
+            const bool edge = (w.j0 + kBlockK > w.L) || (p.causal && w.jl > q0) ||
+                              (p.window > 0 && w.j0 <= qmax - p.window);
+            #pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32(tS + hh * 32, sr);
+                tmem_ld32(tdP + hh * 32, dr);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+                #pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const int cc = hh * 32 + c;
+                    float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2[cc]));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, -l2[cc + 1]));
+                    if (edge) {
+                        const int i0 = q0 + cc, i1 = i0 + 1;
+                        bool v0 = key_ok, v1 = key_ok;
+                        if (p.causal) {
+                            v0 = v0 && kj <= i0 && (p.window <= 0 || kj > i0 - p.window);
+                            v1 = v1 && kj <= i1 && (p.window <= 0 || kj > i1 - p.window);
+                        }
+                        p0 = v0 ? p0 : 0.f;
+                        p1 = v1 ? p1 : 0.f;
+                    }
+                    const float d0 = p0 * (__uint_as_float(dr[c]) - dd[cc]);
+                    const float d1 = p1 * (__uint_as_float(dr[c + 1]) - dd[cc + 1]);
+                    pk[c >> 1] = pack_bf16(p0, p1);
+                    dk[c >> 1] = pack_bf16(d0, d1);
+                }
+                tmem_st16(tS + hh * 16, pk);
+                // dS^T row r, queries hh*32 .. hh*32+31: four 16-byte chunks,
+                // chunk index XOR (row & 7) (128-byte swizzle)
+                #pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int chunk = hh * 4 + c4;
+                    uint4 v = make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
+                    *reinterpret_cast<uint4 *>(dsb + ((chunk ^ (r & 7)) << 4)) = v;
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.p_full[wg]);
+        }
+        // ---- unit end: warpgroup 0 writes dV, warpgroup 1 writes scale * dK
+        if (!mbar_wait_warp(&sh.acc_full, uc & 1, abort)) return;
+        ++uc;
+        tc_fence_after();
+        const uint32_t tAcc = sh.tmem_base + lanes + (wg ? kColDK : kColDV);
+        const float mul = wg ? p.scale : 1.f;
+        uint16_t *dst = static_cast<uint16_t *>(wg ? p.dk : p.dv) +
+                        ((size_t)(w.tok0 + kj) * p.Hkv + w.kvh) * kD;
+        #pragma unroll
+        for (int c = 0; c < kD; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tAcc + c, v);
+            tmem_wait_ld();
+            if (key_ok) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+                #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    uint4 o;
+                    o.x = pack_bf16(__uint_as_float(v[8 * e + 0]) * mul, __uint_as_float(v[8 * e + 1]) * mul);
+                    o.y = pack_bf16(__uint_as_float(v[8 * e + 2]) * mul, __uint_as_float(v[8 * e + 3]) * mul);
+                    o.z = pack_bf16(__uint_as_float(v[8 * e + 4]) * mul, __uint_as_float(v[8 * e + 5]) * mul);
+                    o.w = pack_bf16(__uint_as_float(v[8 * e + 6]) * mul, __uint_as_float(v[8 * e + 7]) * mul);
+                    d4[e] = o;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.acc_free);
+    }
+}
+
+// ------------------------------------------------------------- dQ drain
+// dQ^T of a tile (lane = d index, column = query) is read from TMEM, scaled,
+// written transposed into a shared-memory staging buffer (32 query rows x d,
+// fp32) and added into the global accumulator by one TMA reduce-add per 32
+// rows; two staging buffers alternate so the next rows are written while the
+// previous reduce still reads.  Rows past the sequence add exact zeros (their
+// P, hence dS, is 0).
+__device__ void dq_drain(const CUtensorMap *tmDQ, const Params &p, Shared &sh, uint8_t *smem) {
+    volatile int *abort = &sh.abort;
+    const int warp = warp_id(), lane = lane_id();
+    const int c = (warp & 3) * 32 + lane;       // d index (TMEM lane of dQ^T)
+    const bool leader = (warp == kWarpDrain && lane == 0);
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    float *stage = reinterpret_cast<float *>(smem + kOffDQ);
+    uint32_t n = 0, hs = 0;
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        for (int k = 0; k < w.ntiles; ++k, ++n) {
+            const int b = n & 1;
+            const bool ok = mbar_wait_warp(&sh.dq_full[b], (n >> 1) & 1, abort);
+            if (!named_bar_and(kBarDrain, 128, ok)) goto out;
+            tc_fence_after();
+            uint32_t v[64];
+            const uint32_t t = sh.tmem_base + lanes + kColDP + b * kBlockQ;
+            tmem_ld32(t, v);
+            tmem_ld32(t + 32, v + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.dq_free[b]);
+            int h, q0;
+            tile_of(w, p, k, h, q0);
+            #pragma unroll
+            for (int half = 0; half < 2; ++half, ++hs) {
+                float *buf = stage + (hs & 1) * (kDQHalf * kD);
+                if (leader) bulk_wait_group_read<1>();   // the reduce that used buf is done reading
+                named_bar_sync(kBarDrain, 128);
+                #pragma unroll
+                for (int i = 0; i < kDQHalf; ++i)
+                    buf[i * kD + c] = __uint_as_float(v[half * kDQHalf + i]) * p.scale;
+                fence_proxy_async_smem();
+                named_bar_sync(kBarDrain, 128);
+                if (leader) {
+                    tma_reduce_add_3d(tmDQ, buf, 0, h, w.tok0 + q0 + half * kDQHalf);
+                    bulk_commit_group();
+                }
+            }
+        }
+    }
+out:
+    if (leader) bulk_wait_group_all();
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+           const __grid_constant__ CUtensorMap tmDQ, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Shared sh;
+    const uint32_t base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (base & 1023)) & 1023);
+    const int warp = warp_id();
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sh.kv_full, 1);
+        mbar_init(&sh.kv_empty, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.qd_full[s], 2);   // TMA bytes + the LSE/D rows
+            mbar_init(&sh.qd_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.s_full[b], 1);
+            mbar_init(&sh.p_full[b], 4);
+            mbar_init(&sh.dq_full[b], 1);
+            mbar_init(&sh.dq_free[b], 4);
+        }
+        mbar_init(&sh.acc_full, 1);
+        mbar_init(&sh.acc_free, 8);
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) tmem_alloc(&sh.tmem_base, kTmemCols);
+    if (warp == kWarpTma && lane_id() == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+        tma_prefetch_desc(&tmDQ);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp < 8) {
+        softmax_wg(p, sh, smem);
+    } else if (warp < 12) {
+        dq_drain(&tmDQ, p, sh, smem);
+    } else if (warp == kWarpTma) {
+        producer(&tmQ, &tmK, &tmV, &tmdO, p, sh, smem);
+    } else if (warp == kWarpMma) {
+        if (lane_id() == 0) mma_issuer(p, sh, smem);
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(sh.tmem_base, kTmemCols);
+    }
+}
+
+// D = rowsum(O * dO) for every (token, query head), in the LSE layout; zeroes
+// the dQ accumulator.  One warp per row of d = 128 elements.
+__global__ void __launch_bounds__(256)
+bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dout,
+                float *__restrict__ dd, float *__restrict__ dq_acc, int total, int Hq,
+                int seqlen, int dense) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (long long)total * Hq) return;
+    const uint2 a = reinterpret_cast<const uint2 *>(o + row * kD)[lane];
+    const uint2 b = reinterpret_cast<const uint2 *>(dout + row * kD)[lane];
+    auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
+    auto hi = [](uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); };
+    float acc = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    reinterpret_cast<float4 *>(dq_acc + row * kD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0) {
+        const long long tok = row / Hq;
+        const int h = (int)(row % Hq);
+        size_t idx;
+        if (dense) {
+            const long long bseq = tok / seqlen, i = tok % seqlen;
+            idx = ((size_t)bseq * Hq + h) * seqlen + i;
+        } else {
+            idx = (size_t)h * total + tok;
+        }
+        dd[idx] = acc;
+    }
+}
+
+// dQ (bf16) = the fp32 accumulator, eight elements per thread.
+__global__ void __launch_bounds__(256)
+bwd_convert_kernel(const float *__restrict__ acc, uint16_t *__restrict__ dq, long long n8) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n8) return;
+    const float4 a = reinterpret_cast<const float4 *>(acc)[2 * i];
+    const float4 b = reinterpret_cast<const float4 *>(acc)[2 * i + 1];
+    uint4 o;
+    o.x = pack_bf16(a.x, a.y);
+    o.y = pack_bf16(a.z, a.w);
+    o.z = pack_bf16(b.x, b.y);
+    o.w = pack_bf16(b.z, b.w);
+    reinterpret_cast<uint4 *>(dq)[i] = o;
+}
+
+}  // namespace bwd_impl
+
+size_t bwd_workspace_bytes(long long total_tokens, int Hq, int d) {
+    if (total_tokens < 0 || Hq <= 0 || d != bwd_impl::kD) return 0;
+    const size_t acc = (size_t)total_tokens * Hq * d * sizeof(float);
+    const size_t dd = (size_t)total_tokens * Hq * sizeof(float);
+    return ((acc + 255) & ~(size_t)255) + ((dd + 255) & ~(size_t)255);
+}
+
+int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
+    using namespace bwd_impl;
+    if (a.d != kD) return -2;
+    const long long total = a.total_tokens;
+    if (total == 0 || a.num_seqs == 0) return 0;
+    const size_t acc_bytes = ((size_t)total * a.Hq * kD * sizeof(float) + 255) & ~(size_t)255;
+    float *dq_acc = static_cast<float *>(a.workspace);
+    float *dd = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) + acc_bytes);
+
+    const long long rows = total * a.Hq;
+    bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const uint16_t *>(a.o), static_cast<const uint16_t *>(a.dout), dd, dq_acc,
+        (int)total, a.Hq, a.seqlen, a.cu_seqlens ? 0 : 1);
+    if (cudaGetLastError() != cudaSuccess) return -5;
+
+    alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
+    const uint64_t T = (uint64_t)total;
+    if (encode_tensor_map_3d(&tq, a.q, 2, kD, a.Hq, T, (uint64_t)kD * 2, (uint64_t)a.Hq * kD * 2,
+                             64, 1, kBlockQ, true) ||
+        encode_tensor_map_3d(&tdo, a.dout, 2, kD, a.Hq, T, (uint64_t)kD * 2,
+                             (uint64_t)a.Hq * kD * 2, 64, 1, kBlockQ, true) ||
+        encode_tensor_map_3d(&tk, a.k, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
+                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, true) ||
+        encode_tensor_map_3d(&tv, a.v, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
+                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, true) ||
+        encode_tensor_map_3d(&tdq, dq_acc, 4, kD, a.Hq, T, (uint64_t)kD * 4,
+                             (uint64_t)a.Hq * kD * 4, kD, 1, kDQHalf, false))
+        return -5;
+    Params p;
+    p.lse = a.lse;
+    p.dd = dd;
+    p.dq_acc = dq_acc;
+    p.dk = a.dk;
+    p.dv = a.dv;
+    p.cu_seqlens = a.cu_seqlens;
+    p.num_seqs = a.num_seqs;
+    p.seqlen = a.seqlen;
+    p.total_tokens = (int)total;
+    p.Hq = a.Hq;
+    p.Hkv = a.Hkv;
+    p.group = a.Hq / a.Hkv;
+    p.causal = a.causal;
+    p.window = a.causal ? a.window : 0;
+    p.scale = a.scale;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.num_kblocks = (a.max_seqlen + kBlockK - 1) / kBlockK;
+    const long long units = (long long)p.num_kblocks * a.num_seqs * a.Hkv;
+    if (units > (1ll << 30)) return -2;
+    p.num_units = (int)units;
+    if (units > 0) {
+        if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes) != cudaSuccess)
+            return -5;
+        const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
+        bwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
+        if (cudaGetLastError() != cudaSuccess) return -5;
+    }
+    const long long n8 = total * a.Hq * kD / 8;
+    bwd_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<uint16_t *>(a.dq), n8);
+    return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+}  // namespace fa

@@ -46,6 +46,7 @@ struct DecodeParams {
     int HG, WPK, NW, num_hg, nst;
     uint32_t box_bytes;
     float scale_log2;
+    const float *k_scale, *v_scale;   // FP8 cache: [num_pages][Hkv] dequantisation scales
 };
 
 // Walks the flat unit index space (sequence-major, then head group, then
@@ -103,6 +104,41 @@ __device__ __forceinline__ void unpack8(uint4 a, float *f) {
     f[6] = __uint_as_float(a.w << 16); f[7] = __uint_as_float(a.w & 0xffff0000u);
 }
 
+// Two FP8 E4M3 codes (bits 0-7: the lower index) to a packed fp32 pair, by
+// way of the hardware e4m3x2 -> f16x2 conversion (exact: every E4M3 value
+// is an f16 value).
+__device__ __forceinline__ uint64_t e4m3x2_to_f2(uint32_t two) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
+    float lo, hi;
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}" : "=f"(lo), "=f"(hi) : "r"(h2));
+    return f2pack(lo, hi);
+}
+
+// N FP8 codes (N = 8 or 16, loaded as one 8- or 16-byte word) to N/2 pairs.
+template <int N>
+__device__ __forceinline__ void unpack_e4m3(const uint8_t *src, uint64_t *f) {
+    if constexpr (N == 16) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(src);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = e4m3x2_to_f2(w[i] & 0xffffu);
+            f[2 * i + 1] = e4m3x2_to_f2(w[i] >> 16);
+        }
+    } else {
+        const uint2 a = *reinterpret_cast<const uint2 *>(src);
+        const uint32_t w[2] = {a.x, a.y};
+        #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            f[2 * i] = e4m3x2_to_f2(w[i] & 0xffffu);
+            f[2 * i + 1] = e4m3x2_to_f2(w[i] >> 16);
+        }
+    }
+}
+
 // Sum NV values over the 8 lanes of a token group (xor 4, 2, 1), leaving
 // lane ds with the totals of flat indices [ds*NV/8, ...) (NV >= 8), or of
 // index ds*NV/8 shared by a lane pair (NV == 4).
@@ -140,7 +176,7 @@ constexpr int kDecRegsControl = 72;
 static_assert(2 * 128 * kDecRegsCompute + 128 * kDecRegsControl <= kDecThreads * 168,
               "register split");
 
-template <int D, int QPW>
+template <int D, int QPW, bool FP8>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const DecodeParams p) {
@@ -218,10 +254,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2);
         #pragma unroll
         for (int qh = 0; qh < QPW; ++qh) {
-            const uint16_t *qp = p.q + ((size_t)seq * p.Hq + h0 + qh) * D + 8 * ds;
+            // d slice of this lane: bf16 cache 8*ds + 64*b + (0..7); FP8 cache
+            // DPL*ds + (0..DPL-1), one 8- or 16-byte word of codes
+            const uint16_t *qp = p.q + ((size_t)seq * p.Hq + h0 + qh) * D +
+                                 (FP8 ? DPL * ds : 8 * ds);
             #pragma unroll
             for (int b = 0; b < DPL / 8; ++b) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qp + 64 * b));
+                const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(qp + (FP8 ? 8 : 64) * b));
                 unpack8x2(raw, &q2[qh][4 * b]);
             }
             #pragma unroll
@@ -238,7 +277,31 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         const int pages = (L + kPage - 1) / kPage;
         const int pg0 = chunk * kChunkPages, pg1 = min(pages, pg0 + kChunkPages);
+        // FP8: this KV head's dequantisation scales, fetched two pages ahead
+        // (page index first, the scales one page later) so the loads never
+        // stall the warp.
+        auto page_at = [&](int pg) {
+            const int page = __ldg(p.block_table + (size_t)seq * p.max_pages + pg);
+            return (page < 0 || page >= p.num_pages) ? 0 : page;
+        };
+        float ks_cur = 1.f, vs_cur = 1.f, ks_nxt = 1.f, vs_nxt = 1.f;
+        if constexpr (FP8) {
+            if (pg0 < pg1) {
+                const size_t i0 = (size_t)page_at(pg0) * p.Hkv + kvh;
+                ks_cur = __ldg(p.k_scale + i0);
+                vs_cur = __ldg(p.v_scale + i0);
+            }
+            if (pg0 + 1 < pg1) {
+                const size_t i1 = (size_t)page_at(pg0 + 1) * p.Hkv + kvh;
+                ks_nxt = __ldg(p.k_scale + i1);
+                vs_nxt = __ldg(p.v_scale + i1);
+            }
+        }
         for (int pg = pg0; pg < pg1; ++pg) {
+            int page2 = 0;
+            if constexpr (FP8) {
+                if (pg + 2 < pg1) page2 = page_at(pg + 2);
+            }
             const int st = it % p.nst;
             if (!mbar_wait_warp(&sh.full[st], (it / p.nst) & 1, abort)) return;
             ++it;
@@ -250,12 +313,16 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int t = tg + 4 * k;
-                const uint16_t *kr = reinterpret_cast<const uint16_t *>(sK) +
-                                     ((size_t)(t * p.HG + hl) * D + 8 * ds);
                 uint64_t kv2[DPL / 2];
-                #pragma unroll
-                for (int b = 0; b < DPL / 8; ++b)
-                    unpack8x2(*reinterpret_cast<const uint4 *>(kr + 64 * b), &kv2[4 * b]);
+                if constexpr (FP8) {
+                    unpack_e4m3<DPL>(sK + (size_t)(t * p.HG + hl) * D + DPL * ds, kv2);
+                } else {
+                    const uint16_t *kr = reinterpret_cast<const uint16_t *>(sK) +
+                                         ((size_t)(t * p.HG + hl) * D + 8 * ds);
+                    #pragma unroll
+                    for (int b = 0; b < DPL / 8; ++b)
+                        unpack8x2(*reinterpret_cast<const uint4 *>(kr + 64 * b), &kv2[4 * b]);
+                }
                 #pragma unroll
                 for (int qh = 0; qh < QPW; ++qh) {
                     uint64_t a0 = f2mul(q2[qh][0], kv2[0]);
@@ -279,7 +346,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const bool tok_ok = (tg + 4 * kslot) < nvalid;
             float s_own[HELD];
             #pragma unroll
-            for (int i = 0; i < HELD; ++i) s_own[i] = tok_ok ? sc[i] : -INFINITY;
+            for (int i = 0; i < HELD; ++i) s_own[i] = tok_ok ? (FP8 ? sc[i] * ks_cur : sc[i]) : -INFINITY;
             // ---- page max per head, known to every lane
             float pmax_own[HELD];
             #pragma unroll
@@ -345,15 +412,20 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 #pragma unroll
                 for (int qh = 0; qh < QPW; ++qh) l_acc[qh] += pr[k][qh];
                 if (t < nvalid) {   // slots past seq_len may hold anything
-                    const uint16_t *vr = reinterpret_cast<const uint16_t *>(sV) +
-                                         ((size_t)(t * p.HG + hl) * D + 8 * ds);
                     uint64_t vv2[DPL / 2];
-                    #pragma unroll
-                    for (int b = 0; b < DPL / 8; ++b)
-                        unpack8x2(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv2[4 * b]);
+                    if constexpr (FP8) {
+                        unpack_e4m3<DPL>(sV + (size_t)(t * p.HG + hl) * D + DPL * ds, vv2);
+                    } else {
+                        const uint16_t *vr = reinterpret_cast<const uint16_t *>(sV) +
+                                             ((size_t)(t * p.HG + hl) * D + 8 * ds);
+                        #pragma unroll
+                        for (int b = 0; b < DPL / 8; ++b)
+                            unpack8x2(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv2[4 * b]);
+                    }
                     #pragma unroll
                     for (int qh = 0; qh < QPW; ++qh) {
-                        const uint64_t pp = f2pack(pr[k][qh], pr[k][qh]);
+                        const float pv = FP8 ? pr[k][qh] * vs_cur : pr[k][qh];
+                        const uint64_t pp = f2pack(pv, pv);
                         #pragma unroll
                         for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2fma(pp, vv2[i], o2[qh][i]);
                     }
@@ -361,6 +433,15 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.empty[st]);
+            if constexpr (FP8) {
+                ks_cur = ks_nxt;
+                vs_cur = vs_nxt;
+                if (pg + 2 < pg1) {
+                    const size_t i2 = (size_t)page2 * p.Hkv + kvh;
+                    ks_nxt = __ldg(p.k_scale + i2);
+                    vs_nxt = __ldg(p.v_scale + i2);
+                }
+            }
         }
         // ---- merge the four token groups and write this chunk's partial
         float o[QPW][DPL];
@@ -381,10 +462,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             #pragma unroll
             for (int qh = 0; qh < QPW; ++qh) {
                 const float inv = l_acc[qh] > 0.f ? 1.f / l_acc[qh] : 0.f;
-                float *dst = p.part_o + (row0 + qh) * D + 8 * ds;
+                float *dst = p.part_o + (row0 + qh) * D + (FP8 ? DPL * ds : 8 * ds);
                 #pragma unroll
                 for (int b = 0; b < DPL / 8; ++b) {
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + 64 * b);
+                    float4 *d4 = reinterpret_cast<float4 *>(dst + (FP8 ? 8 : 64) * b);
                     d4[0] = make_float4(o[qh][8 * b + 0] * inv, o[qh][8 * b + 1] * inv,
                                         o[qh][8 * b + 2] * inv, o[qh][8 * b + 3] * inv);
                     d4[1] = make_float4(o[qh][8 * b + 4] * inv, o[qh][8 * b + 5] * inv,
@@ -409,8 +490,8 @@ template <int D>
 __global__ void __launch_bounds__(32 * kCombineWarps)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_lse,
                       const int *__restrict__ seq_lens, uint16_t *__restrict__ o,
-                      float *__restrict__ lse, int num_seqs, int Hq, int max_pages,
-                      int max_chunks) {
+                      float *__restrict__ lse, const float *__restrict__ sinks,
+                      int num_seqs, int Hq, int max_pages, int max_chunks) {
     constexpr int PER = D / 32;
     __shared__ float s_acc[kCombineWarps][D];
     __shared__ float s_w[kCombineWarps];
@@ -425,6 +506,9 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
     for (int c = lane; c < nc; c += 32) m = fmaxf(m, lse_p[(size_t)c * Hq]);
     #pragma unroll
     for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    // A learned sink is one more partial: LSE z, output zero.
+    const float z = sinks ? __ldg(sinks + h) : -INFINITY;
+    m = fmaxf(m, z);
     float acc[PER];
     #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
@@ -457,6 +541,7 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
     float tw = 0.f;
     #pragma unroll
     for (int w = 0; w < kCombineWarps; ++w) tw += s_w[w];
+    if (z != -INFINITY) tw += __expf(z - m);
     const float inv = tw > 0.f ? 1.f / tw : 0.f;
     float r[PER];
     #pragma unroll
@@ -479,7 +564,7 @@ struct Plan {
     int max_chunks;
 };
 
-bool make_plan(int Hq, int Hkv, int d, int max_pages, Plan &pl) {
+bool make_plan(int Hq, int Hkv, int d, int max_pages, int elem_bytes, Plan &pl) {
     if (Hkv <= 0 || Hq % Hkv) return false;
     const int g = Hq / Hkv;
     pl.QPW = (g % 4 == 0) ? 4 : (g % 2 == 0) ? 2 : 1;
@@ -491,7 +576,7 @@ bool make_plan(int Hq, int Hkv, int d, int max_pages, Plan &pl) {
         if (Hkv % c == 0) { pl.HG = c; break; }
     pl.NW = pl.HG * pl.WPK;
     pl.num_hg = Hkv / pl.HG;
-    pl.box_bytes = (uint32_t)(kPage * pl.HG * d * 2);
+    pl.box_bytes = (uint32_t)(kPage * pl.HG * d * elem_bytes);
     pl.nst = kSmemBudget / (2 * (int)pl.box_bytes);
     if (pl.nst > 8) pl.nst = 8;
     if (pl.nst < 2) return false;
@@ -501,15 +586,27 @@ bool make_plan(int Hq, int Hkv, int d, int max_pages, Plan &pl) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-template <int D, int QPW>
+template <int D, int QPW, bool FP8>
 int launch_split(const CUtensorMap &tk, const CUtensorMap &tv, const DecodeParams &p,
                  cudaStream_t stream) {
     const int smem = p.nst * 2 * (int)p.box_bytes + 128;
-    if (cudaFuncSetAttribute(decode_split_kernel<D, QPW>,
+    if (cudaFuncSetAttribute(decode_split_kernel<D, QPW, FP8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return -5;
-    decode_split_kernel<D, QPW><<<device_sm_count(), kDecThreads, smem, stream>>>(tk, tv, p);
+    decode_split_kernel<D, QPW, FP8><<<device_sm_count(), kDecThreads, smem, stream>>>(tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+template <bool FP8>
+int launch_split_d(int d, int qpw, const CUtensorMap &tk, const CUtensorMap &tv,
+                   const DecodeParams &p, cudaStream_t stream) {
+    if (d == 128)
+        return qpw == 4 ? launch_split<128, 4, FP8>(tk, tv, p, stream)
+             : qpw == 2 ? launch_split<128, 2, FP8>(tk, tv, p, stream)
+                        : launch_split<128, 1, FP8>(tk, tv, p, stream);
+    return qpw == 4 ? launch_split<64, 4, FP8>(tk, tv, p, stream)
+         : qpw == 2 ? launch_split<64, 2, FP8>(tk, tv, p, stream)
+                    : launch_split<64, 1, FP8>(tk, tv, p, stream);
 }
 
 }  // namespace decode_impl
@@ -526,16 +623,17 @@ size_t decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size, int ma
 
 int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     Plan pl;
-    if (!make_plan(a.Hq, a.Hkv, a.d, a.max_pages, pl)) return -2;
+    const int eb = a.fp8 ? 1 : 2;
+    if (!make_plan(a.Hq, a.Hkv, a.d, a.max_pages, eb, pl)) return -2;
     const size_t need = decode_workspace_bytes(a.num_seqs, a.Hq, a.d, a.page_size, a.max_pages);
     if (need == 0) return -2;
     if (!a.workspace || a.workspace_bytes < need) return -4;
     if (a.num_seqs == 0) return 0;
     alignas(64) CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)a.num_pages * kPage;
-    const uint64_t s1 = (uint64_t)a.d * 2, s2 = (uint64_t)a.Hkv * a.d * 2;
-    if (encode_tensor_map_3d(&tk, a.k_cache, 2, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false) ||
-        encode_tensor_map_3d(&tv, a.v_cache, 2, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false))
+    const uint64_t s1 = (uint64_t)a.d * eb, s2 = (uint64_t)a.Hkv * a.d * eb;
+    if (encode_tensor_map_3d(&tk, a.k_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false) ||
+        encode_tensor_map_3d(&tv, a.v_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false))
         return -5;
     DecodeParams p;
     p.q = static_cast<const uint16_t *>(a.q);
@@ -559,25 +657,23 @@ int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.nst = pl.nst;
     p.box_bytes = pl.box_bytes;
     p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
     int rc;
-    if (a.d == 128)
-        rc = pl.QPW == 4 ? launch_split<128, 4>(tk, tv, p, stream)
-           : pl.QPW == 2 ? launch_split<128, 2>(tk, tv, p, stream)
-                         : launch_split<128, 1>(tk, tv, p, stream);
+    if (a.fp8)
+        rc = launch_split_d<true>(a.d, pl.QPW, tk, tv, p, stream);
     else
-        rc = pl.QPW == 4 ? launch_split<64, 4>(tk, tv, p, stream)
-           : pl.QPW == 2 ? launch_split<64, 2>(tk, tv, p, stream)
-                         : launch_split<64, 1>(tk, tv, p, stream);
+        rc = launch_split_d<false>(a.d, pl.QPW, tk, tv, p, stream);
     if (rc) return rc;
     const int blocks = a.num_seqs * a.Hq;
     if (a.d == 128)
         decode_combine_kernel<128><<<blocks, 32 * kCombineWarps, 0, stream>>>(
-            p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.num_seqs,
-            a.Hq, a.max_pages, pl.max_chunks);
+            p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.sinks,
+            a.num_seqs, a.Hq, a.max_pages, pl.max_chunks);
     else
         decode_combine_kernel<64><<<blocks, 32 * kCombineWarps, 0, stream>>>(
-            p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.num_seqs,
-            a.Hq, a.max_pages, pl.max_chunks);
+            p.part_o, p.part_lse, a.seq_lens, static_cast<uint16_t *>(a.o), a.lse, a.sinks,
+            a.num_seqs, a.Hq, a.max_pages, pl.max_chunks);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 

@@ -49,12 +49,19 @@ int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t d
                          uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
                          bool swizzle128) {
     auto fn = encode_fn();
-    if (!fn || elem_bytes != 2) return -1;
+    if (!fn) return -1;
+    CUtensorMapDataType dt;
+    switch (elem_bytes) {
+    case 1: dt = CU_TENSOR_MAP_DATA_TYPE_UINT8; break;
+    case 2: dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; break;
+    case 4: dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; break;
+    default: return -1;
+    }
     cuuint64_t dims[3] = {dim0, dim1, dim2};
     cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
     cuuint32_t box[3] = {box0, box1, box2};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(static_cast<CUtensorMap *>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    CUresult r = fn(static_cast<CUtensorMap *>(map), dt, 3,
                     const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -106,9 +113,13 @@ int check_common(int Hq, int Hkv, int d, int causal, int window, float scale, in
 
 extern "C" {
 
-int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
-           int Hkv, int N, int d, int causal, int window, float scale, int o_dtype,
-           void *stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
+              const float *sinks, int B, int Hq, int Hkv, int N, int d, int causal, int window,
+              float scale, int o_dtype, void *stream) {
     if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
     if (rc) return rc;
@@ -130,13 +141,14 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     a.window = window > 0 ? window : 0;
     a.scale = scale;
     a.o_fp32 = o_dtype == FA_OUT_FP32;
+    a.sinks = sinks;
     return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
-int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
-                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
-                  int Hq, int Hkv, int d, int causal, int window, float scale, int o_dtype,
-                  void *stream) {
+int fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+               const float *sinks, const int *cu_seqlens, int num_seqs, int total_tokens,
+               int max_seqlen, int Hq, int Hkv, int d, int causal, int window, float scale,
+               int o_dtype, void *stream) {
     if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
     if (rc) return rc;
@@ -159,7 +171,134 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
     a.window = window > 0 ? window : 0;
     a.scale = scale;
     a.o_fp32 = o_dtype == FA_OUT_FP32;
+    a.sinks = sinks;
     return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int N, int d, int causal, int window, float scale, int o_dtype,
+           void *stream) {
+    return fwd_dense(q, k, v, o, lse, nullptr, B, Hq, Hkv, N, d, causal, window, scale,
+                     o_dtype, stream);
+}
+
+int fa_fwd_sinks(const void *q, const void *k, const void *v, void *o, float *lse,
+                 const float *sinks, int B, int Hq, int Hkv, int N, int d, int causal,
+                 int window, float scale, int o_dtype, void *stream) {
+    if (!sinks) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(sinks) & 3) return FA_ERR_ALIGNMENT;
+    return fwd_dense(q, k, v, o, lse, sinks, B, Hq, Hkv, N, d, causal, window, scale,
+                     o_dtype, stream);
+}
+
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
+                  int Hq, int Hkv, int d, int causal, int window, float scale, int o_dtype,
+                  void *stream) {
+    return fwd_varlen(q, k, v, o, lse, nullptr, cu_seqlens, num_seqs, total_tokens,
+                      max_seqlen, Hq, Hkv, d, causal, window, scale, o_dtype, stream);
+}
+
+int fa_fwd_varlen_sinks(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const float *sinks, const int *cu_seqlens, int num_seqs,
+                        int total_tokens, int max_seqlen, int Hq, int Hkv, int d, int causal,
+                        int window, float scale, int o_dtype, void *stream) {
+    if (!sinks) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(sinks) & 3) return FA_ERR_ALIGNMENT;
+    return fwd_varlen(q, k, v, o, lse, sinks, cu_seqlens, num_seqs, total_tokens,
+                      max_seqlen, Hq, Hkv, d, causal, window, scale, o_dtype, stream);
+}
+
+size_t fa_bwd_workspace_bytes(int total_tokens, int Hq, int d) {
+    return fa::bwd_workspace_bytes(total_tokens, Hq, d);
+}
+
+}  // extern "C"
+
+namespace {
+
+int bwd_common(const void *q, const void *k, const void *v, const void *o, const void *dout,
+               const float *lse, void *dq, void *dk, void *dv, int Hq, int Hkv, int d,
+               int causal, int window, float scale, long long total, void *workspace,
+               size_t workspace_bytes) {
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
+    if (rc) return rc;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (total > INT32_MAX / 2 || total * Hq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3))
+        return FA_ERR_ALIGNMENT;
+    const size_t need = fa::bwd_workspace_bytes(total, Hq, d);
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return FA_ERR_ALIGNMENT;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N, int d,
+           int causal, int window, float scale, void *workspace, size_t workspace_bytes,
+           void *stream) {
+    if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
+    if (rc) return rc;
+    if (B == 0 || N == 0) return FA_OK;
+    rc = bwd_common(q, k, v, o, dout, lse, dq, dk, dv, Hq, Hkv, d, causal, window, scale,
+                    (long long)B * N, workspace, workspace_bytes);
+    if (rc) return rc;
+    fa::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.cu_seqlens = nullptr;
+    a.num_seqs = B;
+    a.seqlen = N;
+    a.total_tokens = B * N;
+    a.max_seqlen = N;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.workspace = workspace;
+    return map_rc(fa::launch_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
+                  int Hq, int Hkv, int d, int causal, int window, float scale, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
+    if (rc) return rc;
+    if (num_seqs == 0 || total_tokens == 0 || max_seqlen == 0) return FA_OK;
+    if (!cu_seqlens) return FA_ERR_INVALID_ARG;
+    rc = bwd_common(q, k, v, o, dout, lse, dq, dk, dv, Hq, Hkv, d, causal, window, scale,
+                    total_tokens, workspace, workspace_bytes);
+    if (rc) return rc;
+    if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3) return FA_ERR_ALIGNMENT;
+    fa::BwdArgs a{};
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.cu_seqlens = cu_seqlens;
+    a.num_seqs = num_seqs;
+    a.seqlen = 0;
+    a.total_tokens = total_tokens;
+    a.max_seqlen = max_seqlen;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.workspace = workspace;
+    return map_rc(fa::launch_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t fa_decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size,
@@ -167,11 +306,16 @@ size_t fa_decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size,
     return fa::decode_workspace_bytes(num_seqs, Hq, d, page_size, max_pages_per_seq);
 }
 
-int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
-                    const int *block_table, const int *seq_lens, void *o, float *lse,
-                    int num_seqs, int num_pages, int Hq, int Hkv, int d, int page_size,
-                    int max_pages_per_seq, float scale, void *workspace, size_t workspace_bytes,
-                    void *stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_impl_call(const void *q, const void *k_cache, const void *v_cache,
+                     const int *block_table, const int *seq_lens, void *o, float *lse,
+                     const float *sinks, int num_seqs, int num_pages, int Hq, int Hkv, int d,
+                     int page_size, int max_pages_per_seq, float scale, void *workspace,
+                     size_t workspace_bytes, void *stream, const float *k_scale = nullptr,
+                     const float *v_scale = nullptr) {
     if (num_seqs < 0 || num_pages < 0 || max_pages_per_seq <= 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, 0, 0, scale, FA_OUT_BF16);
     if (rc) return rc;
@@ -198,8 +342,53 @@ int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
     a.max_pages = max_pages_per_seq;
     a.scale = scale;
     a.workspace = workspace;
+    a.sinks = sinks;
+    a.fp8 = k_scale != nullptr;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
     a.workspace_bytes = workspace_bytes;
     return map_rc(fa::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
+                    const int *block_table, const int *seq_lens, void *o, float *lse,
+                    int num_seqs, int num_pages, int Hq, int Hkv, int d, int page_size,
+                    int max_pages_per_seq, float scale, void *workspace, size_t workspace_bytes,
+                    void *stream) {
+    return decode_impl_call(q, k_cache, v_cache, block_table, seq_lens, o, lse, nullptr,
+                            num_seqs, num_pages, Hq, Hkv, d, page_size, max_pages_per_seq,
+                            scale, workspace, workspace_bytes, stream);
+}
+
+int fa_decode_paged_fp8(const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int *block_table,
+                        const int *seq_lens, void *o, float *lse, const float *sinks,
+                        int num_seqs, int num_pages, int Hq, int Hkv, int d, int page_size,
+                        int max_pages_per_seq, float scale, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    if (!k_scale || !v_scale) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k_scale) & 3) || (reinterpret_cast<uintptr_t>(v_scale) & 3) ||
+        (sinks && (reinterpret_cast<uintptr_t>(sinks) & 3)))
+        return FA_ERR_ALIGNMENT;
+    return decode_impl_call(q, k_cache, v_cache, block_table, seq_lens, o, lse, sinks,
+                            num_seqs, num_pages, Hq, Hkv, d, page_size, max_pages_per_seq,
+                            scale, workspace, workspace_bytes, stream, k_scale, v_scale);
+}
+
+int fa_decode_paged_sinks(const void *q, const void *k_cache, const void *v_cache,
+                          const int *block_table, const int *seq_lens, void *o, float *lse,
+                          const float *sinks, int num_seqs, int num_pages, int Hq, int Hkv,
+                          int d, int page_size, int max_pages_per_seq, float scale,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    if (!sinks) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(sinks) & 3) return FA_ERR_ALIGNMENT;
+    return decode_impl_call(q, k_cache, v_cache, block_table, seq_lens, o, lse, sinks,
+                            num_seqs, num_pages, Hq, Hkv, d, page_size, max_pages_per_seq,
+                            scale, workspace, workspace_bytes, stream);
 }
 
 const char *fa_status_string(int status) {

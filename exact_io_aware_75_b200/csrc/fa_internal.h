@@ -21,6 +21,7 @@ struct PrefillArgs {
     int causal, window;
     float scale;
     int o_fp32;
+    const float *sinks;     // device [Hq] learned sink logits; nullptr = none
 };
 
 int launch_prefill(const PrefillArgs &a, cudaStream_t stream);
@@ -34,10 +35,29 @@ struct DecodeArgs {
     float scale;
     void *workspace;
     size_t workspace_bytes;
+    const float *sinks;     // device [Hq] learned sink logits; nullptr = none
+    int fp8;                // caches hold FP8 E4M3 codes (1 byte) instead of bf16
+    const float *k_scale, *v_scale;  // FP8: device [num_pages][Hkv] scales
 };
 
 size_t decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size, int max_pages);
 int launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// Sizes the backward launch needs; validated by the public entry points.
+struct BwdArgs {
+    const void *q, *k, *v, *o, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    const int *cu_seqlens;  // device; nullptr = dense batch
+    int num_seqs, seqlen, total_tokens, max_seqlen;
+    int Hq, Hkv, d;
+    int causal, window;
+    float scale;
+    void *workspace;
+};
+
+size_t bwd_workspace_bytes(long long total_tokens, int Hq, int d);
+int launch_bwd(const BwdArgs &a, cudaStream_t stream);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

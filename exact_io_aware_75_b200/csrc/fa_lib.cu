@@ -4,3 +4,4 @@
 #include "prefill_sm100.cu"
 #include "decode_sm100.cu"
 #include "decode_noalloc.cu"
+#include "bwd_sm100.cu"

@@ -83,6 +83,7 @@ struct Params {
     int causal, window;
     float scale_log2;
     int o_fp32;
+    const float *sinks;   // [Hq] learned sink logits, or nullptr
     int num_mblocks;   // 256-row blocks per sequence (of max_seqlen)
     int num_units;
 };
@@ -480,10 +481,23 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
             ++pv_cnt;
         }
         // ---- epilogue: O / l, LSE
+        float inv_scale_o = 1.f;
         if (!mbar_wait_warp(&sh.o_full[t], (pv_cnt - 1) & 1, abort)) return;
         tc_fence_after();
         const bool valid = row < w.L;
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        if (p.sinks) {
+            // Learned sink: one more denominator term 2^(z*log2e - m) of a
+            // key whose value is zero; the reference max takes it in too.
+            const float z2 = __ldg(p.sinks + w.h) * 1.4426950408889634f;
+            const float m_new = fmaxf(m_ref, z2);
+            if (m_new != -INFINITY) {
+                const float a = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+                l = l * a + ex2(z2 - m_new);
+                inv_scale_o = a;
+                m_ref = m_new;
+            }
+        }
+        const float inv_l = (l > 0.f) ? inv_scale_o / l : 0.f;
         const size_t orow = ((size_t)(w.tok0 + row) * p.Hq + w.h) * D;
         #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -621,6 +635,7 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.window = a.causal ? a.window : 0;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.o_fp32 = a.o_fp32;
+    p.sinks = a.sinks;
     p.num_mblocks = (a.max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM);
     const long long units = (long long)p.num_mblocks * a.num_seqs * a.Hq;
     if (units <= 0) return 0;

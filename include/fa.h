@@ -98,6 +98,69 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                   float scale, int o_dtype, void *stream);
 
 /*
+ * Bytes of workspace fa_bwd / fa_bwd_varlen need for total_tokens tokens
+ * (B * N for a dense batch): an fp32 dQ accumulator [total, Hq, d] and the
+ * row terms D_i = dO_i . O_i.  0 for an unsupported combination (d != 128).
+ */
+size_t fa_bwd_workspace_bytes(int total_tokens, int Hq, int d);
+
+/*
+ * fa_fwd / fa_fwd_varlen with a learned attention sink per query head
+ * ("Sliding windows and local:global layers": gpt-oss's learned sink per
+ * head).  sinks [Hq] fp32, device, in units of scaled scores: z_h joins every
+ * row's softmax denominator as the score of one extra key whose value is
+ * zero, so O_i = sum_j e^(s_ij) V_j / (e^(z_h) + sum_j e^(s_ij)) and LSE
+ * includes the e^(z_h) term.  -INFINITY for a head means no sink.  Other
+ * arguments, layouts and errors as for fa_fwd / fa_fwd_varlen; sinks must be
+ * non-NULL and 4-byte aligned.  fa_bwd accepts the LSE these calls write (the
+ * sink enters the gradients of Q, K, V only through it).
+ */
+int fa_fwd_sinks(const void *q, const void *k, const void *v, void *o, float *lse,
+                 const float *sinks, int B, int Hq, int Hkv, int N, int d, int causal,
+                 int window, float scale, int o_dtype, void *stream);
+int fa_fwd_varlen_sinks(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const float *sinks, const int *cu_seqlens, int num_seqs,
+                        int total_tokens, int max_seqlen, int Hq, int Hkv, int d, int causal,
+                        int window, float scale, int o_dtype, void *stream);
+
+/*
+ * Backward of dense prefill: the gradients of sum(dO * O) with respect to Q,
+ * K and V, for O = fa_fwd(q, k, v, ...) with the same mask and scale.  The
+ * attention matrix is recomputed tile by tile from Q, K and the LSE the
+ * forward saved, never stored ("What attention costs", the FlashAttention
+ * paragraph: the backward pass recomputes the matrix from Q, K, V and the
+ * saved softmax statistics).  With grouped heads, dK and dV of a KV head sum
+ * over the query heads that read it.
+ *   q, o, dout [B, N, Hq, d]  bf16, device (o as written by fa_fwd)
+ *   k, v       [B, N, Hkv, d] bf16, device
+ *   lse        [B, Hq, N]     fp32, device: the forward's LSE (natural log)
+ *   dq         [B, N, Hq, d]  bf16, device, written
+ *   dk, dv     [B, N, Hkv, d] bf16, device, written
+ *   workspace  device scratch of at least fa_bwd_workspace_bytes(B * N, Hq, d)
+ *              bytes, 256-byte aligned; contents on entry do not matter; not
+ *              to be shared by calls that may overlap on the GPU.
+ *   causal, window, scale as for fa_fwd.  d must be 128 (others return
+ *   FA_ERR_UNSUPPORTED).  N == 0 or B == 0 is a no-op returning FA_OK.
+ * dQ is accumulated in fp32 with atomic adds, so its last bits may differ
+ * from run to run; dK and dV are deterministic.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N,
+           int d, int causal, int window, float scale, void *workspace,
+           size_t workspace_bytes, void *stream);
+
+/*
+ * Backward of packed variable-length prefill (fa_fwd_varlen's layouts: q, o,
+ * dout, dq [total, Hq, d]; k, v, dk, dv [total, Hkv, d]; lse [Hq, total];
+ * cu_seqlens as there).  Workspace: fa_bwd_workspace_bytes(total_tokens, Hq, d).
+ */
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
+                  int Hq, int Hkv, int d, int causal, int window, float scale,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of workspace fa_decode_paged needs for these sizes (split-KV
  * partial outputs and their log-sum-exps).  0 for an invalid combination.
  */
@@ -133,6 +196,35 @@ int fa_decode_paged(const void *q, const void *k_cache, const void *v_cache,
                     float *lse, int num_seqs, int num_pages, int Hq, int Hkv,
                     int d, int page_size, int max_pages_per_seq, float scale,
                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_decode_paged with a learned attention sink per query head (sinks [Hq]
+ * fp32, device; meaning as for fa_fwd_sinks).  A sequence of length 0 then
+ * gets O = 0 and LSE = z_h.
+ */
+int fa_decode_paged_sinks(const void *q, const void *k_cache, const void *v_cache,
+                          const int *block_table, const int *seq_lens, void *o, float *lse,
+                          const float *sinks, int num_seqs, int num_pages, int Hq, int Hkv,
+                          int d, int page_size, int max_pages_per_seq, float scale,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_decode_paged over an FP8 cache ("FP8 KV cache": the post's cache-size
+ * paragraphs before "Paging and prefix sharing" -- fewer bits per cached
+ * value).  k_cache/v_cache [num_pages, page_size, Hkv, d] hold OCP FP8 E4M3
+ * codes (the "fn" variant, one byte each); the cached value is
+ * e4m3(code) * scale with k_scale/v_scale [num_pages, Hkv] fp32, device (one
+ * scale per page and KV head; a per-head scale is the case of equal page
+ * scales).  sinks [Hq] or NULL (as fa_decode_paged_sinks).  Halves the bytes
+ * read per token.  Other arguments, the workspace and errors as for
+ * fa_decode_paged; codes of unused slots may hold anything, NaN included.
+ */
+int fa_decode_paged_fp8(const void *q, const void *k_cache, const void *v_cache,
+                        const float *k_scale, const float *v_scale, const int *block_table,
+                        const int *seq_lens, void *o, float *lse, const float *sinks,
+                        int num_seqs, int num_pages, int Hq, int Hkv, int d, int page_size,
+                        int max_pages_per_seq, float scale, void *workspace,
+                        size_t workspace_bytes, void *stream);
 
 /*
  * fa_decode_paged without a workspace argument, for callers that cannot

@@ -19,7 +19,7 @@ def fa():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "fa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_exports_match_header(fa):
@@ -111,6 +111,76 @@ def test_decode_workspace_formula(fa):
     assert fa.decode_workspace_bytes(S, Hq, d, 16, maxp) == r256(rows * d * 4) + r256(rows * 4)
     assert fa.decode_workspace_bytes(S, Hq, d, 8, maxp) == 0
     assert fa.decode_workspace_bytes(0, Hq, d, 16, maxp) == 0
+
+
+def bwd(fa, **kw):
+    a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, B=1, Hq=4, Hkv=2, N=256, d=128,
+             causal=1, window=0, scale=0.125, ws=P, wsb=1 << 30)
+    a.update(kw)
+    return fa.library().fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"],
+                               a["dk"], a["dv"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                               a["causal"], a["window"], a["scale"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), -1), (dict(scale=-1.0), -1), (dict(causal=3), -1), (dict(d=64), -2),
+    (dict(d=80), -2), (dict(window=8, causal=0), -2), (dict(do=0), -1), (dict(lse=0), -1),
+    (dict(dq=0), -1), (dict(dv=P + 4), -3), (dict(lse=P + 1), -3), (dict(ws=0), -4),
+    (dict(wsb=1000), -4), (dict(ws=P + 16), -3), (dict(B=-2), -1)])
+def test_bwd_rejects(fa, kw, status):
+    assert bwd(fa, **kw) == status
+
+
+def test_bwd_empty_is_noop(fa):
+    assert bwd(fa, B=0, q=0, ws=0) == 0
+    assert bwd(fa, N=0, q=0, ws=0) == 0
+
+
+def test_bwd_varlen_rejects(fa):
+    lib = fa.library()
+    args = [P] * 9
+    # cu_seqlens missing, then misaligned
+    assert lib.fa_bwd_varlen(*args, None, 2, 100, 60, 4, 2, 128, 1, 0, 0.1, P, 1 << 30, None) == -1
+    assert lib.fa_bwd_varlen(*args, P + 2, 2, 100, 60, 4, 2, 128, 1, 0, 0.1, P, 1 << 30,
+                             None) == -3
+    assert lib.fa_bwd_varlen(*args, P, 0, 0, 0, 4, 2, 128, 1, 0, 0.1, None, 0, None) == 0
+
+
+def test_bwd_workspace_formula(fa):
+    r256 = lambda x: (x + 255) // 256 * 256
+    T, Hq = 4096, 32
+    assert fa.bwd_workspace_bytes(T, Hq, 128) == r256(T * Hq * 128 * 4) + r256(T * Hq * 4)
+    assert fa.bwd_workspace_bytes(T, Hq, 64) == 0
+
+
+def test_sinks_entry_points_reject(fa):
+    lib = fa.library()
+    # fa_fwd_sinks: sinks NULL, then misaligned
+    assert lib.fa_fwd_sinks(P, P, P, P, 0, None, 1, 2, 2, 128, 64, 0, 0, 0.1, 0, None) == -1
+    assert lib.fa_fwd_sinks(P, P, P, P, 0, P + 2, 1, 2, 2, 128, 64, 0, 0, 0.1, 0, None) == -3
+    # otherwise the same validation as fa_fwd
+    assert lib.fa_fwd_sinks(P, P, P, P, 0, P, 1, 3, 2, 128, 64, 0, 0, 0.1, 0, None) == -1
+    assert lib.fa_fwd_varlen_sinks(P, P, P, P, 0, None, P, 2, 100, 60, 2, 2, 64, 1, 0, 0.1, 0,
+                                   None) == -1
+    assert lib.fa_decode_paged_sinks(P, P, P, P, P, P, 0, None, 4, 100, 32, 8, 128, 16, 64, 0.1,
+                                     P, 1 << 30, None) == -1
+    assert lib.fa_decode_paged_sinks(P, P, P, P, P, P, 0, P + 1, 4, 100, 32, 8, 128, 16, 64,
+                                     0.1, P, 1 << 30, None) == -3
+
+
+def test_fp8_decode_rejects(fa):
+    lib = fa.library()
+    base = [P, P, P]
+    tail = [P, P, P, 0, None, 4, 100, 32, 8, 128, 16, 64, 0.1, P, 1 << 30, None]
+    assert lib.fa_decode_paged_fp8(*base, None, P, *tail) == -1          # k_scale NULL
+    assert lib.fa_decode_paged_fp8(*base, P, None, *tail) == -1          # v_scale NULL
+    assert lib.fa_decode_paged_fp8(*base, P + 2, P, *tail) == -3         # misaligned scale
+    t2 = list(tail)
+    t2[3] = P + 1                                                        # misaligned sinks
+    assert lib.fa_decode_paged_fp8(*base, P, P, *t2) == -3
+    t3 = list(tail)
+    t3[10] = 8                                                           # page size 8
+    assert lib.fa_decode_paged_fp8(*base, P, P, *t3) == -2
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
