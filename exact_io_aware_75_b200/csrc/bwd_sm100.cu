@@ -56,6 +56,13 @@ constexpr int kWarpDrain = 8;  // warps 8..11
 constexpr int kWarpTma = 12;
 constexpr int kWarpMma = 13;
 constexpr int kStages = 3;
+// Register split (launched with 512 x 128 = 65,536): the two elementwise
+// warpgroups hold a whole 64-column row of Sᵀ and dPᵀ each.
+constexpr int kRegsSoftmax = 176;
+constexpr int kRegsDrain = 88;
+constexpr int kRegsControl = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsDrain + 128 * kRegsControl <= kThreads * 128,
+              "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // S^T of buffer b at b * 64 (P^T overwrites its first 32)
 constexpr uint32_t kColDP = 128;  // dP^T of buffer b at 128 + b * 64, then the tile's dQ^T
@@ -189,7 +196,7 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
                     tma_load_3d(st + kQTile + b * kQBox, tmdO, &sh.qd_full[s], b * 64, h, w.tok0 + q0);
                 }
             }
-            // The tile's LSE (log2 units) and D; rows past the sequence get
+            // The tile's -LSE (log2 units) and -D; rows past the sequence get
             // LSE = +inf, so their P is exactly 0.
             float *rs = rows + s * 2 * kBlockQ;
             #pragma unroll
@@ -201,8 +208,8 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
                     l2 = __ldg(p.lse + idx) * 1.4426950408889634f;
                     dv = __ldg(p.dd + idx);
                 }
-                rs[rr] = l2;
-                rs[kBlockQ + rr] = dv;
+                rs[rr] = -l2;
+                rs[kBlockQ + rr] = -dv;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.qd_full[s]);
@@ -230,8 +237,8 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
 
     // S^T(b) = K Q^T and dP^T(b) = V dO^T: K-major operands, d/16 steps; a
     // step moves 32 bytes inside a 64-column box, 4 steps cross to the next box.
-    auto issue_s_dp = [&](int b, int s) {
-        const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+    auto issue_s = [&](int b, int s) {
+        const uint32_t q = aStage + s * kStageBytes;
         #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
             const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
@@ -239,6 +246,9 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
             mma_ss(tmem + kColS + b * kBlockQ, smem_desc_sw128(aK + okv, 16, 1024),
                    smem_desc_sw128(q + oq, 16, 1024), idS, ks > 0);
         }
+    };
+    auto issue_dp = [&](int b, int s) {
+        const uint32_t dO = aStage + s * kStageBytes + kQTile;
         #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
             const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
@@ -284,9 +294,12 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
         for (int k = 0; k < w.ntiles; ++k, ++n) {
             const int b = n & 1, s = n % kStages;
             if (!mbar_wait(&sh.qd_full[s], (n / kStages) & 1, abort)) goto out;
+            tc_fence_after();
+            issue_s(b, s);
+            // dPᵀ(b) overwrites the dQᵀ of tile n-2: wait until it is drained
             if (n >= 2 && !mbar_wait(&sh.dq_free[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
-            issue_s_dp(b, s);
+            issue_dp(b, s);
             tc_commit(&sh.s_full[b]);
             if (k > 0 && !issue_grads(n - 1, k == 1)) goto out;
         }
@@ -327,47 +340,62 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
             int h, q0;
             tile_of(w, p, k, h, q0);
             (void)h;
-            const float *l2 = rows + s * 2 * kBlockQ;
-            const float *dd = l2 + kBlockQ;
+            const float4 *nl4 = reinterpret_cast<const float4 *>(rows + s * 2 * kBlockQ);
+            const float4 *nd4 = nl4 + kBlockQ / 4;
             const int qmax = min(q0 + kBlockQ, w.L) - 1;
             const bool edge = (w.j0 + kBlockK > w.L) || (p.causal && w.jl > q0) ||
                               (p.window > 0 && w.j0 <= qmax - p.window);
+            // Sᵀ and dPᵀ rows of this key: all four loads in flight at once
+            uint32_t sr[kBlockQ], dr[kBlockQ];
+            tmem_ld32(tS, sr);
+            tmem_ld32(tS + 32, sr + 32);
+            tmem_ld32(tdP, dr);
+            tmem_ld32(tdP + 32, dr + 32);
+            tmem_wait_ld();
+            const uint64_t c2 = f2pack(sl2, sl2);
+            uint32_t pk[kBlockQ / 2], dk[kBlockQ / 2];
             #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(tS + hh * 32, sr);
-                tmem_ld32(tdP + hh * 32, dr);
-                tmem_wait_ld();
-                uint32_t pk[16], dk[16];
-                #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const int cc = hh * 32 + c;
-                    float p0 = ex2(fmaf(__uint_as_float(sr[c]), sl2, -l2[cc]));
-                    float p1 = ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, -l2[cc + 1]));
-                    if (edge) {
-                        const int i0 = q0 + cc, i1 = i0 + 1;
-                        bool v0 = key_ok, v1 = key_ok;
-                        if (p.causal) {
-                            v0 = v0 && kj <= i0 && (p.window <= 0 || kj > i0 - p.window);
-                            v1 = v1 && kj <= i1 && (p.window <= 0 || kj > i1 - p.window);
-                        }
-                        p0 = v0 ? p0 : 0.f;
-                        p1 = v1 ? p1 : 0.f;
+            for (int c = 0; c < kBlockQ; c += 4) {
+                const float4 nl = nl4[c >> 2], nd = nd4[c >> 2];   // -LSE2, -D (broadcast)
+                float x0, x1, x2, x3;
+                f2unpack(f2fma(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2,
+                               f2pack(nl.x, nl.y)), x0, x1);
+                f2unpack(f2fma(f2pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), c2,
+                               f2pack(nl.z, nl.w)), x2, x3);
+                float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+                if (edge) {
+                    const int i0 = q0 + c;
+                    bool v[4];
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        v[e] = key_ok;
+                        if (p.causal)
+                            v[e] = v[e] && kj <= i0 + e && (p.window <= 0 || kj > i0 + e - p.window);
                     }
-                    const float d0 = p0 * (__uint_as_float(dr[c]) - dd[cc]);
-                    const float d1 = p1 * (__uint_as_float(dr[c + 1]) - dd[cc + 1]);
-                    pk[c >> 1] = pack_bf16(p0, p1);
-                    dk[c >> 1] = pack_bf16(d0, d1);
+                    p0 = v[0] ? p0 : 0.f;
+                    p1 = v[1] ? p1 : 0.f;
+                    p2 = v[2] ? p2 : 0.f;
+                    p3 = v[3] ? p3 : 0.f;
                 }
-                tmem_st16(tS + hh * 16, pk);
-                // dS^T row r, queries hh*32 .. hh*32+31: four 16-byte chunks,
-                // chunk index XOR (row & 7) (128-byte swizzle)
-                #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int chunk = hh * 4 + c4;
-                    uint4 v = make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
-                    *reinterpret_cast<uint4 *>(dsb + ((chunk ^ (r & 7)) << 4)) = v;
-                }
+                float d0, d1, d2, d3;
+                f2unpack(f2mul(f2pack(p0, p1),
+                               f2add(f2pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                                     f2pack(nd.x, nd.y))), d0, d1);
+                f2unpack(f2mul(f2pack(p2, p3),
+                               f2add(f2pack(__uint_as_float(dr[c + 2]), __uint_as_float(dr[c + 3])),
+                                     f2pack(nd.z, nd.w))), d2, d3);
+                pk[c >> 1] = pack_bf16(p0, p1);
+                pk[(c >> 1) + 1] = pack_bf16(p2, p3);
+                dk[c >> 1] = pack_bf16(d0, d1);
+                dk[(c >> 1) + 1] = pack_bf16(d2, d3);
+            }
+            tmem_st32(tS, pk);
+            // dSᵀ row r: eight 16-byte chunks of 8 queries, chunk index XOR
+            // (row & 7) (128-byte swizzle)
+            #pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint4 v = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+                *reinterpret_cast<uint4 *>(dsb + ((ch ^ (r & 7)) << 4)) = v;
             }
             tmem_wait_st();
             fence_proxy_async_smem();
@@ -503,13 +531,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tc_fence_after();
 
     if (warp < 8) {
+        regs_increase<kRegsSoftmax>();
         softmax_wg(p, sh, smem);
     } else if (warp < 12) {
+        regs_decrease<kRegsDrain>();
         dq_drain(&tmDQ, p, sh, smem);
-    } else if (warp == kWarpTma) {
-        producer(&tmQ, &tmK, &tmV, &tmdO, p, sh, smem);
-    } else if (warp == kWarpMma) {
-        if (lane_id() == 0) mma_issuer(p, sh, smem);
+    } else {
+        regs_decrease<kRegsControl>();
+        if (warp == kWarpTma) {
+            producer(&tmQ, &tmK, &tmV, &tmdO, p, sh, smem);
+        } else if (warp == kWarpMma) {
+            if (lane_id() == 0) mma_issuer(p, sh, smem);
+        }
     }
     __syncwarp();
     tc_fence_before();
