@@ -56,7 +56,8 @@ def parse():
     # profiling aids (the default run times both kernels on the named workloads)
     ap.add_argument("--no-next", action="store_true",
                     help="skip the extension rows (backward, FP8-cache decode)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "bwd", "decode_fp8"],
+                    default="all",
                     help="time one kernel family only (for profiler captures)")
     ap.add_argument("--prefill-workload", default=PREFILL,
                     choices=["gqa4k", "long32k", "long32k_w4096"])
@@ -232,8 +233,10 @@ def bench_ours(args):
     pk, pk_src = peaks()
 
     # ---- inputs (seeded per rank; resident in HBM before timing)
-    do_p = args.only in ("all", "prefill")
-    do_d = args.only in ("all", "decode")
+    do_p = args.only in ("all", "prefill", "bwd")
+    do_d = args.only in ("all", "decode", "decode_fp8")
+    if args.only in ("bwd", "decode_fp8"):
+        return bench_only_next(fa_import(), args, do_p, do_d)
     pname = args.prefill_workload
     seed = rank_seed(args.seed, rank)
     pin = workloads.make(pname, seed=seed)
@@ -410,8 +413,43 @@ def bench_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def fa_import():
+    import exact_io_aware_75_b200 as fa
+    return fa
+
+
+def bench_only_next(fa, args, do_p, do_d):
+    """--only bwd / --only decode_fp8: that extension row alone (for profiling)."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    pk, _ = peaks()
+    seed = args.seed
+    pin = workloads.make(args.prefill_workload if do_p else PREFILL, seed=seed,
+                         **({} if do_p else {"N": 128}))
+    q, k, v = pin.q.to(dev), pin.k.to(dev), pin.v.to(dev)
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    flops = prefill_flops(B, Hq, N, d, True, pin.window)
+    din = workloads.make(DECODE, seed=seed, num_seqs=args.decode_seqs if do_d else 1,
+                         **({} if do_d else {"len_lo": 16, "len_hi": 16}))
+    dq, dk, dv = din.q.to(dev), din.k_cache.to(dev), din.v_cache.to(dev)
+    dbt, dsl = din.block_table.to(dev), din.seq_lens.to(dev)
+    S = dq.shape[0]
+    ws = torch.empty(fa.decode_workspace_bytes(S, dq.shape[1], dq.shape[2], 16, dbt.shape[1]),
+                     dtype=torch.uint8, device=dev)
+    dout = torch.empty_like(dq)
+    dlse = torch.empty((S, dq.shape[1]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nxt = bench_next(fa, args, dev, torch.cuda.current_stream(), flush, pk, recorded_traffic(),
+                     pin, q, k, v, o, lse, flops, din, dq, dk, dv, dbt, dsl, ws, dout, dlse,
+                     which=args.only)
+    print(json.dumps({"note": f"--only {args.only}: one extension row alone, for profiling",
+                      "next": nxt, "kernel_source": kernel_source_hash()}), flush=True)
+
+
 def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, lse, flops,
-               din, dq, dk, dv, dbt, dsl, ws, dout, dlse):
+               din, dq, dk, dv, dbt, dsl, ws, dout, dlse, which="all"):
     """The rows built beyond the headline path, each timed with CUDA events
     over K calls (L2 flushed before each), with its own roofline:
       bwd        -- fa_bwd on the prefill workload: FLOPs = 2.5 x the forward's
@@ -437,6 +475,18 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
         torch.cuda.synchronize()
         return max_over_ranks([sum(a.elapsed_time(b) for a, b in evs)], dev)[0] / K
 
+    if which in ("all", "bwd"):
+        bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, flops, out)
+    if which in ("all", "decode_fp8"):
+        bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, dsl, ws,
+                       dout, dlse, out)
+    err = fa.check_device_error()
+    if err:
+        raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
+    return out
+
+
+def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, flops, out):
     # backward: O and LSE from the forward, a seeded upstream gradient
     fa.fwd(q, k, v, True, pin.window, pin.scale, out=o, lse=lse)
     g = workloads.grad_out(tuple(q.shape), seed=args.seed).to(dev)
@@ -456,6 +506,9 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
                                "traffic": traffic_all.get("bwd_gqa4k")}}
     del g, gq, gk, gv, wsb
 
+
+def bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, dsl, ws, dout,
+                   dlse, out):
     # FP8 cache: quantised on the device from the bf16 cache (input preparation)
     def quant(x):
         amax = x.float().abs().amax(dim=(1, 3))
@@ -483,10 +536,6 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
                                       "kernel": "decode_split_kernel<128,4,fp8> + combine",
                                       "traffic": traffic_all.get("decode_fp8_decode64")}}
     del kc8, vc8, ks8, vs8
-    err = fa.check_device_error()
-    if err:
-        raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
-    return out
 
 
 # ---------------------------------------------------------------- reference

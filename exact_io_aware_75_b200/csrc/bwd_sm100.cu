@@ -626,15 +626,15 @@ int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
     const uint64_t T = (uint64_t)total;
     if (encode_tensor_map_3d(&tq, a.q, 2, kD, a.Hq, T, (uint64_t)kD * 2, (uint64_t)a.Hq * kD * 2,
-                             64, 1, kBlockQ, true) ||
+                             64, 1, kBlockQ, 128) ||
         encode_tensor_map_3d(&tdo, a.dout, 2, kD, a.Hq, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hq * kD * 2, 64, 1, kBlockQ, true) ||
+                             (uint64_t)a.Hq * kD * 2, 64, 1, kBlockQ, 128) ||
         encode_tensor_map_3d(&tk, a.k, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, true) ||
+                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, 128) ||
         encode_tensor_map_3d(&tv, a.v, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, true) ||
+                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, 128) ||
         encode_tensor_map_3d(&tdq, dq_acc, 4, kD, a.Hq, T, (uint64_t)kD * 4,
-                             (uint64_t)a.Hq * kD * 4, kD, 1, kDQHalf, false))
+                             (uint64_t)a.Hq * kD * 4, kD, 1, kDQHalf, 0))
         return -5;
     Params p;
     p.lse = a.lse;

@@ -641,8 +641,8 @@ int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     alignas(64) CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)a.num_pages * kPage;
     const uint64_t s1 = (uint64_t)a.d * eb, s2 = (uint64_t)a.Hkv * a.d * eb;
-    if (encode_tensor_map_3d(&tk, a.k_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false) ||
-        encode_tensor_map_3d(&tv, a.v_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, false))
+    if (encode_tensor_map_3d(&tk, a.k_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, 0) ||
+        encode_tensor_map_3d(&tv, a.v_cache, eb, a.d, a.Hkv, rows, s1, s2, a.d, pl.HG, kPage, 0))
         return -5;
     DecodeParams p;
     p.q = static_cast<const uint16_t *>(a.q);

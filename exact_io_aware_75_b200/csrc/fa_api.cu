@@ -47,7 +47,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t dim0,
                          uint64_t dim1, uint64_t dim2, uint64_t stride1_bytes,
                          uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2,
-                         bool swizzle128) {
+                         int swizzle_bytes) {
     auto fn = encode_fn();
     if (!fn) return -1;
     CUtensorMapDataType dt;
@@ -57,6 +57,14 @@ int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t d
     case 4: dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; break;
     default: return -1;
     }
+    CUtensorMapSwizzle sw;
+    switch (swizzle_bytes) {
+    case 0: sw = CU_TENSOR_MAP_SWIZZLE_NONE; break;
+    case 32: sw = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: sw = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: sw = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return -1;
+    }
     cuuint64_t dims[3] = {dim0, dim1, dim2};
     cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
     cuuint32_t box[3] = {box0, box1, box2};
@@ -64,7 +72,7 @@ int encode_tensor_map_3d(void *map, const void *base, int elem_bytes, uint64_t d
     CUresult r = fn(static_cast<CUtensorMap *>(map), dt, 3,
                     const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    sw,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? 0 : -1;
 }

@@ -66,6 +66,6 @@ int device_sm_count();
 int encode_tensor_map_3d(void *map, const void *base, int elem_bytes,
                          uint64_t dim0, uint64_t dim1, uint64_t dim2,
                          uint64_t stride1_bytes, uint64_t stride2_bytes,
-                         uint32_t box0, uint32_t box1, uint32_t box2, bool swizzle128);
+                         uint32_t box0, uint32_t box1, uint32_t box2, int swizzle_bytes);
 
 }  // namespace fa

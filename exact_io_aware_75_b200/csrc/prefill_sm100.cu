@@ -614,11 +614,11 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     alignas(64) CUtensorMap tq, tk, tv;
     const uint64_t T = (uint64_t)a.total_tokens;
     if (encode_tensor_map_3d(&tq, a.q, 2, D, a.Hq, T, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2,
-                             64, 1, kBlockM, true) ||
+                             64, 1, kBlockM, 128) ||
         encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kBlockN, true) ||
+                             64, 1, kBlockN, 128) ||
         encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kBlockN, true))
+                             64, 1, kBlockN, 128))
         return -5;
     Params p;
     p.o = a.o;
