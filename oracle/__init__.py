@@ -67,6 +67,11 @@ def lib():
             _u16p, _u8p, _u8p, _f32p, _f32p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, _f64p, _f64p]
         L.oracle_decode_paged_fp8.restype = ctypes.c_int
+        L.oracle_prefill_paged.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
+            _f64p, _f64p]
+        L.oracle_prefill_paged.restype = ctypes.c_int
         L.oracle_attn_bwd_varlen.argtypes = [
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _f64p, _f64p, _f64p]
@@ -348,3 +353,27 @@ def decode_paged_fp8(q, k_codes, v_codes, k_scale, v_scale, block_table, seq_len
                                          bt.shape[1], P, float(scale), sp, o, lse),
            "decode_paged_fp8")
     return o, lse
+
+
+def prefill_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, causal=True,
+                  window=0, scale=None, sinks=None):
+    """Chunked prefill over a paged cache: q [Tq,Hq,d] holds each sequence's
+    last L_q tokens; caches [P,ps,Hkv,d]; -> O [Tq,Hq,d], LSE [Hq,Tq]."""
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    Tq, Hq, d = qb.shape
+    P, ps, Hkv, _ = kb.shape
+    bt = _i32(block_table)
+    cu = _i32(cu_seqlens_q)
+    sl = _i32(seq_lens_k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    sp = None
+    if sinks is not None:
+        sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(Hq))
+        sp = sk.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((Tq, Hq, d), np.float64)
+    lse = np.empty((Tq, Hq), np.float64)
+    _check(lib().oracle_prefill_paged(qb, kb, vb, bt, cu, sl, len(cu) - 1, Hq, Hkv, d, ps,
+                                      bt.shape[1], P, int(causal), int(window), float(scale),
+                                      sp, o, lse), "prefill_paged")
+    return o, np.ascontiguousarray(lse.T)

@@ -698,3 +698,76 @@ int oracle_decode_paged_fp8(const uint16_t *q, const uint8_t *k_cache, const uin
     }
     return bad ? -2 : 0;
 }
+
+/*
+ * Chunked prefill over a paged cache ("Chunked-prefill serving ... pairs
+ * FlashAttention with KV paging", FlashAttention explainer, real-world
+ * examples): sequence s has seq_lens_k[s] tokens in its pages (earlier
+ * context plus this chunk's own keys), and its L_q = cu_seqlens_q[s+1] -
+ * cu_seqlens_q[s] new query tokens are the last L_q of them: query i of the
+ * chunk sits at position seq_lens_k[s] - L_q + i (the causal reading that
+ * makes L_q = 1 the decode case and L_q = seq_lens_k the plain prefill).
+ *   q [total_q, Hq, d]; k_cache/v_cache [num_pages, page_size, Hkv, d]
+ *   block_table [S, max_pages]; sinks [Hq] or NULL
+ *   o [total_q, Hq, d]; lse [total_q, Hq]
+ * Returns -1 if some L_q > seq_lens_k or a used table entry is out of range.
+ */
+int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                         const int32_t *block_table, const int32_t *cu_seqlens_q,
+                         const int32_t *seq_lens_k, int S, int Hq, int Hkv, int d,
+                         int page_size, int max_pages, int64_t num_pages, int causal,
+                         int window, double scale, const double *sinks, double *o,
+                         double *lse)
+{
+    if (S < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || page_size <= 0) return -1;
+    int64_t maxlen = 0;
+    for (int s = 0; s < S; ++s) {
+        const int64_t Lq = (int64_t)cu_seqlens_q[s + 1] - cu_seqlens_q[s];
+        const int64_t Lk = seq_lens_k[s];
+        if (Lq < 0 || Lk < Lq || Lk > (int64_t)max_pages * page_size) return -1;
+        if (Lk > maxlen) maxlen = Lk;
+        for (int64_t p = 0; p < (Lk + page_size - 1) / page_size; ++p) {
+            int32_t pg = block_table[(int64_t)s * max_pages + p];
+            if (pg < 0 || pg >= num_pages) return -1;
+        }
+    }
+    const int group = Hq / Hkv;
+    const int64_t total_q = cu_seqlens_q[S];
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sb = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
+        unsigned char *vis = (unsigned char *)malloc(n);
+        if (!sb || !qd || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < total_q * (int64_t)Hq; ++task) {
+                const int64_t t = task / Hq;
+                const int h = (int)(task % Hq), g = h / group;
+                int s = 0;
+                while (s < S && cu_seqlens_q[s + 1] <= t) ++s;
+                const int64_t Lq = (int64_t)cu_seqlens_q[s + 1] - cu_seqlens_q[s];
+                const int64_t Lk = seq_lens_k[s];
+                const int64_t pos = Lk - Lq + (t - cu_seqlens_q[s]);
+                for (int c = 0; c < d; ++c) qd[c] = widen(q[(t * Hq + h) * (int64_t)d + c]);
+                for (int64_t j = 0; j < Lk; ++j) {
+                    const int64_t pg = block_table[(int64_t)s * max_pages + j / page_size];
+                    const int64_t slot = j % page_size;
+                    kp[j] = k_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    vp[j] = v_cache + ((pg * page_size + slot) * Hkv + g) * (int64_t)d;
+                    vis[j] = (unsigned char)allowed(pos, j, causal, window);
+                }
+                attend_row_sink(qd, d, Lk, kp, vp, vis, scale, sinks ? sinks[h] : -INFINITY,
+                                sb, o + task * (int64_t)d, lse + task, NULL);
+            }
+        }
+        free(sb); free(qd); free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
