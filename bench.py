@@ -56,7 +56,8 @@ def parse():
     # profiling aids (the default run times both kernels on the named workloads)
     ap.add_argument("--no-next", action="store_true",
                     help="skip the extension rows (backward, FP8-cache decode)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode", "bwd", "decode_fp8"],
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "bwd", "decode_fp8",
+                                       "prefill_paged"],
                     default="all",
                     help="time one kernel family only (for profiler captures)")
     ap.add_argument("--prefill-workload", default=PREFILL,
@@ -235,7 +236,7 @@ def bench_ours(args):
     # ---- inputs (seeded per rank; resident in HBM before timing)
     do_p = args.only in ("all", "prefill", "bwd")
     do_d = args.only in ("all", "decode", "decode_fp8")
-    if args.only in ("bwd", "decode_fp8"):
+    if args.only in ("bwd", "decode_fp8", "prefill_paged"):
         return bench_only_next(fa_import(), args, do_p, do_d)
     pname = args.prefill_workload
     seed = rank_seed(args.seed, rank)
@@ -480,6 +481,8 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
     if which in ("all", "decode_fp8"):
         bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, dsl, ws,
                        dout, dlse, out)
+    if which in ("all", "prefill_paged"):
+        bench_next_paged(fa, args, dev, timed, pk, traffic_all, out)
     err = fa.check_device_error()
     if err:
         raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
@@ -505,6 +508,40 @@ def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, 
                                "kernel": "bwd_kernel (+ bwd_prep_kernel, bwd_convert_kernel)",
                                "traffic": traffic_all.get("bwd_gqa4k")}}
     del g, gq, gk, gv, wsb
+
+
+def paged_prefill_workload(seed):
+    """Chunked prefill: 8 sequences with 8K-14K tokens of earlier context and a
+    new chunk of 512-2048 tokens each (Hq=32, Hkv=8, d=128, causal)."""
+    g = torch.Generator("cpu").manual_seed(seed + 3)
+    lens_q = workloads.draw_lengths(8, 512, 2048, g)
+    lens_k = [q + c for q, c in zip(lens_q, workloads.draw_lengths(8, 8192, 14336, g))]
+    return workloads.paged_prefill(lens_k, lens_q, Hq=32, Hkv=8, d=128, seed=seed)
+
+
+def bench_next_paged(fa, args, dev, timed, pk, traffic_all, out):
+    w = paged_prefill_workload(args.seed)
+    q, kc, vc = w.q.to(dev), w.k_cache.to(dev), w.v_cache.to(dev)
+    bt, cu, sl = w.block_table.to(dev), w.cu_seqlens_q.to(dev), w.seq_lens_k.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=dev)
+    ms = timed(lambda: fa.fwd_paged(q, kc, vc, bt, cu, sl, w.max_seqlen_q, True, 0, w.scale,
+                                    out=o, lse=lse))
+    Hq, d = q.shape[1], q.shape[2]
+    pairs = 0.0
+    for Lq, Lk in zip(w.lens_q, w.seq_lens_k.tolist()):
+        pairs += Lq * (Lk - Lq) + Lq * (Lq + 1) / 2       # visible (query, key) pairs
+    flop = 4.0 * Hq * d * pairs
+    ach = flop / (ms * 1e-3) / 1e12
+    out["prefill_paged"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+                            "flop_per_call": flop, "launches_per_call": 1,
+                            "workload": "chunked prefill over a 16-token paged cache: 8 sequences, "
+                                        f"chunks {w.lens_q}, context+chunk {w.seq_lens_k.tolist()}",
+                            "roofline": {"bound": "tensor", "achieved": round(ach, 2),
+                                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                                         "frac": round(ach / pk["bf16_tflops"], 4),
+                                         "kernel": "prefill_kernel<128> (paged mode)",
+                                         "traffic": traffic_all.get("prefill_paged_chunks8")}}
 
 
 def bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, dsl, ws, dout,

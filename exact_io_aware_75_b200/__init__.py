@@ -36,7 +36,7 @@ FA_ERR_TIMEOUT = -6
 FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
-EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks",
+EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa_fwd_paged",
            "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
            "fa_decode_paged_fp8",
@@ -67,6 +67,8 @@ def _load():
     lib.fa_fwd_varlen_sinks.restype = i
     lib.fa_decode_paged_sinks.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged_sinks.restype = i
+    lib.fa_fwd_paged.argtypes = [vp] * 9 + [i] * 11 + [f, i, vp]
+    lib.fa_fwd_paged.restype = i
     lib.fa_decode_paged_fp8.argtypes = [vp] * 10 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged_fp8.restype = i
     lib.fa_bwd_workspace_bytes.argtypes = [i] * 3
@@ -191,6 +193,37 @@ def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=No
                               _ptr(cu_seqlens), cu_seqlens.numel() - 1, T, int(max_seqlen),
                               Hq, Hkv, d, int(causal), int(window), float(scale), od,
                               _stream(stream)), "fa_fwd_varlen")
+    return out, lse
+
+
+def fwd_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, max_seqlen_q,
+              causal=True, window=0, scale=None, sinks=None, out_dtype=torch.bfloat16, out=None,
+              lse=None, return_lse=True, stream=None):
+    """Chunked prefill over a paged cache.  q [Tq,Hq,d] (each sequence's last L_q
+    tokens), caches [P,16,Hkv,d], block_table [S,maxp], cu_seqlens_q [S+1],
+    seq_lens_k [S] -> (O [Tq,Hq,d], LSE [Hq,Tq])."""
+    _need(q, torch.bfloat16, 3, "q")
+    _need(k_cache, torch.bfloat16, 4, "k_cache")
+    _need(v_cache, torch.bfloat16, 4, "v_cache")
+    _need(block_table, torch.int32, 2, "block_table")
+    _need(cu_seqlens_q, torch.int32, 1, "cu_seqlens_q")
+    _need(seq_lens_k, torch.int32, 1, "seq_lens_k")
+    T, Hq, d = q.shape
+    P, ps, Hkv, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+    od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    _check(_lib.fa_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                             _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(out), _ptr(lse),
+                             _ptr(sinks), cu_seqlens_q.numel() - 1, T, int(max_seqlen_q), P,
+                             Hq, Hkv, d, ps, block_table.shape[1], int(causal), int(window),
+                             float(scale), od, _stream(stream)), "fa_fwd_paged")
     return out, lse
 
 

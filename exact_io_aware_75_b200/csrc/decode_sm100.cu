@@ -357,9 +357,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
             group_transpose_sum<NV>(sc, lane);
             // lane holds flat indices [ds*NV/8, +HELD): token slot k = ds/2,
-            // heads hq0 .. hq0+HELD-1
+            // heads (ds & 1) * QPW/2 .. + HELD-1
             const int kslot = ds >> 1;
-            const int hq0 = (QPW >= 2) ? (ds & 1) * (QPW / 2) : 0;
             const bool tok_ok = (tg + 4 * kslot) < nvalid;
             float s_own[HELD];
             #pragma unroll
@@ -404,7 +403,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             float p_own[HELD];
             #pragma unroll
             for (int i = 0; i < HELD; ++i) {
-                const float mr = m_ref[hq0 + i];
+                // select, not m_ref[hq0 + i]: a run-time index would put
+                // m_ref in local memory
+                const float mr = (QPW >= 2 && (ds & 1)) ? m_ref[QPW / 2 + i] : m_ref[i];
                 p_own[i] = ex2(s_own[i] - (mr == -INFINITY ? 0.f : mr));
             }
             // ---- gather the token group's probabilities [4 slots][QPW]

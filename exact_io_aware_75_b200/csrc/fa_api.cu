@@ -221,6 +221,53 @@ int fa_fwd_varlen_sinks(const void *q, const void *k, const void *v, void *o, fl
                       max_seqlen, Hq, Hkv, d, causal, window, scale, o_dtype, stream);
 }
 
+int fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache,
+                 const int *block_table, const int *cu_seqlens_q, const int *seq_lens_k,
+                 void *o, float *lse, const float *sinks, int num_seqs, int total_q,
+                 int max_seqlen_q, int num_pages, int Hq, int Hkv, int d, int page_size,
+                 int max_pages_per_seq, int causal, int window, float scale, int o_dtype,
+                 void *stream) {
+    if (num_seqs < 0 || total_q < 0 || max_seqlen_q < 0 || num_pages < 0 ||
+        max_pages_per_seq <= 0)
+        return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
+    if (rc) return rc;
+    if (page_size != 16) return FA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || total_q == 0 || max_seqlen_q == 0) return FA_OK;
+    if (num_pages == 0) return FA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_table || !cu_seqlens_q || !seq_lens_k || !o)
+        return FA_ERR_INVALID_ARG;
+    if (total_q > INT32_MAX / 2 || (long long)num_pages * page_size > INT32_MAX / 2 ||
+        (long long)max_pages_per_seq * page_size > INT32_MAX / 2)
+        return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3) ||
+        (reinterpret_cast<uintptr_t>(seq_lens_k) & 3) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) ||
+        (sinks && (reinterpret_cast<uintptr_t>(sinks) & 3)))
+        return FA_ERR_ALIGNMENT;
+    fa::PrefillArgs a{};
+    a.q = q; a.k = k_cache; a.v = v_cache; a.o = o; a.lse = lse;
+    a.cu_seqlens = cu_seqlens_q;
+    a.num_seqs = num_seqs;
+    a.seqlen = 0;
+    a.total_tokens = total_q;
+    a.max_seqlen = max_seqlen_q;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.o_fp32 = o_dtype == FA_OUT_FP32;
+    a.sinks = sinks;
+    a.paged = 1;
+    a.block_table = block_table;
+    a.seq_lens_k = seq_lens_k;
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_bwd_workspace_bytes(int total_tokens, int Hq, int d) {
     return fa::bwd_workspace_bytes(total_tokens, Hq, d);
 }

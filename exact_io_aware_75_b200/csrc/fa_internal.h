@@ -22,6 +22,10 @@ struct PrefillArgs {
     float scale;
     int o_fp32;
     const float *sinks;     // device [Hq] learned sink logits; nullptr = none
+    // chunked prefill over a paged cache (k, v are the caches)
+    int paged;
+    const int *block_table, *seq_lens_k;
+    int max_pages, num_pages;
 };
 
 int launch_prefill(const PrefillArgs &a, cudaStream_t stream);

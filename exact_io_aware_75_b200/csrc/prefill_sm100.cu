@@ -64,6 +64,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // One score pair in kPolyPeriod takes the FMA-pipe exponential (0 = none).
 constexpr int kPolyPeriod = FA_POLY_PERIOD;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kPageRows = 16;                 // tokens per cache page (paged mode)
+constexpr int kPagesPerTile = 128 / kPageRows;
 
 template <int D>
 struct Cfg {
@@ -86,6 +88,13 @@ struct Params {
     const float *sinks;   // [Hq] learned sink logits, or nullptr
     int num_mblocks;   // 256-row blocks per sequence (of max_seqlen)
     int num_units;
+    // Chunked prefill over a paged cache: keys of sequence s come from its
+    // pages (block_table row s, 16 tokens per page), seq_lens_k[s] of them;
+    // its queries are the last L_q tokens (cu_seqlens holds the query packing).
+    int paged;
+    const int *block_table, *seq_lens_k;
+    const uint16_t *v_cache;
+    int max_pages, num_pages;
 };
 
 struct Unit {
@@ -93,10 +102,13 @@ struct Unit {
     int tok0;   // packed index of the sequence's first token
     int L;      // sequence length
     int q0;     // first query row of the unit, local to the sequence
+    int Lk;     // keys of the sequence (= L except for the paged chunked prefill)
+    int off;    // key position of query row 0 (Lk - L)
     int lo[2], hi[2];  // key-block range per tile, [lo, hi)
     int lo_all, hi_all;
 };
 
+template <bool PAGED>
 __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     const int per_mb = p.num_seqs * p.Hq;
     const int mb = p.num_mblocks - 1 - u / per_mb;
@@ -113,7 +125,18 @@ __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     }
     w.q0 = mb * 2 * kBlockM;
     if (w.L <= 0 || w.q0 >= w.L) return false;
-    const int nkb = (w.L + kBlockN - 1) / kBlockN;
+    w.Lk = w.L;
+    w.off = 0;
+    if constexpr (PAGED) {
+        const int Lk = __ldg(p.seq_lens_k + w.seq);
+        if (Lk < w.L || Lk > p.max_pages * kPageRows) {   // unusable lengths: skip, report
+            report_error(kDevErrInput);
+            return false;
+        }
+        w.Lk = Lk;
+        w.off = Lk - w.L;
+    }
+    const int nkb = (w.Lk + kBlockN - 1) / kBlockN;
     w.lo_all = 1 << 30;
     w.hi_all = 0;
     for (int t = 0; t < 2; ++t) {
@@ -121,9 +144,9 @@ __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
         if (r0 >= w.L) { w.lo[t] = w.hi[t] = 0; continue; }
         int lo = 0, hi = nkb;
         if (p.causal) {
-            const int last = min(r0 + kBlockM - 1, w.L - 1);
+            const int last = w.off + min(r0 + kBlockM - 1, w.L - 1);
             hi = min(nkb, last / kBlockN + 1);
-            if (p.window > 0) lo = max(0, r0 - p.window + 1) / kBlockN;
+            if (p.window > 0) lo = max(0, w.off + r0 - p.window + 1) / kBlockN;
         }
         w.lo[t] = lo;
         w.hi[t] = hi;
@@ -155,6 +178,7 @@ struct Shared {
 };
 
 // ------------------------------------------------------------- TMA producer
+// Dense and packed batches: one thread issues every copy.
 template <int D>
 __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                          const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
@@ -164,7 +188,7 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
     uint32_t kv_it = 0;
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit(u, p, w)) continue;
+        if (!get_unit<false>(u, p, w)) continue;
         for (int t = 0; t < 2; ++t) {
             if (w.lo[t] >= w.hi[t]) continue;
             if (!mbar_wait(&sh.q_empty[t], (q_uses[t] & 1) ^ 1, abort)) goto out;
@@ -200,8 +224,116 @@ out:
         if (q_uses[t]) mbar_drain_wait(&sh.q_full[t], (q_uses[t] - 1) & 1);
 }
 
-// ------------------------------------------------------------ MMA issuer
+// Chunked prefill over a paged cache: one warp.  A K or V tile is 8 cache
+// pages: lane p (< 8) looks up page p of the tile in
+// the block table and copies it (a 16-row box per 64 columns); pages past the
+// sequence's keys are read from beyond the cache's extent, which TMA fills with
+// zeros.  A page the sequence ends inside is copied for K (its tail keys are
+// masked) but for V the whole warp copies its valid rows and writes zeros
+// after them, because a masked key still multiplies its V row by P = 0 and
+// unused slots may hold NaN.  Every kv_full phase gets two arrivals: one with
+// the TMA byte count and one after the warp's own writes.
 template <int D>
+__device__ void producer_paged(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                         const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
+    using C = Cfg<D>;
+    volatile int *abort = &sh.abort;
+    const int lane = lane_id();
+    constexpr int kPageBytes = kPageRows * D * 2;     // one page of one KV head, all boxes
+    uint32_t q_uses[2] = {0, 0};
+    uint32_t kv_it = 0;
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit<true>(u, p, w)) continue;
+        for (int t = 0; t < 2; ++t) {
+            if (w.lo[t] >= w.hi[t]) continue;
+            if (!mbar_wait_warp(&sh.q_empty[t], (q_uses[t] & 1) ^ 1, abort)) goto out;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sh.q_full[t], C::kTileBytes);
+                for (int b = 0; b < D / 64; ++b)
+                    tma_load_3d(sQ + t * C::kTileBytes + b * C::kBoxBytes, tmQ, &sh.q_full[t],
+                                b * 64, w.h, w.tok0 + w.q0 + t * kBlockM);
+            }
+            ++q_uses[t];
+        }
+        for (int j = w.lo_all; j < w.hi_all; ++j) {
+            // paged: lane p < 8 holds page p of this key block (-1: past the keys)
+            int page = -1;
+            if (lane < kPagesPerTile) {
+                const int pidx = j * kPagesPerTile + lane;
+                if (pidx * kPageRows < w.Lk) {
+                    page = __ldg(p.block_table + (size_t)w.seq * p.max_pages + pidx);
+                    if (page < 0 || page >= p.num_pages) {
+                        report_error(kDevErrInput);
+                        page = 0;
+                    }
+                }
+            }
+            const int tail = w.Lk - j * kBlockN;          // valid keys in this tile (paged)
+            const int part = (tail > 0 && tail < kBlockN && (tail % kPageRows) != 0)
+                                 ? tail / kPageRows : -1;  // page the keys end inside
+            for (int kv = 0; kv < 2; ++kv) {
+                const int slot = kv_it % C::kStages;
+                const uint32_t use = kv_it / C::kStages;
+                uint8_t *dst = sKV + slot * C::kTileBytes;
+                if (!mbar_wait_warp(&sh.kv_empty[slot], (use & 1) ^ 1, abort)) goto out;
+                {
+                    const bool manual = kv == 1 && part >= 0;
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&sh.kv_full[slot],
+                                              C::kTileBytes - (manual ? kPageBytes : 0));
+                    __syncwarp();
+                    if (lane < kPagesPerTile && !(manual && lane == part)) {
+                        const int row = page >= 0 ? page * kPageRows : p.num_pages * kPageRows;
+                        for (int b = 0; b < D / 64; ++b)
+                            tma_load_3d(dst + b * C::kBoxBytes + lane * kPageRows * 128,
+                                        kv ? tmV : tmK, &sh.kv_full[slot], b * 64, w.kvh, row);
+                    }
+                    if (manual) {
+                        // V rows of the page the keys end inside: copy the
+                        // valid ones, zero the rest, in the 128-byte-swizzled
+                        // layout the TMA boxes use.
+                        const int vpage = __shfl_sync(0xffffffffu, page, part);
+                        const int valid = tail - part * kPageRows;
+                        constexpr int kChunks = kPageRows * (D / 8);   // 16-byte chunks
+                        for (int idx = lane; idx < kChunks; idx += 32) {
+                            const int srow = idx / (D / 8), rem = idx % (D / 8);
+                            const int b = rem >> 3, c = rem & 7;
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (srow < valid)
+                                v = __ldg(reinterpret_cast<const uint4 *>(
+                                    p.v_cache + ((size_t)(vpage * kPageRows + srow) * p.Hkv + w.kvh) * D +
+                                    b * 64 + c * 8));
+                            const int trow = part * kPageRows + srow;
+                            *reinterpret_cast<uint4 *>(dst + b * C::kBoxBytes + trow * 128 +
+                                                       ((c ^ (trow & 7)) << 4)) = v;
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sh.kv_full[slot]);
+                }
+                ++kv_it;
+            }
+        }
+    }
+    return;
+out:
+    // Leave no copy in flight: wait for the last load issued into each slot.
+    if (lane == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            if (kv_it > (uint32_t)s) {
+                const uint32_t last = (kv_it - 1 - s) / C::kStages;
+                mbar_drain_wait(&sh.kv_full[s], last & 1);
+            }
+        }
+        for (int t = 0; t < 2; ++t)
+            if (q_uses[t]) mbar_drain_wait(&sh.q_full[t], (q_uses[t] - 1) & 1);
+    }
+}
+
+// ------------------------------------------------------------ MMA issuer
+template <int D, bool PAGED>
 __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
     using C = Cfg<D>;
     volatile int *abort = &sh.abort;
@@ -262,7 +394,7 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
 
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit(u, p, w)) continue;
+        if (!get_unit<PAGED>(u, p, w)) continue;
         bool first_pv[2] = {true, true};
         for (int t = 0; t < 2; ++t) {
             if (w.lo[t] >= w.hi[t]) continue;
@@ -354,7 +486,7 @@ __device__ __forceinline__ void exp_half(const float (&v)[kHalf], float sl2, flo
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D>
+template <int D, bool PAGED>
 __device__ void softmax_wg(const Params &p, Shared &sh) {
     using C = Cfg<D>;
     volatile int *abort = &sh.abort;
@@ -369,8 +501,10 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
 
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit(u, p, w)) continue;
-        const int lo = w.lo[t], hi = w.hi[t];
+        if (!get_unit<PAGED>(u, p, w)) continue;
+        // (selects, not w.lo[t]: a run-time index would keep the unit in
+        // local memory)
+        const int lo = t ? w.lo[1] : w.lo[0], hi = t ? w.hi[1] : w.hi[0];
         if (lo >= hi) continue;
         const int row = w.q0 + t * kBlockM + r;    // row index within the sequence
         const int rmin = w.q0 + t * kBlockM, rmax = rmin + kBlockM - 1;
@@ -381,12 +515,19 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
             tc_fence_after();
             const bool first = (j == lo);
             const int k0 = j * kBlockN;
-            const bool edge = (k0 + kBlockN > w.L) || (p.causal && k0 + kBlockN - 1 > rmin) ||
-                              (p.window > 0 && k0 <= rmax - p.window);
-            // visible keys of this row in the tile: c in [c_lo, c_hi)
-            int c_hi = w.L - k0;
-            if (p.causal) c_hi = min(c_hi, row + 1 - k0);
-            const int c_lo = (p.window > 0) ? row - p.window + 1 - k0 : 0;
+            // keys of the sequence and the key position of query row 0:
+            // L and 0 for dense and packed batches
+            const int Lk = PAGED ? w.Lk : w.L;
+            const int off = PAGED ? w.off : 0;
+            const bool edge = (k0 + kBlockN > Lk) ||
+                              (p.causal && k0 + kBlockN - 1 > off + rmin) ||
+                              (p.window > 0 && k0 <= off + rmax - p.window);
+            // visible keys of this row in the tile: c in [c_lo, c_hi); the
+            // row's key position is off + row
+            const int pos = off + row;
+            int c_hi = Lk - k0;
+            if (p.causal) c_hi = min(c_hi, pos + 1 - k0);
+            const int c_lo = (p.window > 0) ? pos - p.window + 1 - k0 : 0;
             // Scores in two halves of 64 keys: the second half's TMEM load is
             // in flight while the first half is masked and reduced.
             float sA[kHalf], sB[kHalf];
@@ -542,7 +683,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
     }
 }
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -566,7 +707,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mbar_init(&sh.o_empty[t], 4);
         }
         for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&sh.kv_full[s], 1);
+            mbar_init(&sh.kv_full[s], PAGED ? 2 : 1);
             mbar_init(&sh.kv_empty[s], 1);
         }
         mbar_init(&sh.drain, 1);
@@ -585,13 +726,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (warp < kSoftmaxWarps) {
         regs_increase<kRegsSoftmax>();
-        softmax_wg<D>(p, sh);
+        softmax_wg<D, PAGED>(p, sh);
     } else {
         regs_decrease<kRegsControl>();
         if (warp == kWarpTma) {
-            if (lane_id() == 0) producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+            if constexpr (PAGED)
+                producer_paged<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+            else if (lane_id() == 0)
+                producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
         } else if (warp == kWarpMma) {
-            if (lane_id() == 0) mma_issuer<D>(p, sh, sQ, sKV);
+            if (lane_id() == 0) mma_issuer<D, PAGED>(p, sh, sQ, sKV);
         }
     }
     __syncwarp();
@@ -613,12 +757,16 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     using C = Cfg<D>;
     alignas(64) CUtensorMap tq, tk, tv;
     const uint64_t T = (uint64_t)a.total_tokens;
+    // K/V: the packed tokens (dense, varlen), or the cache's num_pages * 16
+    // rows read one 16-row page box at a time (paged)
+    const uint64_t TK = a.paged ? (uint64_t)a.num_pages * kPageRows : T;
+    const uint32_t kv_box = a.paged ? kPageRows : kBlockN;
     if (encode_tensor_map_3d(&tq, a.q, 2, D, a.Hq, T, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2,
                              64, 1, kBlockM, 128) ||
-        encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kBlockN, 128) ||
-        encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, T, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kBlockN, 128))
+        encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kv_box, 128) ||
+        encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kv_box, 128))
         return -5;
     Params p;
     p.o = a.o;
@@ -636,6 +784,12 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.o_fp32 = a.o_fp32;
     p.sinks = a.sinks;
+    p.paged = a.paged;
+    p.block_table = a.block_table;
+    p.seq_lens_k = a.seq_lens_k;
+    p.v_cache = static_cast<const uint16_t *>(a.v);
+    p.max_pages = a.max_pages;
+    p.num_pages = a.num_pages;
     p.num_mblocks = (a.max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM);
     const long long units = (long long)p.num_mblocks * a.num_seqs * a.Hq;
     if (units <= 0) return 0;
@@ -643,11 +797,12 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.num_units = (int)units;
     // Setting the attribute is idempotent and cheap; do it on every call so
     // that any device the caller switches to is covered.
-    if (cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kernel = a.paged ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemBytes) != cudaSuccess)
         return -5;
     const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
-    prefill_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 

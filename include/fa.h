@@ -98,6 +98,36 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                   float scale, int o_dtype, void *stream);
 
 /*
+ * Chunked prefill over a paged cache ("Chunked-prefill serving in vLLM pairs
+ * FlashAttention with KV paging", FlashAttention explainer, real-world
+ * examples).  Sequence s has seq_lens_k[s] tokens in its pages -- the earlier
+ * context plus this chunk, whose K/V the caller has already written -- and
+ * its L_q = cu_seqlens_q[s+1] - cu_seqlens_q[s] queries are the LAST L_q of
+ * them: query i of the chunk sits at position seq_lens_k[s] - L_q + i and,
+ * with causal, sees keys 0 .. seq_lens_k[s] - L_q + i (window W: the last W
+ * of those).  L_q = 1 is the decode; L_q = seq_lens_k is a plain prefill.
+ *   q            [total_q, Hq, d] bf16, device (chunks packed by cu_seqlens_q)
+ *   k_cache,
+ *   v_cache      [num_pages, page_size, Hkv, d] bf16, device
+ *   block_table  [num_seqs, max_pages_per_seq] int32, device (as fa_decode_paged)
+ *   cu_seqlens_q [num_seqs + 1] int32, device; seq_lens_k [num_seqs] int32,
+ *                device, with L_q <= seq_lens_k[s] <= max_pages_per_seq * 16
+ *                (a sequence that breaks this is skipped, its rows left
+ *                unwritten, and fa_check_device_error reports
+ *                FA_ERR_INVALID_ARG)
+ *   o            [total_q, Hq, d] bf16 or fp32, written; lse [Hq, total_q] or NULL
+ *   sinks        [Hq] fp32 learned sink logits, or NULL (as fa_fwd_sinks)
+ *   page_size    16.  max_seqlen_q >= every L_q.
+ * Cache slots past seq_lens_k may hold anything, NaN included.
+ */
+int fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache,
+                 const int *block_table, const int *cu_seqlens_q, const int *seq_lens_k,
+                 void *o, float *lse, const float *sinks, int num_seqs, int total_q,
+                 int max_seqlen_q, int num_pages, int Hq, int Hkv, int d, int page_size,
+                 int max_pages_per_seq, int causal, int window, float scale, int o_dtype,
+                 void *stream);
+
+/*
  * Bytes of workspace fa_bwd / fa_bwd_varlen need for total_tokens tokens
  * (B * N for a dense batch): an fp32 dQ accumulator [total, Hq, d] and the
  * row terms D_i = dO_i . O_i.  0 for an unsupported combination (d != 128).

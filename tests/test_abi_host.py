@@ -183,6 +183,31 @@ def test_fp8_decode_rejects(fa):
     assert lib.fa_decode_paged_fp8(*base, P, P, *t3) == -2
 
 
+def paged_fwd(fa, **kw):
+    a = dict(q=P, kc=P, vc=P, bt=P, cu=P, sl=P, o=P, lse=0, sinks=0, S=2, Tq=100, maxq=64,
+             npages=40, Hq=8, Hkv=2, d=128, ps=16, maxp=8, causal=1, window=0, scale=0.1,
+             od=0)
+    a.update(kw)
+    return fa.library().fa_fwd_paged(a["q"], a["kc"], a["vc"], a["bt"], a["cu"], a["sl"],
+                                     a["o"], a["lse"], a["sinks"], a["S"], a["Tq"], a["maxq"],
+                                     a["npages"], a["Hq"], a["Hkv"], a["d"], a["ps"], a["maxp"],
+                                     a["causal"], a["window"], a["scale"], a["od"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), -1), (dict(ps=8), -2), (dict(d=96), -2), (dict(window=4, causal=0), -2),
+    (dict(npages=0), -1), (dict(bt=0), -1), (dict(cu=0), -1), (dict(sl=0), -1), (dict(q=0), -1),
+    (dict(kc=P + 8), -3), (dict(cu=P + 2), -3), (dict(sinks=P + 1), -3), (dict(lse=P + 2), -3),
+    (dict(maxp=0), -1), (dict(S=-1), -1), (dict(od=5), -1)])
+def test_fwd_paged_rejects(fa, kw, status):
+    assert paged_fwd(fa, **kw) == status
+
+
+def test_fwd_paged_empty_is_noop(fa):
+    assert paged_fwd(fa, S=0, q=0) == 0
+    assert paged_fwd(fa, Tq=0, q=0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """Importing the binding with the shared library absent raises, rather
     than falling back to anything else."""

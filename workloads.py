@@ -177,6 +177,39 @@ def paged(lens=None, num_seqs=64, len_lo=4096, len_hi=32768, Hq=32, Hkv=8,
 
 
 @dataclass
+class PagedPrefill:
+    q: torch.Tensor            # [total_q, Hq, d] bf16: each sequence's last L_q tokens
+    k_cache: torch.Tensor      # [num_pages, page_size, Hkv, d] bf16
+    v_cache: torch.Tensor
+    block_table: torch.Tensor  # [S, max_pages] int32
+    cu_seqlens_q: torch.Tensor  # [S + 1] int32
+    seq_lens_k: torch.Tensor   # [S] int32
+    lens_q: list
+    scale: float
+
+    @property
+    def max_seqlen_q(self) -> int:
+        return max(self.lens_q) if self.lens_q else 0
+
+
+def paged_prefill(lens_k, lens_q, Hq=32, Hkv=8, d=128, seed=0, scale=None, poison=False,
+                  spare_pages=0) -> PagedPrefill:
+    """A chunked-prefill batch: the paged cache of ``paged(lens=lens_k)`` and,
+    per sequence, L_q new query tokens (its last L_q positions), drawn from a
+    generator of their own (seed + 2)."""
+    base = paged(lens=lens_k, Hq=Hq, Hkv=Hkv, d=d, seed=seed, scale=scale, poison=poison,
+                 spare_pages=spare_pages)
+    lens_q = [int(x) for x in lens_q]
+    g = torch.Generator("cpu").manual_seed(seed + 2)
+    q = randn_bf16((sum(lens_q), Hq, d), g)
+    cu = [0]
+    for L in lens_q:
+        cu.append(cu[-1] + L)
+    return PagedPrefill(q, base.k_cache, base.v_cache, base.block_table,
+                        torch.tensor(cu, dtype=torch.int32), base.seq_lens, lens_q, base.scale)
+
+
+@dataclass
 class PagedFP8:
     q: torch.Tensor            # [S, Hq, d] bf16
     k_codes: torch.Tensor      # [num_pages, page_size, Hkv, d] uint8 (FP8 E4M3 codes)
