@@ -76,6 +76,10 @@ def lib():
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _f64p, _f64p, _f64p]
         L.oracle_attn_bwd_varlen.restype = ctypes.c_int
+        L.oracle_attn_bwd_varlen_sinks.argtypes = [
+            _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, _f64p, _f64p, _f64p, _f64p, _f64p]
+        L.oracle_attn_bwd_varlen_sinks.restype = ctypes.c_int
         L.oracle_attn_bwd_dq_rows.argtypes = [
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
@@ -377,3 +381,23 @@ def prefill_paged(q, k_cache, v_cache, block_table, cu_seqlens_q, seq_lens_k, ca
                                       bt.shape[1], P, int(causal), int(window), float(scale),
                                       sp, o, lse), "prefill_paged")
     return o, np.ascontiguousarray(lse.T)
+
+
+def attn_bwd_sinks(q, k, v, dout, sinks, causal=False, window=0, scale=None):
+    """Dense-batch gradients with learned sinks: -> dQ, dK, dV, dsinks [Hq]."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    sk = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(Hq))
+    dq = np.empty((B * N, Hq, d), np.float64)
+    dk = np.empty((B * N, Hkv, d), np.float64)
+    dv = np.empty((B * N, Hkv, d), np.float64)
+    ds = np.empty((Hq,), np.float64)
+    _check(lib().oracle_attn_bwd_varlen_sinks(
+        qb.reshape(B * N, Hq, d), kb.reshape(B * N, Hkv, d), vb.reshape(B * N, Hkv, d),
+        db.reshape(B * N, Hq, d), cu, B, Hq, Hkv, d, int(causal), int(window), float(scale),
+        sk, dq, dk, dv, ds), "attn_bwd_sinks")
+    return (dq.reshape(B, N, Hq, d), dk.reshape(B, N, Hkv, d), dv.reshape(B, N, Hkv, d), ds)

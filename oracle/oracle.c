@@ -427,11 +427,12 @@ int oracle_lse_combine(const double *o_parts, const double *lse_parts,
  */
 static void bwd_row(const double *qd, const double *dod, int d, int64_t nkeys,
                     const uint16_t *const *kp, const uint16_t *const *vp,
-                    const unsigned char *vis, double scale, double *sc, double *p,
-                    double *dp, double *ds, double *orow, double *dq)
+                    const unsigned char *vis, double scale, double sink, double *sc,
+                    double *p, double *dp, double *ds, double *orow, double *dq,
+                    double *lse_out, double *D_out)
 {
     double lse_i, D = 0.0;
-    attend_row(qd, d, nkeys, kp, vp, vis, scale, sc, orow, &lse_i, p);
+    attend_row_sink(qd, d, nkeys, kp, vp, vis, scale, sink, sc, orow, &lse_i, p);
     /* dP and the Jacobian term D_i */
     for (int64_t j = 0; j < nkeys; ++j) {
         dp[j] = 0.0;
@@ -445,12 +446,15 @@ static void bwd_row(const double *qd, const double *dod, int d, int64_t nkeys,
         if (!vis[j]) continue;
         for (int c = 0; c < d; ++c) dq[c] += scale * ds[j] * widen(kp[j][c]);
     }
+    if (lse_out) *lse_out = lse_i;
+    if (D_out) *D_out = D;
 }
 
-int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                           const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
-                           int Hq, int Hkv, int d, int causal, int window, double scale,
-                           double *dq, double *dk, double *dv)
+static int attn_bwd_varlen_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                 const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                                 int Hq, int Hkv, int d, int causal, int window, double scale,
+                                 const double *sinks, double *dq, double *dk, double *dv,
+                                 double *dsinks)
 {
     if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
     const int group = Hq / Hkv;
@@ -459,6 +463,13 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
         int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
         if (L < 0) return -1;
         if (L > maxlen) maxlen = L;
+    }
+    /* per-(sequence, KV head) partial sums of the sink gradient, summed in
+       a fixed order afterwards so the result does not depend on threads */
+    double *part = NULL;
+    if (dsinks) {
+        part = (double *)calloc((size_t)num_seqs * Hq + 1, sizeof(double));
+        if (!part) return -2;
     }
     int bad = 0;
 #pragma omp parallel
@@ -500,8 +511,13 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
                         }
                         for (int64_t j = 0; j < L; ++j)
                             vis[j] = (unsigned char)allowed(i, j, causal, window);
-                        bwd_row(qd, dod, d, L, kp, vp, vis, scale, sc, p, dp, ds, orow,
-                                dq + row);
+                        double lse_i, D_i;
+                        const double z = sinks ? sinks[h] : -INFINITY;
+                        bwd_row(qd, dod, d, L, kp, vp, vis, scale, z, sc, p, dp, ds, orow,
+                                dq + row, &lse_i, &D_i);
+                        /* the sink's weight exp(z - LSE_i) times (0 - D_i) */
+                        if (part && z != -INFINITY)
+                            part[task * group + (h - g * group)] -= exp(z - lse_i) * D_i;
                         for (int64_t j = 0; j < L; ++j) {
                             if (!vis[j]) continue;
                             double *dkj = dk + ((start + j) * Hkv + g) * (int64_t)d;
@@ -518,7 +534,42 @@ int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t 
         free(sc); free(p); free(dp); free(ds); free(qd); free(dod); free(orow);
         free(kp); free(vp); free(vis);
     }
+    if (dsinks) {
+        for (int h = 0; h < Hq; ++h) {
+            double acc = 0.0;
+            for (int seq = 0; seq < num_seqs; ++seq)
+                acc += part[((int64_t)seq * Hkv + h / group) * group + h % group];
+            dsinks[h] = acc;
+        }
+        free(part);
+    }
     return bad ? -2 : 0;
+}
+
+int oracle_attn_bwd_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                           int Hq, int Hkv, int d, int causal, int window, double scale,
+                           double *dq, double *dk, double *dv)
+{
+    return attn_bwd_varlen_sinks(q, k, v, dout, cu_seqlens, num_seqs, Hq, Hkv, d, causal,
+                                 window, scale, NULL, dq, dk, dv, NULL);
+}
+
+/*
+ * The same with a learned sink logit per query head (sinks[Hq]): P is the
+ * softmax with the sink in its denominator, and dsinks[h] = d Loss / d z_h =
+ * sum over rows of head h of exp(z_h - LSE_i) * (0 - D_i) (the sink's value
+ * is zero, so its dP is 0).
+ */
+int oracle_attn_bwd_varlen_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                 const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                                 int Hq, int Hkv, int d, int causal, int window, double scale,
+                                 const double *sinks, double *dq, double *dk, double *dv,
+                                 double *dsinks)
+{
+    if (!sinks || !dsinks) return -1;
+    return attn_bwd_varlen_sinks(q, k, v, dout, cu_seqlens, num_seqs, Hq, Hkv, d, causal,
+                                 window, scale, sinks, dq, dk, dv, dsinks);
 }
 
 /*
@@ -578,8 +629,8 @@ int oracle_attn_bwd_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t
                     vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
                     vis[j] = (unsigned char)allowed(i, j, causal, window);
                 }
-                bwd_row(qd, dod, d, L, kp, vp, vis, scale, sc, p, dp, ds, orow,
-                        dq + (r * Hq + h) * (int64_t)d);
+                bwd_row(qd, dod, d, L, kp, vp, vis, scale, -INFINITY, sc, p, dp, ds, orow,
+                        dq + (r * Hq + h) * (int64_t)d, NULL, NULL);
             }
         }
         free(sc); free(p); free(dp); free(ds); free(qd); free(dod); free(orow);

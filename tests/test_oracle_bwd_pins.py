@@ -159,3 +159,52 @@ def test_dq_rows_match_full_backward():
         rows = [0, 5, 39, 40, 41, 100, 116]
         got = oracle.attn_bwd_dq_rows(q, k, v, do, cu, rows, causal, window, 0.3)
         assert np.array_equal(got, dq[rows])
+
+
+def autograd_grads_sinks(q, k, v, dout, sinks, causal, window, scale):
+    """fp64 autograd with the sink as one extra score column (value zero)."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    qd = q.double().requires_grad_()
+    kd = k.double().requires_grad_()
+    vd = v.double().requires_grad_()
+    z = torch.tensor(sinks, dtype=torch.float64).requires_grad_()
+    kk = kd.repeat_interleave(Hq // Hkv, dim=2)
+    vv = vd.repeat_interleave(Hq // Hkv, dim=2)
+    s = torch.einsum("bihc,bjhc->bhij", qd, kk) * scale
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    allowed = torch.ones(N, N, dtype=torch.bool)
+    if causal:
+        allowed &= j <= i
+        if window > 0:
+            allowed &= j > i - window
+    s = s.masked_fill(~allowed, float("-inf"))
+    zc = z.view(1, Hq, 1, 1).expand(B, Hq, N, 1)
+    pr = torch.softmax(torch.cat([s, zc], dim=-1), dim=-1)[..., :N]
+    o = torch.einsum("bhij,bjhc->bihc", pr, vv)
+    (o * dout.double()).sum().backward()
+    return qd.grad.numpy(), kd.grad.numpy(), vd.grad.numpy(), z.grad.numpy()
+
+
+@pytest.mark.parametrize("causal,window", [(0, 0), (1, 0), (1, 6)])
+def test_backward_with_sinks_matches_autograd(causal, window):
+    B, N, Hq, Hkv, d = 2, 29, 4, 2, 16
+    q, k, v = rnd((B, N, Hq, d), 51), rnd((B, N, Hkv, d), 52), rnd((B, N, Hkv, d), 53)
+    do = rnd((B, N, Hq, d), 54)
+    z = [0.7, -1.3, 2.5, 0.0]
+    dq, dk, dv, dz = oracle.attn_bwd_sinks(q, k, v, do, z, causal, window, 0.25)
+    rq, rk, rv, rz = autograd_grads_sinks(q, k, v, do, z, causal, window, 0.25)
+    for got, ref in ((dq, rq), (dk, rk), (dv, rv), (dz, rz)):
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_minus_inf_sinks_backward_is_plain():
+    B, N, Hq, Hkv, d = 1, 33, 2, 1, 16
+    q, k, v = rnd((B, N, Hq, d), 61), rnd((B, N, Hkv, d), 62), rnd((B, N, Hkv, d), 63)
+    do = rnd((B, N, Hq, d), 64)
+    a = oracle.attn_bwd(q, k, v, do, 1, 0, 0.3)
+    b = oracle.attn_bwd_sinks(q, k, v, do, [-math.inf, -math.inf], 1, 0, 0.3)
+    for x, y in zip(a, b[:3]):
+        assert np.array_equal(x, y)
+    assert np.all(b[3] == 0.0)
