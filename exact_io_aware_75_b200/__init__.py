@@ -37,7 +37,8 @@ FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa_fwd_paged",
-           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen",
+           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen", "fa_bwd_sinks",
+           "fa_bwd_varlen_sinks",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
            "fa_decode_paged_fp8",
            "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
@@ -77,6 +78,10 @@ def _load():
     lib.fa_bwd.restype = i
     lib.fa_bwd_varlen.argtypes = [vp] * 10 + [i] * 8 + [f, vp, sz, vp]
     lib.fa_bwd_varlen.restype = i
+    lib.fa_bwd_sinks.argtypes = [vp] * 11 + [i] * 7 + [f, vp, sz, vp]
+    lib.fa_bwd_sinks.restype = i
+    lib.fa_bwd_varlen_sinks.argtypes = [vp] * 12 + [i] * 8 + [f, vp, sz, vp]
+    lib.fa_bwd_varlen_sinks.restype = i
     lib.fa_decode_workspace_bytes.argtypes = [i] * 5
     lib.fa_decode_workspace_bytes.restype = sz
     lib.fa_decode_paged.argtypes = [vp] * 7 + [i] * 7 + [f, vp, sz, vp]
@@ -232,9 +237,10 @@ def bwd_workspace_bytes(total_tokens, Hq, d) -> int:
 
 
 def bwd(q, k, v, o, dout, lse, causal=False, window=0, scale=None, dq=None, dk=None, dv=None,
-        workspace=None, stream=None):
+        workspace=None, stream=None, sinks=None, dsinks=None):
     """Dense backward.  q/o/dout [B,N,Hq,d], k/v [B,N,Hkv,d] bf16, lse [B,Hq,N] fp32
-    (from fwd) -> (dQ, dK, dV) bf16."""
+    (from fwd) -> (dQ, dK, dV) bf16; with ``sinks`` (the forward's sink logits,
+    fp32 [Hq]) fa_bwd_sinks, returning (dQ, dK, dV, dsinks)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _need(t, torch.bfloat16, 4, n)
     _need(lse, torch.float32, 3, "lse")
@@ -252,6 +258,16 @@ def bwd(q, k, v, o, dout, lse, causal=False, window=0, scale=None, dq=None, dk=N
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    if sinks is not None:
+        _need(sinks, torch.float32, 1, "sinks")
+        if dsinks is None:
+            dsinks = torch.empty((Hq,), dtype=torch.float32, device=q.device)
+        _check(_lib.fa_bwd_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                 _ptr(sinks), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsinks), B, Hq,
+                                 Hkv, N, d, int(causal), int(window), float(scale),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)),
+               "fa_bwd_sinks")
+        return dq, dk, dv, dsinks
     _check(_lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                        _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, int(causal), int(window),
                        float(scale), _ptr(workspace), workspace.numel(), _stream(stream)),

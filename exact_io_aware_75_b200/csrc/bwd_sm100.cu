@@ -584,6 +584,40 @@ bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dou
     }
 }
 
+// Gradient of a learned sink logit z_h: the sink is one more score with a
+// zero value, so its dP is 0 and d Loss / d z_h = sum over the rows of head h
+// of exp(z_h - LSE_i) * (0 - D_i).  One block per head; a fixed-order tree
+// reduction (deterministic).
+__global__ void __launch_bounds__(256)
+bwd_dsink_kernel(const float *__restrict__ lse, const float *__restrict__ dd,
+                 const float *__restrict__ sinks, float *__restrict__ dsinks, int num_seqs,
+                 int Hq, int seqlen, int total, int dense) {
+    const int h = blockIdx.x;
+    const float z = sinks[h];
+    float acc = 0.f;
+    if (z != -INFINITY) {
+        const long long rows = dense ? (long long)num_seqs * seqlen : total;
+        for (long long r = threadIdx.x; r < rows; r += blockDim.x) {
+            size_t idx;
+            if (dense)
+                idx = ((size_t)(r / seqlen) * Hq + h) * seqlen + (r % seqlen);
+            else
+                idx = (size_t)h * total + r;
+            acc -= __expf(z - lse[idx]) * dd[idx];
+        }
+    }
+    #pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    __shared__ float part[8];
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < 8; ++w) t += part[w];
+        dsinks[h] = t;
+    }
+}
+
 // dQ (bf16) = the fp32 accumulator, eight elements per thread.
 __global__ void __launch_bounds__(256)
 bwd_convert_kernel(const float *__restrict__ acc, uint16_t *__restrict__ dq, long long n8) {
@@ -622,6 +656,12 @@ int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
         static_cast<const uint16_t *>(a.o), static_cast<const uint16_t *>(a.dout), dd, dq_acc,
         (int)total, a.Hq, a.seqlen, a.cu_seqlens ? 0 : 1);
     if (cudaGetLastError() != cudaSuccess) return -5;
+    if (a.sinks) {
+        bwd_dsink_kernel<<<a.Hq, 256, 0, stream>>>(a.lse, dd, a.sinks, a.dsinks, a.num_seqs,
+                                                   a.Hq, a.seqlen, (int)total,
+                                                   a.cu_seqlens ? 0 : 1);
+        if (cudaGetLastError() != cudaSuccess) return -5;
+    }
 
     alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
     const uint64_t T = (uint64_t)total;

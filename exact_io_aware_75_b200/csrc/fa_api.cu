@@ -299,10 +299,15 @@ int bwd_common(const void *q, const void *k, const void *v, const void *o, const
 
 extern "C" {
 
-int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
-           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N, int d,
-           int causal, int window, float scale, void *workspace, size_t workspace_bytes,
-           void *stream) {
+}  // extern "C"
+
+namespace {
+
+int bwd_dense_call(const void *q, const void *k, const void *v, const void *o,
+                   const void *dout, const float *lse, const float *sinks, void *dq, void *dk,
+                   void *dv, float *dsinks, int B, int Hq, int Hkv, int N, int d, int causal,
+                   int window, float scale, void *workspace, size_t workspace_bytes,
+                   void *stream) {
     if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
     if (rc) return rc;
@@ -323,14 +328,17 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
     a.window = window > 0 ? window : 0;
     a.scale = scale;
     a.workspace = workspace;
+    a.sinks = sinks;
+    a.dsinks = dsinks;
     return map_rc(fa::launch_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 
-int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
-                  const void *dout, const float *lse, void *dq, void *dk, void *dv,
-                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
-                  int Hq, int Hkv, int d, int causal, int window, float scale, void *workspace,
-                  size_t workspace_bytes, void *stream) {
+int bwd_varlen_call(const void *q, const void *k, const void *v, const void *o,
+                    const void *dout, const float *lse, const float *sinks, void *dq, void *dk,
+                    void *dv, float *dsinks, const int *cu_seqlens, int num_seqs,
+                    int total_tokens, int max_seqlen, int Hq, int Hkv, int d, int causal,
+                    int window, float scale, void *workspace, size_t workspace_bytes,
+                    void *stream) {
     if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
     if (rc) return rc;
@@ -353,7 +361,61 @@ int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
     a.window = window > 0 ? window : 0;
     a.scale = scale;
     a.workspace = workspace;
+    a.sinks = sinks;
+    a.dsinks = dsinks;
     return map_rc(fa::launch_bwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+int check_sink_pair(const float *sinks, const float *dsinks) {
+    if (!sinks || !dsinks) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(sinks) & 3) || (reinterpret_cast<uintptr_t>(dsinks) & 3))
+        return FA_ERR_ALIGNMENT;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N, int d,
+           int causal, int window, float scale, void *workspace, size_t workspace_bytes,
+           void *stream) {
+    return bwd_dense_call(q, k, v, o, dout, lse, nullptr, dq, dk, dv, nullptr, B, Hq, Hkv, N,
+                          d, causal, window, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_sinks(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, const float *sinks, void *dq, void *dk, void *dv,
+                 float *dsinks, int B, int Hq, int Hkv, int N, int d, int causal, int window,
+                 float scale, void *workspace, size_t workspace_bytes, void *stream) {
+    const int rc = check_sink_pair(sinks, dsinks);
+    if (rc) return rc;
+    return bwd_dense_call(q, k, v, o, dout, lse, sinks, dq, dk, dv, dsinks, B, Hq, Hkv, N, d,
+                          causal, window, scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                  const int *cu_seqlens, int num_seqs, int total_tokens, int max_seqlen,
+                  int Hq, int Hkv, int d, int causal, int window, float scale, void *workspace,
+                  size_t workspace_bytes, void *stream) {
+    return bwd_varlen_call(q, k, v, o, dout, lse, nullptr, dq, dk, dv, nullptr, cu_seqlens,
+                           num_seqs, total_tokens, max_seqlen, Hq, Hkv, d, causal, window,
+                           scale, workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_varlen_sinks(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *lse, const float *sinks, void *dq,
+                        void *dk, void *dv, float *dsinks, const int *cu_seqlens, int num_seqs,
+                        int total_tokens, int max_seqlen, int Hq, int Hkv, int d, int causal,
+                        int window, float scale, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    const int rc = check_sink_pair(sinks, dsinks);
+    if (rc) return rc;
+    return bwd_varlen_call(q, k, v, o, dout, lse, sinks, dq, dk, dv, dsinks, cu_seqlens,
+                           num_seqs, total_tokens, max_seqlen, Hq, Hkv, d, causal, window,
+                           scale, workspace, workspace_bytes, stream);
 }
 
 size_t fa_decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size,

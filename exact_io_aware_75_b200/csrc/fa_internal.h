@@ -58,6 +58,8 @@ struct BwdArgs {
     int causal, window;
     float scale;
     void *workspace;
+    const float *sinks;     // [Hq] learned sink logits, or nullptr
+    float *dsinks;          // [Hq] their gradient (written when sinks is set)
 };
 
 size_t bwd_workspace_bytes(long long total_tokens, int Hq, int d);

@@ -180,6 +180,26 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const voi
            size_t workspace_bytes, void *stream);
 
 /*
+ * fa_bwd / fa_bwd_varlen for a forward run with learned sinks (fa_fwd_sinks,
+ * fa_fwd_varlen_sinks): lse is that forward's LSE (it includes the sink
+ * term), so dQ, dK, dV follow as without sinks; additionally
+ * dsinks [Hq] fp32, device, written = d Loss / d z_h = sum over the rows of
+ * head h of exp(z_h - LSE_i) * (0 - D_i), D_i = dO_i . O_i (the sink is one
+ * more score with a zero value).  sinks and dsinks must be non-NULL and
+ * 4-byte aligned; other arguments as for fa_bwd / fa_bwd_varlen.
+ */
+int fa_bwd_sinks(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, const float *sinks, void *dq, void *dk, void *dv,
+                 float *dsinks, int B, int Hq, int Hkv, int N, int d, int causal, int window,
+                 float scale, void *workspace, size_t workspace_bytes, void *stream);
+int fa_bwd_varlen_sinks(const void *q, const void *k, const void *v, const void *o,
+                        const void *dout, const float *lse, const float *sinks, void *dq,
+                        void *dk, void *dv, float *dsinks, const int *cu_seqlens, int num_seqs,
+                        int total_tokens, int max_seqlen, int Hq, int Hkv, int d, int causal,
+                        int window, float scale, void *workspace, size_t workspace_bytes,
+                        void *stream);
+
+/*
  * Backward of packed variable-length prefill (fa_fwd_varlen's layouts: q, o,
  * dout, dq [total, Hq, d]; k, v, dk, dv [total, Hkv, d]; lse [Hq, total];
  * cu_seqlens as there).  Workspace: fa_bwd_workspace_bytes(total_tokens, Hq, d).

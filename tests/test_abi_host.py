@@ -136,6 +136,17 @@ def test_bwd_empty_is_noop(fa):
     assert bwd(fa, N=0, q=0, ws=0) == 0
 
 
+def test_bwd_sinks_rejects(fa):
+    lib = fa.library()
+    head = [P] * 6                    # q, k, v, o, dout, lse
+    tail = [1, 4, 2, 256, 128, 1, 0, 0.125, P, 1 << 30, None]
+    assert lib.fa_bwd_sinks(*head, None, P, P, P, P, *tail) == -1          # sinks NULL
+    assert lib.fa_bwd_sinks(*head, P, P, P, P, None, *tail) == -1          # dsinks NULL
+    assert lib.fa_bwd_sinks(*head, P + 2, P, P, P, P, *tail) == -3
+    assert lib.fa_bwd_varlen_sinks(*head, P, P, P, P, P + 1, P, 2, 100, 60, 4, 2, 128, 1, 0,
+                                   0.1, P, 1 << 30, None) == -3
+
+
 def test_bwd_varlen_rejects(fa):
     lib = fa.library()
     args = [P] * 9

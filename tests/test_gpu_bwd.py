@@ -145,3 +145,27 @@ def test_gqa4k_full_size(fa):
     dv64 = dv.double().cpu()[0]
     ref_v = do.double()[0].view(N, Hkv, Hq // Hkv, d).sum(dim=(0, 2))
     assert ((dv64.sum(0) - ref_v).abs() <= 1e-3 * dv64.abs().sum(0) + 1e-2).all()
+
+
+def test_sinks_backward(fa):
+    """Backward of a forward with learned sinks: dQ, dK, dV and the sink-logit
+    gradient against the oracle (dsinks within the same relative bound)."""
+    import math
+    B, Hq, Hkv, N = 1, 8, 2, 333
+    inp = workloads.dense(B, Hq, Hkv, N, 128, causal=True, seed=41)
+    do = workloads.grad_out((B, N, Hq, 128), seed=41)
+    g = torch.Generator("cpu").manual_seed(41)
+    z = torch.randn(Hq, generator=g) * 2.0
+    z[0] = -math.inf
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    o, lse = fa.fwd(q, k, v, True, 0, inp.scale, sinks=z.cuda())
+    dq, dk, dv, dz = fa.bwd(q, k, v, o, do.cuda(), lse, True, 0, inp.scale, sinks=z.cuda())
+    assert fa.check_device_error() == 0
+    rq, rk, rv, rz = oracle.attn_bwd_sinks(inp.q, inp.k, inp.v, do, z.double().numpy(), True,
+                                           0, inp.scale)
+    check("dQ", dq, rq, "sinks")
+    check("dK", dk, rk, "sinks")
+    check("dV", dv, rv, "sinks")
+    got = dz.double().cpu().numpy()
+    assert got[0] == 0.0
+    assert np.abs(got - rz).max() <= TOL_MAX_REL * np.abs(rz).max() + TOL_MAX_ABS
