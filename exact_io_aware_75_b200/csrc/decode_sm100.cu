@@ -86,7 +86,7 @@ struct UnitWalker {
 
 struct DecShared {
     uint64_t full[8], empty[8];
-    float scl[8][16];   // FP8: per stage, k scales then v scales of the head group (x 2^60)
+    float scl[8][16];   // FP8: per stage, k scales then v scales of the head group
     int abort;
 };
 
@@ -105,39 +105,40 @@ __device__ __forceinline__ void unpack8(uint4 a, float *f) {
     f[6] = __uint_as_float(a.w << 16); f[7] = __uint_as_float(a.w & 0xffff0000u);
 }
 
-// FP8 E4M3 codes to fp32 by bit placement, 2^-120 times the true value:
-// a code's 7 magnitude bits (exponent, mantissa) moved to bits 20-26 of an
-// fp32 word with its sign at bit 31 read as an fp32 exponent biased by 127
-// instead of 7, which scales every value -- subnormal codes included, as
-// fp32 subnormals -- by exactly 2^-120.  The caller folds 2^120 back into
-// its scales.  Eleven integer operations for four codes; the hardware
-// e4m3x2 -> f16x2 -> f32 conversions would take six quarter-rate ones.
-// (A NaN code becomes a finite value: codes in the used slots are finite.)
-constexpr float kE4m3Half = 1.152921504606847e18f;     // 2^60
-
-__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, uint64_t &p01, uint64_t &p23) {
-    // odd codes 1, 3: magnitudes >> 4 land at bits 4-10 / 20-26, signs stay
-    const uint32_t h = ((w & 0x7F007F00u) >> 4) | (w & 0x80008000u);
-    // even codes 0, 2: magnitudes << 4, signs << 8
-    const uint32_t g = ((w & 0x007F007Fu) << 4) | ((w << 8) & 0x80008000u);
-    p01 = f2pack(__uint_as_float(g << 16), __uint_as_float(h << 16));
-    p23 = f2pack(__uint_as_float(g & 0xFFFF0000u), __uint_as_float(h & 0xFFFF0000u));
+// Two FP8 E4M3 codes (bits 0-7: the lower index) to a packed fp32 pair, by
+// way of the hardware e4m3x2 -> f16x2 conversion and two f16 -> f32
+// conversions (both exact: every E4M3 value, subnormals included, is an f16
+// normal).  Measured faster here than building the fp32 words with integer
+// bit placement, which loads the integer pipe the dot products also use.
+__device__ __forceinline__ uint64_t e4m3x2_to_f2(uint32_t two) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h2) : "r"(two));
+    float lo, hi;
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}" : "=f"(lo), "=f"(hi) : "r"(h2));
+    return f2pack(lo, hi);
 }
 
-// N FP8 codes (N = 8 or 16, loaded as one 8- or 16-byte word) to N/2 pairs,
-// each value 2^-120 times its true value.
+// N FP8 codes (N = 8 or 16, loaded as one 8- or 16-byte word) to N/2 pairs.
 template <int N>
 __device__ __forceinline__ void unpack_e4m3(const uint8_t *src, uint64_t *f) {
     if constexpr (N == 16) {
         const uint4 a = *reinterpret_cast<const uint4 *>(src);
-        e4m3x4_to_f32(a.x, f[0], f[1]);
-        e4m3x4_to_f32(a.y, f[2], f[3]);
-        e4m3x4_to_f32(a.z, f[4], f[5]);
-        e4m3x4_to_f32(a.w, f[6], f[7]);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = e4m3x2_to_f2(w[i] & 0xffffu);
+            f[2 * i + 1] = e4m3x2_to_f2(w[i] >> 16);
+        }
     } else {
         const uint2 a = *reinterpret_cast<const uint2 *>(src);
-        e4m3x4_to_f32(a.x, f[0], f[1]);
-        e4m3x4_to_f32(a.y, f[2], f[3]);
+        const uint32_t w[2] = {a.x, a.y};
+        #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            f[2 * i] = e4m3x2_to_f2(w[i] & 0xffffu);
+            f[2 * i + 1] = e4m3x2_to_f2(w[i] >> 16);
+        }
     }
 }
 
@@ -207,8 +208,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (FP8 && warp == kDecWarpScales) {
             // ------------------------------------------------ FP8 scales
             // The same page sequence as the producer: each stage gets its
-            // page's k and v scales (lane l: KV head hg*HG + l), pre-multiplied
-            // by 2^60, then one arrival on the stage's full barrier.  Global
+            // page's k and v scales (lane l: KV head hg*HG + l), then one
+            // arrival on the stage's full barrier.  Global
             // loads stall only this warp.
             UnitWalker walk;
             uint32_t it = 0;
@@ -223,8 +224,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     if (page < 0 || page >= p.num_pages) page = 0;
                     if (lane < p.HG) {
                         const size_t i = (size_t)page * p.Hkv + hg * p.HG + lane;
-                        sh.scl[st][lane] = __ldg(p.k_scale + i) * kE4m3Half;
-                        sh.scl[st][8 + lane] = __ldg(p.v_scale + i) * kE4m3Half;
+                        sh.scl[st][lane] = __ldg(p.k_scale + i);
+                        sh.scl[st][8 + lane] = __ldg(p.v_scale + i);
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sh.full[st]);
@@ -296,11 +297,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             }
             #pragma unroll
             for (int i = 0; i < DPL / 2; ++i) q2[qh][i] = f2mul(q2[qh][i], sc2);
-            if constexpr (FP8) {   // half of the 2^120 the codes lack
-                const uint64_t h2 = f2pack(kE4m3Half, kE4m3Half);
-                #pragma unroll
-                for (int i = 0; i < DPL / 2; ++i) q2[qh][i] = f2mul(q2[qh][i], h2);
-            }
         }
         uint64_t o2[QPW][DPL / 2];
         float m_ref[QPW], l_acc[QPW];
@@ -470,8 +466,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const size_t row0 = ((size_t)seq * p.max_chunks + chunk) * p.Hq + h0;
             #pragma unroll
             for (int qh = 0; qh < QPW; ++qh) {
-                // FP8: P V carries 2^-120 (codes) x 2^60 (scale): restore 2^60
-                const float inv = l_acc[qh] > 0.f ? (FP8 ? kE4m3Half : 1.f) / l_acc[qh] : 0.f;
+                const float inv = l_acc[qh] > 0.f ? 1.f / l_acc[qh] : 0.f;
                 float *dst = p.part_o + (row0 + qh) * D + (FP8 ? DPL * ds : 8 * ds);
                 #pragma unroll
                 for (int b = 0; b < DPL / 8; ++b) {
