@@ -55,6 +55,11 @@ def lib():
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _f64p,
             ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
         L.oracle_attn_varlen_rows_sinks.restype = ctypes.c_int
+        L.oracle_attn_varlen_rows_doc.argtypes = [
+            _u16p, _u16p, _u16p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _i32p,
+            ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
+        L.oracle_attn_varlen_rows_doc.restype = ctypes.c_int
         L.oracle_decode_paged_sinks.argtypes = [
             _u16p, _u16p, _u16p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_int64, ctypes.c_double, _f64p, _f64p, _f64p]
@@ -401,3 +406,30 @@ def attn_bwd_sinks(q, k, v, dout, sinks, causal=False, window=0, scale=None):
         db.reshape(B * N, Hq, d), cu, B, Hq, Hkv, d, int(causal), int(window), float(scale),
         sk, dq, dk, dv, ds), "attn_bwd_sinks")
     return (dq.reshape(B, N, Hq, d), dk.reshape(B, N, Hkv, d), dv.reshape(B, N, Hkv, d), ds)
+
+
+def attn_doc(q, k, v, doc_ids, causal=False, window=0, scale=None, rows=None):
+    """Dense batch with a document mask: doc_ids [B,N] int32; key j is visible
+    from query i only if doc_ids[b,i] == doc_ids[b,j].  -> O [B,N,Hq,d], LSE
+    [B,Hq,N]; with ``rows`` (list of (b, i)) only those: O [R,Hq,d], LSE [R,Hq]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    doc = _i32(doc_ids).reshape(B * N)
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        nrows, rp = B * N, None
+    else:
+        r = np.ascontiguousarray(np.asarray([int(b) * N + int(i) for b, i in rows], dtype=np.int64))
+        nrows, rp = r.size, r.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((nrows, Hq, d), np.float64)
+    lse = np.empty((nrows, Hq), np.float64)
+    _check(lib().oracle_attn_varlen_rows_doc(qb.reshape(B * N, Hq, d), kb.reshape(B * N, Hkv, d),
+                                             vb.reshape(B * N, Hkv, d), cu, B, Hq, Hkv, d,
+                                             int(causal), int(window), float(scale), doc, rp,
+                                             nrows, o, lse), "attn_doc")
+    if rows is not None:
+        return o, lse
+    return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(B, N, Hq).transpose(0, 2, 1))

@@ -153,8 +153,8 @@ static void attend_row(const double *q, int d, int64_t nkeys,
 static int attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                   const int32_t *cu_seqlens, int num_seqs,
                                   int Hq, int Hkv, int d, int causal, int window,
-                                  double scale, const double *sinks, const int64_t *rows,
-                                  int64_t nrows, double *o, double *lse)
+                                  double scale, const double *sinks, const int32_t *doc,
+                                  const int64_t *rows, int64_t nrows, double *o, double *lse)
 {
     if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
     const int group = Hq / Hkv;
@@ -199,7 +199,8 @@ static int attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const ui
                 for (int64_t j = 0; j < L; ++j) {
                     kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
                     vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
-                    vis[j] = (unsigned char)allowed(i, j, causal, window);
+                    vis[j] = (unsigned char)(allowed(i, j, causal, window) &&
+                                             (!doc || doc[start + i] == doc[start + j]));
                 }
                 attend_row_sink(qd, d, L, kp, vp, vis, scale, sinks ? sinks[h] : -INFINITY, s,
                                 o + (r * Hq + h) * (int64_t)d, lse + r * Hq + h, NULL);
@@ -217,7 +218,7 @@ int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t
                             double *o, double *lse)
 {
     return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
-                                  scale, NULL, rows, nrows, o, lse);
+                                  scale, NULL, NULL, rows, nrows, o, lse);
 }
 
 /*
@@ -234,7 +235,26 @@ int oracle_attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const ui
 {
     if (!sinks) return -1;
     return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
-                                  scale, sinks, rows, nrows, o, lse);
+                                  scale, sinks, NULL, rows, nrows, o, lse);
+}
+
+/*
+ * Packed sequences with a document mask in any form ("FlexAttention":
+ * document masks among the attention variants, Ales Analytics kernels page):
+ * doc[total] holds a document id per token, and key j is visible from query
+ * i only if both carry the same id (on top of the causal / window rule), so
+ * a document's tokens need not be contiguous.  rows as for
+ * oracle_attn_varlen_rows.
+ */
+int oracle_attn_varlen_rows_doc(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const int32_t *cu_seqlens, int num_seqs,
+                                int Hq, int Hkv, int d, int causal, int window,
+                                double scale, const int32_t *doc, const int64_t *rows,
+                                int64_t nrows, double *o, double *lse)
+{
+    if (!doc) return -1;
+    return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
+                                  scale, NULL, doc, rows, nrows, o, lse);
 }
 
 /* Dense batch: q [B,N,Hq,d], k/v [B,N,Hkv,d]; o [B,N,Hq,d]; lse [B,Hq,N]. */
