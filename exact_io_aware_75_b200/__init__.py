@@ -37,6 +37,7 @@ FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa_fwd_paged",
+           "fa_fwd_doc",
            "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen", "fa_bwd_sinks",
            "fa_bwd_varlen_sinks",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
@@ -68,6 +69,8 @@ def _load():
     lib.fa_fwd_varlen_sinks.restype = i
     lib.fa_decode_paged_sinks.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged_sinks.restype = i
+    lib.fa_fwd_doc.argtypes = [vp] * 6 + [i] * 7 + [f, i, vp]
+    lib.fa_fwd_doc.restype = i
     lib.fa_fwd_paged.argtypes = [vp] * 9 + [i] * 11 + [f, i, vp]
     lib.fa_fwd_paged.restype = i
     lib.fa_decode_paged_fp8.argtypes = [vp] * 10 + [i] * 7 + [f, vp, sz, vp]
@@ -142,9 +145,10 @@ def _need(t, dtype, ndim, name):
 
 
 def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
-        out=None, lse=None, return_lse=True, stream=None, sinks=None):
+        out=None, lse=None, return_lse=True, stream=None, sinks=None, doc_ids=None):
     """Dense prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 -> (O [B,N,Hq,d], LSE [B,Hq,N]).
-    ``sinks`` (fp32 [Hq], device) selects fa_fwd_sinks."""
+    ``sinks`` (fp32 [Hq], device) selects fa_fwd_sinks; ``doc_ids`` (int32 [B,N],
+    device) selects fa_fwd_doc."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, 4, n)
     B, N, Hq, d = q.shape
@@ -158,6 +162,16 @@ def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    if doc_ids is not None:
+        if sinks is not None:
+            raise FAError(FA_ERR_UNSUPPORTED, "sinks with doc_ids")
+        _need(doc_ids, torch.int32, 2, "doc_ids")
+        if tuple(doc_ids.shape) != (B, N):
+            raise FAError(FA_ERR_INVALID_ARG, "doc_ids shape")
+        _check(_lib.fa_fwd_doc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(doc_ids),
+                               B, Hq, Hkv, N, d, int(causal), int(window), float(scale), od,
+                               _stream(stream)), "fa_fwd_doc")
+        return out, lse
     if sinks is not None:
         _need(sinks, torch.float32, 1, "sinks")
         _check(_lib.fa_fwd_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(sinks),

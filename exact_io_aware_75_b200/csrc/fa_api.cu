@@ -127,7 +127,7 @@ namespace {
 
 int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
               const float *sinks, int B, int Hq, int Hkv, int N, int d, int causal, int window,
-              float scale, int o_dtype, void *stream) {
+              float scale, int o_dtype, void *stream, const int *doc = nullptr) {
     if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
     if (rc) return rc;
@@ -150,6 +150,7 @@ int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
     a.scale = scale;
     a.o_fp32 = o_dtype == FA_OUT_FP32;
     a.sinks = sinks;
+    a.doc = doc;
     return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -201,6 +202,15 @@ int fa_fwd_sinks(const void *q, const void *k, const void *v, void *o, float *ls
     if (reinterpret_cast<uintptr_t>(sinks) & 3) return FA_ERR_ALIGNMENT;
     return fwd_dense(q, k, v, o, lse, sinks, B, Hq, Hkv, N, d, causal, window, scale,
                      o_dtype, stream);
+}
+
+int fa_fwd_doc(const void *q, const void *k, const void *v, void *o, float *lse,
+               const int *doc_ids, int B, int Hq, int Hkv, int N, int d, int causal,
+               int window, float scale, int o_dtype, void *stream) {
+    if (!doc_ids) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(doc_ids) & 3) return FA_ERR_ALIGNMENT;
+    return fwd_dense(q, k, v, o, lse, nullptr, B, Hq, Hkv, N, d, causal, window, scale,
+                     o_dtype, stream, doc_ids);
 }
 
 int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -26,6 +26,8 @@ struct PrefillArgs {
     int paged;
     const int *block_table, *seq_lens_k;
     int max_pages, num_pages;
+    // document mask: one id per token; nullptr = none
+    const int *doc;
 };
 
 int launch_prefill(const PrefillArgs &a, cudaStream_t stream);

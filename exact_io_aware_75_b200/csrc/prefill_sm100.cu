@@ -30,6 +30,7 @@
 //     and O and l stay consistent because both use the same reference max.
 //   * The epilogue divides O by l once ("FlashAttention-2": delayed
 //     normalisation) and writes O and LSE = ln2 * (m + log2 l).
+#include <climits>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -67,12 +68,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kPageRows = 16;                 // tokens per cache page (paged mode)
 constexpr int kPagesPerTile = 128 / kPageRows;
 
-template <int D>
+template <int D, bool DOC = false>
 struct Cfg {
     static constexpr int kBoxBytes = kBlockM * 64 * 2;             // 128 rows x 64 bf16
     static constexpr int kTileBytes = kBlockM * D * 2;             // Q tile or K/V tile
-    static constexpr int kStages = (D == 128) ? 5 : 6;             // K/V ring slots
-    static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + 1024;
+    // K/V ring slots (one fewer with a document mask, for its key-id buffers)
+    static constexpr int kStages = (D == 128) ? (DOC ? 4 : 5) : 6;
+    static constexpr int kDocBytes = DOC ? 8 * 2 * 128 * 4 : 0;   // [warp][parity][key]
+    static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + kDocBytes + 1024;
     static constexpr uint32_t kColO = 256;                         // O_t at 256 + t*D
 };
 
@@ -95,6 +98,9 @@ struct Params {
     const int *block_table, *seq_lens_k;
     const uint16_t *v_cache;
     int max_pages, num_pages;
+    // Document mask: one id per token (packed order); key j is visible from
+    // query i only if both ids are equal.
+    const int *doc;
 };
 
 struct Unit {
@@ -179,10 +185,10 @@ struct Shared {
 
 // ------------------------------------------------------------- TMA producer
 // Dense and packed batches: one thread issues every copy.
-template <int D>
+template <int D, bool DOC>
 __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                          const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
-    using C = Cfg<D>;
+    using C = Cfg<D, DOC>;
     volatile int *abort = &sh.abort;
     uint32_t q_uses[2] = {0, 0};
     uint32_t kv_it = 0;
@@ -333,9 +339,9 @@ out:
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool DOC>
 __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
-    using C = Cfg<D>;
+    using C = Cfg<D, DOC>;
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
     const uint32_t idS = idesc_bf16_f32(kBlockM, kBlockN, false);
@@ -486,9 +492,9 @@ __device__ __forceinline__ void exp_half(const float (&v)[kHalf], float sl2, flo
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D, bool PAGED>
-__device__ void softmax_wg(const Params &p, Shared &sh) {
-    using C = Cfg<D>;
+template <int D, bool PAGED, bool DOC>
+__device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
+    using C = Cfg<D, DOC>;
     volatile int *abort = &sh.abort;
     const int warp = warp_id(), lane = lane_id();
     const int t = warp >> 2;                 // tile of this warpgroup
@@ -508,9 +514,33 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
         if (lo >= hi) continue;
         const int row = w.q0 + t * kBlockM + r;    // row index within the sequence
         const int rmin = w.q0 + t * kBlockM, rmax = rmin + kBlockM - 1;
+        // Document mask: this row's id, and the key ids of the next block
+        // (lane l holds keys 4l .. 4l+3), loaded one block ahead; ids past the
+        // sequence never match (those keys are masked anyway).
+        int mydoc = 0, nd[4] = {0, 0, 0, 0};
+        auto load_key_docs = [&](int jb) {
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k = jb * kBlockN + 4 * lane + e;
+                nd[e] = (jb < hi && k < w.L) ? __ldg(p.doc + w.tok0 + k) : INT_MIN;
+            }
+        };
+        if constexpr (DOC) {
+            mydoc = (row < w.L) ? __ldg(p.doc + w.tok0 + row) : INT_MIN + 1;
+            load_key_docs(lo);
+        }
         float m_ref = -INFINITY, l = 0.f;
         for (int j = lo; j < hi; ++j) {
             if (!mbar_wait_warp(&sh.s_full[t], s_cnt & 1, abort)) return;
+            // the block's key ids, staged per warp (no cross-warp barrier)
+            const int *kd = nullptr;
+            if constexpr (DOC) {
+                int *buf = kdoc + (warp * 2 + (s_cnt & 1)) * kBlockN;
+                *reinterpret_cast<int4 *>(buf + 4 * lane) = make_int4(nd[0], nd[1], nd[2], nd[3]);
+                __syncwarp();
+                kd = buf;
+                load_key_docs(j + 1);
+            }
             ++s_cnt;
             tc_fence_after();
             const bool first = (j == lo);
@@ -542,10 +572,10 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
             uint32_t rawB[kHalf];
             tmem_ld32(tS + 64, rawB);
             tmem_ld32(tS + 96, rawB + 32);
-            if (edge) {
+            if (DOC || edge) {
                 #pragma unroll
                 for (int c = 0; c < kHalf; ++c)
-                    if (c >= c_hi || c < c_lo) sA[c] = -INFINITY;
+                    if (c >= c_hi || c < c_lo || (DOC && kd[c] != mydoc)) sA[c] = -INFINITY;
             }
             const float mA = row_max64(sA);
             // With the reference max unchanged (the common case under the
@@ -558,10 +588,11 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
             tmem_wait_ld();
             #pragma unroll
             for (int c = 0; c < kHalf; ++c) sB[c] = __uint_as_float(rawB[c]);
-            if (edge) {
+            if (DOC || edge) {
                 #pragma unroll
                 for (int c = 0; c < kHalf; ++c)
-                    if (c + kHalf >= c_hi || c + kHalf < c_lo) sB[c] = -INFINITY;
+                    if (c + kHalf >= c_hi || c + kHalf < c_lo || (DOC && kd[c + kHalf] != mydoc))
+                        sB[c] = -INFINITY;
             }
             const float m_blk = fmaxf(mA, row_max64(sB)) * sl2;
             bool redo = first;
@@ -683,11 +714,11 @@ __device__ void softmax_wg(const Params &p, Shared &sh) {
     }
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool DOC>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
-    using C = Cfg<D>;
+    using C = Cfg<D, DOC>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Shared sh;
     const uint32_t base = smem_u32(smem_raw);
@@ -726,16 +757,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (warp < kSoftmaxWarps) {
         regs_increase<kRegsSoftmax>();
-        softmax_wg<D, PAGED>(p, sh);
+        softmax_wg<D, PAGED, DOC>(p, sh, reinterpret_cast<int *>(sKV + C::kStages * C::kTileBytes));
     } else {
         regs_decrease<kRegsControl>();
         if (warp == kWarpTma) {
             if constexpr (PAGED)
                 producer_paged<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
             else if (lane_id() == 0)
-                producer<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+                producer<D, DOC>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
         } else if (warp == kWarpMma) {
-            if (lane_id() == 0) mma_issuer<D, PAGED>(p, sh, sQ, sKV);
+            if (lane_id() == 0) mma_issuer<D, PAGED, DOC>(p, sh, sQ, sKV);
         }
     }
     __syncwarp();
@@ -751,10 +782,26 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 // (Q tiles, K/V ring, 1 KiB alignment slack) within the 227 KiB opt-in limit.
 static_assert(Cfg<128>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 static_assert(Cfg<64>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
+static_assert(Cfg<128, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
+static_assert(Cfg<64, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
+
+template <int D, bool PAGED, bool DOC>
+int launch_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                  const Params &p, long long units, cudaStream_t stream) {
+    using C = Cfg<D, DOC>;
+    // Setting the attribute is idempotent and cheap; do it on every call so
+    // that any device the caller switches to is covered.
+    if (cudaFuncSetAttribute(prefill_kernel<D, PAGED, DOC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+        return -5;
+    const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
+    prefill_kernel<D, PAGED, DOC><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
 
 template <int D>
 int launch_d(const PrefillArgs &a, cudaStream_t stream) {
-    using C = Cfg<D>;
     alignas(64) CUtensorMap tq, tk, tv;
     const uint64_t T = (uint64_t)a.total_tokens;
     // K/V: the packed tokens (dense, varlen), or the cache's num_pages * 16
@@ -785,6 +832,7 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.o_fp32 = a.o_fp32;
     p.sinks = a.sinks;
     p.paged = a.paged;
+    p.doc = a.doc;
     p.block_table = a.block_table;
     p.seq_lens_k = a.seq_lens_k;
     p.v_cache = static_cast<const uint16_t *>(a.v);
@@ -795,15 +843,9 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     if (units <= 0) return 0;
     if (units > (1ll << 30)) return -2;
     p.num_units = (int)units;
-    // Setting the attribute is idempotent and cheap; do it on every call so
-    // that any device the caller switches to is covered.
-    auto kernel = a.paged ? prefill_kernel<D, true> : prefill_kernel<D, false>;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-        return -5;
-    const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
-    kernel<<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : -5;
+    if (a.paged) return launch_kernel<D, true, false>(tq, tk, tv, p, units, stream);
+    if (a.doc) return launch_kernel<D, false, true>(tq, tk, tv, p, units, stream);
+    return launch_kernel<D, false, false>(tq, tk, tv, p, units, stream);
 }
 
 }  // namespace prefill_impl

@@ -135,6 +135,21 @@ int fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache,
 size_t fa_bwd_workspace_bytes(int total_tokens, int Hq, int d);
 
 /*
+ * fa_fwd with a document mask in any form ("FlexAttention" on the Ales
+ * Analytics kernels page: document masks among the attention variants).
+ *   doc_ids [B, N] int32, device: a document id per token; key j is visible
+ *           from query i only if doc_ids[b][i] == doc_ids[b][j], on top of the
+ *           causal / window rule.  A document's tokens need not be contiguous
+ *           (for contiguous documents fa_fwd_varlen does less work: here every
+ *           key block the causal / window rule admits is computed).
+ * Other arguments, layouts and errors as for fa_fwd; doc_ids non-NULL and
+ * 4-byte aligned.
+ */
+int fa_fwd_doc(const void *q, const void *k, const void *v, void *o, float *lse,
+               const int *doc_ids, int B, int Hq, int Hkv, int N, int d, int causal,
+               int window, float scale, int o_dtype, void *stream);
+
+/*
  * fa_fwd / fa_fwd_varlen with a learned attention sink per query head
  * ("Sliding windows and local:global layers": gpt-oss's learned sink per
  * head).  sinks [Hq] fp32, device, in units of scaled scores: z_h joins every

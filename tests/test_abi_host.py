@@ -219,6 +219,14 @@ def test_fwd_paged_empty_is_noop(fa):
     assert paged_fwd(fa, Tq=0, q=0) == 0
 
 
+def test_fwd_doc_rejects(fa):
+    lib = fa.library()
+    assert lib.fa_fwd_doc(P, P, P, P, 0, None, 1, 2, 2, 128, 64, 1, 0, 0.1, 0, None) == -1
+    assert lib.fa_fwd_doc(P, P, P, P, 0, P + 2, 1, 2, 2, 128, 64, 1, 0, 0.1, 0, None) == -3
+    assert lib.fa_fwd_doc(P, P, P, P, 0, P, 1, 3, 2, 128, 64, 1, 0, 0.1, 0, None) == -1
+    assert lib.fa_fwd_doc(P, P, P, P, 0, P, 0, 2, 2, 128, 64, 1, 0, 0.1, 0, None) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """Importing the binding with the shared library absent raises, rather
     than falling back to anything else."""
