@@ -48,7 +48,7 @@ namespace fa {
 
 namespace bwd_impl {
 
-constexpr int kD = 128;
+constexpr int kD = 128;          // tile width in d; a head dim of 64 is zero-padded to it
 constexpr int kBlockK = 128;   // keys per unit
 constexpr int kBlockQ = 64;    // queries per tile
 constexpr int kThreads = 512;
@@ -313,6 +313,7 @@ out:
 }
 
 // ---------------------------------------------------- softmax-gradient warps
+template <int DH>
 __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const int warp = warp_id(), lane = lane_id();
@@ -410,13 +411,13 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
         const uint32_t tAcc = sh.tmem_base + lanes + (wg ? kColDK : kColDV);
         const float mul = wg ? p.scale : 1.f;
         uint16_t *dst = static_cast<uint16_t *>(wg ? p.dk : p.dv) +
-                        ((size_t)(w.tok0 + kj) * p.Hkv + w.kvh) * kD;
+                        ((size_t)(w.tok0 + kj) * p.Hkv + w.kvh) * DH;
         #pragma unroll
         for (int c = 0; c < kD; c += 32) {
             uint32_t v[32];
             tmem_ld32(tAcc + c, v);
             tmem_wait_ld();
-            if (key_ok) {
+            if (key_ok && c < DH) {   // columns past a 64-wide head are padding
                 uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
                 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -442,6 +443,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
 // rows; two staging buffers alternate so the next rows are written while the
 // previous reduce still reads.  Rows past the sequence add exact zeros (their
 // P, hence dS, is 0).
+template <int DH>
 __device__ void dq_drain(const CUtensorMap *tmDQ, const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const int warp = warp_id(), lane = lane_id();
@@ -473,9 +475,11 @@ __device__ void dq_drain(const CUtensorMap *tmDQ, const Params &p, Shared &sh, u
                 float *buf = stage + (hs & 1) * (kDQHalf * kD);
                 if (leader) bulk_wait_group_read<1>();   // the reduce that used buf is done reading
                 named_bar_sync(kBarDrain, 128);
-                #pragma unroll
-                for (int i = 0; i < kDQHalf; ++i)
-                    buf[i * kD + c] = __uint_as_float(v[half * kDQHalf + i]) * p.scale;
+                if (c < DH) {           // rows of the head dim (the reduce box is DH wide)
+                    #pragma unroll
+                    for (int i = 0; i < kDQHalf; ++i)
+                        buf[i * DH + c] = __uint_as_float(v[half * kDQHalf + i]) * p.scale;
+                }
                 fence_proxy_async_smem();
                 named_bar_sync(kBarDrain, 128);
                 if (leader) {
@@ -489,6 +493,7 @@ out:
     if (leader) bulk_wait_group_all();
 }
 
+template <int DH>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -532,10 +537,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (warp < 8) {
         regs_increase<kRegsSoftmax>();
-        softmax_wg(p, sh, smem);
+        softmax_wg<DH>(p, sh, smem);
     } else if (warp < 12) {
         regs_decrease<kRegsDrain>();
-        dq_drain(&tmDQ, p, sh, smem);
+        dq_drain<DH>(&tmDQ, p, sh, smem);
     } else {
         regs_decrease<kRegsControl>();
         if (warp == kWarpTma) {
@@ -554,7 +559,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 }
 
 // D = rowsum(O * dO) for every (token, query head), in the LSE layout; zeroes
-// the dQ accumulator.  One warp per row of d = 128 elements.
+// the dQ accumulator.  One warp per row of DH = 64 or 128 elements.
+template <int DH>
 __global__ void __launch_bounds__(256)
 bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dout,
                 float *__restrict__ dd, float *__restrict__ dq_acc, int total, int Hq,
@@ -562,14 +568,22 @@ bwd_prep_kernel(const uint16_t *__restrict__ o, const uint16_t *__restrict__ dou
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (long long)total * Hq) return;
-    const uint2 a = reinterpret_cast<const uint2 *>(o + row * kD)[lane];
-    const uint2 b = reinterpret_cast<const uint2 *>(dout + row * kD)[lane];
     auto lo = [](uint32_t x) { return __uint_as_float(x << 16); };
     auto hi = [](uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); };
-    float acc = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+    float acc;
+    if constexpr (DH == 128) {
+        const uint2 a = reinterpret_cast<const uint2 *>(o + row * DH)[lane];
+        const uint2 b = reinterpret_cast<const uint2 *>(dout + row * DH)[lane];
+        acc = lo(a.x) * lo(b.x) + hi(a.x) * hi(b.x) + lo(a.y) * lo(b.y) + hi(a.y) * hi(b.y);
+        reinterpret_cast<float4 *>(dq_acc + row * DH)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+        const uint32_t a = reinterpret_cast<const uint32_t *>(o + row * DH)[lane];
+        const uint32_t b = reinterpret_cast<const uint32_t *>(dout + row * DH)[lane];
+        acc = lo(a) * lo(b) + hi(a) * hi(b);
+        reinterpret_cast<float2 *>(dq_acc + row * DH)[lane] = make_float2(0.f, 0.f);
+    }
     #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    reinterpret_cast<float4 *>(dq_acc + row * kD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (lane == 0) {
         const long long tok = row / Hq;
         const int h = (int)(row % Hq);
@@ -636,7 +650,7 @@ bwd_convert_kernel(const float *__restrict__ acc, uint16_t *__restrict__ dq, lon
 }  // namespace bwd_impl
 
 size_t bwd_workspace_bytes(long long total_tokens, int Hq, int d) {
-    if (total_tokens < 0 || Hq <= 0 || d != bwd_impl::kD) return 0;
+    if (total_tokens < 0 || Hq <= 0 || (d != 64 && d != 128)) return 0;
     const size_t acc = (size_t)total_tokens * Hq * d * sizeof(float);
     const size_t dd = (size_t)total_tokens * Hq * sizeof(float);
     return ((acc + 255) & ~(size_t)255) + ((dd + 255) & ~(size_t)255);
@@ -644,15 +658,17 @@ size_t bwd_workspace_bytes(long long total_tokens, int Hq, int d) {
 
 int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     using namespace bwd_impl;
-    if (a.d != kD) return -2;
+    if (a.d != 64 && a.d != 128) return -2;
+    const int dh = a.d;
     const long long total = a.total_tokens;
     if (total == 0 || a.num_seqs == 0) return 0;
-    const size_t acc_bytes = ((size_t)total * a.Hq * kD * sizeof(float) + 255) & ~(size_t)255;
+    const size_t acc_bytes = ((size_t)total * a.Hq * dh * sizeof(float) + 255) & ~(size_t)255;
     float *dq_acc = static_cast<float *>(a.workspace);
     float *dd = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) + acc_bytes);
 
     const long long rows = total * a.Hq;
-    bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+    auto prep = dh == 128 ? bwd_prep_kernel<128> : bwd_prep_kernel<64>;
+    prep<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
         static_cast<const uint16_t *>(a.o), static_cast<const uint16_t *>(a.dout), dd, dq_acc,
         (int)total, a.Hq, a.seqlen, a.cu_seqlens ? 0 : 1);
     if (cudaGetLastError() != cudaSuccess) return -5;
@@ -663,18 +679,22 @@ int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
         if (cudaGetLastError() != cudaSuccess) return -5;
     }
 
+    // Tensors are dh wide; tiles are kD = 128 wide, loaded as two 64-column
+    // boxes.  With dh = 64 the second box lies wholly past the tensor's inner
+    // extent, and TMA fills it with zeros: the padded columns add nothing to
+    // S or dP, and their dK, dV, dQ columns are never written.
     alignas(64) CUtensorMap tq, tk, tv, tdo, tdq;
     const uint64_t T = (uint64_t)total;
-    if (encode_tensor_map_3d(&tq, a.q, 2, kD, a.Hq, T, (uint64_t)kD * 2, (uint64_t)a.Hq * kD * 2,
+    if (encode_tensor_map_3d(&tq, a.q, 2, dh, a.Hq, T, (uint64_t)dh * 2, (uint64_t)a.Hq * dh * 2,
                              64, 1, kBlockQ, 128) ||
-        encode_tensor_map_3d(&tdo, a.dout, 2, kD, a.Hq, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hq * kD * 2, 64, 1, kBlockQ, 128) ||
-        encode_tensor_map_3d(&tk, a.k, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, 128) ||
-        encode_tensor_map_3d(&tv, a.v, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
-                             (uint64_t)a.Hkv * kD * 2, 64, 1, kBlockK, 128) ||
-        encode_tensor_map_3d(&tdq, dq_acc, 4, kD, a.Hq, T, (uint64_t)kD * 4,
-                             (uint64_t)a.Hq * kD * 4, kD, 1, kDQHalf, 0))
+        encode_tensor_map_3d(&tdo, a.dout, 2, dh, a.Hq, T, (uint64_t)dh * 2,
+                             (uint64_t)a.Hq * dh * 2, 64, 1, kBlockQ, 128) ||
+        encode_tensor_map_3d(&tk, a.k, 2, dh, a.Hkv, T, (uint64_t)dh * 2,
+                             (uint64_t)a.Hkv * dh * 2, 64, 1, kBlockK, 128) ||
+        encode_tensor_map_3d(&tv, a.v, 2, dh, a.Hkv, T, (uint64_t)dh * 2,
+                             (uint64_t)a.Hkv * dh * 2, 64, 1, kBlockK, 128) ||
+        encode_tensor_map_3d(&tdq, dq_acc, 4, dh, a.Hq, T, (uint64_t)dh * 4,
+                             (uint64_t)a.Hq * dh * 4, dh, 1, kDQHalf, 0))
         return -5;
     Params p;
     p.lse = a.lse;
@@ -698,14 +718,15 @@ int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     if (units > (1ll << 30)) return -2;
     p.num_units = (int)units;
     if (units > 0) {
-        if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        auto kernel = dh == 128 ? bwd_kernel<128> : bwd_kernel<64>;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kSmemBytes) != cudaSuccess)
             return -5;
         const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
-        bwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
+        kernel<<<grid, kThreads, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, p);
         if (cudaGetLastError() != cudaSuccess) return -5;
     }
-    const long long n8 = total * a.Hq * kD / 8;
+    const long long n8 = total * a.Hq * dh / 8;
     bwd_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<uint16_t *>(a.dq), n8);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;

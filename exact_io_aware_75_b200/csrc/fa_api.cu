@@ -292,7 +292,6 @@ int bwd_common(const void *q, const void *k, const void *v, const void *o, const
                size_t workspace_bytes) {
     int rc = check_common(Hq, Hkv, d, causal, window, scale, FA_OUT_BF16);
     if (rc) return rc;
-    if (d != 128) return FA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (total > INT32_MAX / 2 || total * Hq > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||

@@ -130,7 +130,8 @@ int fa_fwd_paged(const void *q, const void *k_cache, const void *v_cache,
 /*
  * Bytes of workspace fa_bwd / fa_bwd_varlen need for total_tokens tokens
  * (B * N for a dense batch): an fp32 dQ accumulator [total, Hq, d] and the
- * row terms D_i = dO_i . O_i.  0 for an unsupported combination (d != 128).
+ * row terms D_i = dO_i . O_i.  0 for an unsupported combination (d not 64
+ * or 128).
  */
 size_t fa_bwd_workspace_bytes(int total_tokens, int Hq, int d);
 
@@ -184,8 +185,9 @@ int fa_fwd_varlen_sinks(const void *q, const void *k, const void *v, void *o, fl
  *   workspace  device scratch of at least fa_bwd_workspace_bytes(B * N, Hq, d)
  *              bytes, 256-byte aligned; contents on entry do not matter; not
  *              to be shared by calls that may overlap on the GPU.
- *   causal, window, scale as for fa_fwd.  d must be 128 (others return
- *   FA_ERR_UNSUPPORTED).  N == 0 or B == 0 is a no-op returning FA_OK.
+ *   causal, window, scale as for fa_fwd.  d = 64 or 128 (a head dim of 64 is
+ *   computed on 128-wide tiles with zero padding, at the cost of 128).
+ *   N == 0 or B == 0 is a no-op returning FA_OK.
  * dQ is accumulated in fp32 with atomic adds, so its last bits may differ
  * from run to run; dK and dV are deterministic.
  */

@@ -123,7 +123,7 @@ def bwd(fa, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(Hq=3), -1), (dict(scale=-1.0), -1), (dict(causal=3), -1), (dict(d=64), -2),
+    (dict(Hq=3), -1), (dict(scale=-1.0), -1), (dict(causal=3), -1), (dict(d=96), -2),
     (dict(d=80), -2), (dict(window=8, causal=0), -2), (dict(do=0), -1), (dict(lse=0), -1),
     (dict(dq=0), -1), (dict(dv=P + 4), -3), (dict(lse=P + 1), -3), (dict(ws=0), -4),
     (dict(wsb=1000), -4), (dict(ws=P + 16), -3), (dict(B=-2), -1)])
@@ -161,7 +161,8 @@ def test_bwd_workspace_formula(fa):
     r256 = lambda x: (x + 255) // 256 * 256
     T, Hq = 4096, 32
     assert fa.bwd_workspace_bytes(T, Hq, 128) == r256(T * Hq * 128 * 4) + r256(T * Hq * 4)
-    assert fa.bwd_workspace_bytes(T, Hq, 64) == 0
+    assert fa.bwd_workspace_bytes(T, Hq, 64) == r256(T * Hq * 64 * 4) + r256(T * Hq * 4)
+    assert fa.bwd_workspace_bytes(T, Hq, 96) == 0
 
 
 def test_sinks_entry_points_reject(fa):

@@ -169,3 +169,17 @@ def test_sinks_backward(fa):
     got = dz.double().cpu().numpy()
     assert got[0] == 0.0
     assert np.abs(got - rz).max() <= TOL_MAX_REL * np.abs(rz).max() + TOL_MAX_ABS
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,causal,window", [
+    (1, 4, 2, 300, True, 0), (2, 2, 2, 257, False, 0), (1, 4, 1, 700, True, 130)])
+def test_head_dim_64(fa, B, Hq, Hkv, N, causal, window):
+    """d = 64: computed on zero-padded 128-wide tiles."""
+    inp = workloads.dense(B, Hq, Hkv, N, 64, causal=causal, window=window, seed=N + 64)
+    do = workloads.grad_out((B, N, Hq, 64), seed=N + 64)
+    dq, dk, dv = run_dense(fa, inp, do)
+    rq, rk, rv = oracle.attn_bwd(inp.q, inp.k, inp.v, do, causal, window, inp.scale)
+    what = f"d=64 B={B} Hq={Hq} Hkv={Hkv} N={N} causal={causal} W={window}"
+    check("dQ", dq, rq, what)
+    check("dK", dk, rk, what)
+    check("dV", dv, rv, what)
