@@ -115,9 +115,12 @@ def prefill_flops(B, Hq, N, d, causal=True, window=0):
 
 
 def kernel_source_hash():
+    """sha256 (first 12 hex digits) over every CUDA source and header of the library."""
     h = hashlib.sha256()
-    for f in ("prefill_sm100.cu", "decode_sm100.cu", "sm100.cuh"):
-        h.update(open(os.path.join(ROOT, "exact_io_aware_75_b200", "csrc", f), "rb").read())
+    csrc = os.path.join(ROOT, "exact_io_aware_75_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:12]
 
 

@@ -36,6 +36,17 @@
  *   M = max_s lse_s, w_s = exp(lse_s - M), lse = M + log(sum_s w_s),
  *   O = sum_s w_s O_s / sum_s w_s.
  *
+ * Further functions, each with its reading stated where it is defined:
+ *   - oracle_attn_bwd_varlen (+ _sinks, _dq_rows): the gradients dQ, dK, dV
+ *     (and of the sink logits) by the chain rule through the definition;
+ *   - the learned sink logit per head (the _sinks variants): one more score
+ *     in the denominator with a zero value;
+ *   - oracle_decode_paged_fp8: the decode over an FP8 E4M3 cache with a scale
+ *     per (page, KV head);
+ *   - oracle_prefill_paged: a chunk of new queries over a paged cache, the
+ *     chunk holding each sequence's last positions;
+ *   - oracle_attn_varlen_rows_doc: a document mask by per-token ids.
+ *
  * Inputs are bf16 bit patterns (uint16); each is widened exactly to double.
  * All sums run in a fixed sequential order, so results do not depend on the
  * OpenMP thread count.  libm exp/log in double; build without -ffast-math.
