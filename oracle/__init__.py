@@ -24,6 +24,8 @@ _u16p = np.ctypeslib.ndpointer(dtype=np.uint16, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
 _i64p = np.ctypeslib.ndpointer(dtype=np.int64, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+_f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 
 
 def lib():
@@ -66,8 +68,6 @@ def lib():
         L.oracle_decode_paged_sinks.restype = ctypes.c_int
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_value.restype = ctypes.c_double
-        _u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
-        _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
         L.oracle_decode_paged_fp8.argtypes = [
             _u16p, _u8p, _u8p, _f32p, _f32p, _i32p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_int64, ctypes.c_double, ctypes.c_void_p, _f64p, _f64p]
@@ -89,6 +89,17 @@ def lib():
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
         L.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
+        L.oracle_hadamard_rotate.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int,
+                                             ctypes.c_void_p, _f64p]
+        L.oracle_hadamard_rotate.restype = ctypes.c_int
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_quantize_e4m3_blocks.argtypes = [_f64p] + [ctypes.c_int] * 5 + [_u8p, _f32p]
+        L.oracle_quantize_e4m3_blocks.restype = ctypes.c_int
+        L.oracle_attn_fp8.argtypes = [_u8p, _f32p, ctypes.c_int, _u8p, _f32p, ctypes.c_int,
+                                      _u8p, _f32p] + [ctypes.c_int] * 7 + [
+            ctypes.c_double, _f64p, _f64p]
+        L.oracle_attn_fp8.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -433,3 +444,81 @@ def attn_doc(q, k, v, doc_ids, causal=False, window=0, scale=None, rows=None):
     if rows is not None:
         return o, lse
     return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(B, N, Hq).transpose(0, 2, 1))
+
+
+# ---------------------------------------------------------------- FP8 prefill
+# Incoherent processing ("FlashAttention-3", samanvya.dev "Attention Is the
+# Bottleneck"): Q and K rotated by diag(signs) H / sqrt(d) (H Sylvester
+# Hadamard), then E4M3 with a scale per (batch, head, 128-token block); V
+# unrotated with one scale per (batch, KV head).  oracle.c states the readings.
+FP8_BLOCK = 128
+
+
+def hadamard_rotate(x, signs=None) -> np.ndarray:
+    """x [..., d] bf16 -> fp64 x diag(signs) H / sqrt(d) (signs None: x widened)."""
+    xb = _bits(x)
+    d = xb.shape[-1]
+    rows = xb.size // d
+    y = np.empty(xb.shape, np.float64)
+    sp = None
+    if signs is not None:
+        sg = np.ascontiguousarray(np.asarray(signs, dtype=np.float64).reshape(d))
+        sp = sg.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().oracle_hadamard_rotate(xb, rows, d, sp, y), "hadamard_rotate")
+    return y
+
+
+def e4m3_encode(y: float) -> int:
+    """The E4M3 code nearest to y (ties to even, saturating at 448)."""
+    return int(lib().oracle_e4m3_encode(float(y)))
+
+
+def quantize_e4m3_blocks(x, block):
+    """x [B, N, H, d] fp64 -> (codes uint8 [B, N, H, d], scales fp32 [B, H, nblk])."""
+    xd = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    B, N, H, d = xd.shape
+    nblk = (N + block - 1) // block
+    codes = np.empty(xd.shape, np.uint8)
+    scales = np.empty((B, H, nblk), np.float32)
+    _check(lib().oracle_quantize_e4m3_blocks(xd, B, N, H, d, int(block), codes, scales),
+           "quantize_e4m3_blocks")
+    return codes, scales
+
+
+def fp8_prepare(q, k, v, signs=None):
+    """The quantised operands of the FP8 prefill: q, k, v [B, N, H, d] bf16 ->
+    dict(q8, q_scale [B,Hq,nblk], k8, k_scale [B,Hkv,nblk], v8, v_scale [B,Hkv])."""
+    q8, qs = quantize_e4m3_blocks(hadamard_rotate(q, signs), FP8_BLOCK)
+    k8, ks = quantize_e4m3_blocks(hadamard_rotate(k, signs), FP8_BLOCK)
+    vd = hadamard_rotate(v, None)
+    N = vd.shape[1]
+    v8, vs = quantize_e4m3_blocks(vd, max(N, 1))
+    return {"q8": q8, "q_scale": qs, "k8": k8, "k_scale": ks, "v8": v8,
+            "v_scale": np.ascontiguousarray(vs.reshape(vs.shape[0], vs.shape[1]))}
+
+
+def attn_fp8(q8, q_scale, k8, k_scale, v8, v_scale, causal=False, window=0, scale=None,
+             qblock=FP8_BLOCK, kblock=FP8_BLOCK):
+    """Attention over E4M3 codes [B, N, H, d] and their scales -> O [B,N,Hq,d], LSE [B,Hq,N]."""
+    q8, k8, v8 = _u8(q8), _u8(k8), _u8(v8)
+    B, N, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    qs = np.ascontiguousarray(np.asarray(q_scale, dtype=np.float32))
+    ks = np.ascontiguousarray(np.asarray(k_scale, dtype=np.float32))
+    vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float32))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((B, N, Hq, d), np.float64)
+    lse = np.empty((B, Hq, N), np.float64)
+    _check(lib().oracle_attn_fp8(q8, qs, int(qblock), k8, ks, int(kblock), v8, vs, B, N, Hq,
+                                 Hkv, d, int(causal), int(window), float(scale), o, lse),
+           "attn_fp8")
+    return o, lse
+
+
+def fp8_prefill(q, k, v, signs=None, causal=False, window=0, scale=None):
+    """The whole FP8 prefill: rotate, quantise, attend.  -> (O, LSE, prepared operands)."""
+    prep = fp8_prepare(q, k, v, signs)
+    o, lse = attn_fp8(prep["q8"], prep["q_scale"], prep["k8"], prep["k_scale"], prep["v8"],
+                      prep["v_scale"], causal, window, scale)
+    return o, lse, prep

@@ -45,7 +45,10 @@
  *     per (page, KV head);
  *   - oracle_prefill_paged: a chunk of new queries over a paged cache, the
  *     chunk holding each sequence's last positions;
- *   - oracle_attn_varlen_rows_doc: a document mask by per-token ids.
+ *   - oracle_attn_varlen_rows_doc: a document mask by per-token ids;
+ *   - oracle_hadamard_rotate, oracle_e4m3_encode, oracle_quantize_e4m3_blocks,
+ *     oracle_attn_fp8: the FP8 prefill with incoherent processing (rotation
+ *     of Q and K, block-scaled E4M3 codes, attention over the codes).
  *
  * Inputs are bf16 bit patterns (uint16); each is widened exactly to double.
  * All sums run in a fixed sequential order, so results do not depend on the
@@ -850,6 +853,192 @@ int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_cache, const uint1
             }
         }
         free(sb); free(qd); free(kp); free(vp); free(vis);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * FP8 prefill with incoherent processing ("FlashAttention-3" in the
+ * "FlashAttention: same math, different IO" part of samanvya.dev's post: Q
+ * and K are multiplied by a random orthogonal Hadamard matrix before E4M3
+ * quantisation, which spreads outlier channels over all dimensions; "Low
+ * precision" in the same post's introduction: FP8 GEMMs carry per-block
+ * scales).  Readings, where the pages leave the step open:
+ *   - the orthogonal matrix is M = D H / sqrt(d): D = diag(signs), a random
+ *     +-1 per channel drawn by the caller, H the Sylvester Hadamard matrix of
+ *     order d (a power of two), entry (k, c) = (-1)^popcount(k & c).  Both Q
+ *     and K are rotated by the same M, so (Q M)(K M)^T = Q K^T exactly;
+ *   - Q and K get one scale per (batch, head, block of 128 tokens), V (not
+ *     rotated) one per (batch, KV head): V's contraction runs over all keys,
+ *     so its scale has to factor out of the whole sum;
+ *   - scale = amax / 448 of the block (448 = largest finite E4M3), stored as
+ *     fp32 (1 when the block is all zero); code = the E4M3 value nearest to
+ *     x / scale, ties to the even code, saturated to +-448.
+ * The attention is then the plain definition applied to the dequantised
+ * values code * scale.
+ */
+
+/* Sylvester Hadamard entry of order 2^k: (-1)^popcount(k & c). */
+static int hadamard_sign(int k, int c)
+{
+    unsigned x = (unsigned)(k & c);
+    int par = 0;
+    while (x) { par ^= 1; x &= x - 1; }
+    return par ? -1 : 1;
+}
+
+/*
+ * y[r][c] = sum_k signs[k] * x[r][k] * H[k][c] / sqrt(d) for rows of d bf16
+ * values (signs NULL: y = x, no rotation).  d must be a power of two.
+ */
+int oracle_hadamard_rotate(const uint16_t *x, int64_t rows, int d, const double *signs,
+                           double *y)
+{
+    if (d <= 0 || (d & (d - 1)) || rows < 0) return -1;
+    const double inv = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = x + r * d;
+        double *yr = y + r * d;
+        if (!signs) {
+            for (int c = 0; c < d; ++c) yr[c] = widen(xr[c]);
+            continue;
+        }
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int k = 0; k < d; ++k)
+                acc += signs[k] * widen(xr[k]) * (double)hadamard_sign(k, c);
+            yr[c] = acc * inv;
+        }
+    }
+    return 0;
+}
+
+/*
+ * The E4M3 code nearest to y (ties to the even code), saturating at +-448.
+ * The grid: spacing 2^(e-3) on [2^e, 2^(e+1)) for e >= -6, and the
+ * subnormals m * 2^-9 below 2^-6.
+ */
+uint8_t oracle_e4m3_encode(double y)
+{
+    if (isnan(y)) return 0x7F;
+    const int sign = signbit(y) ? 1 : 0;
+    const double a = fabs(y);
+    if (a >= 448.0) return (uint8_t)((sign << 7) | 0x7E);
+    int e = -6;
+    if (a >= ldexp(1.0, -6)) {
+        frexp(a, &e);   /* a = f * 2^e, f in [0.5, 1) */
+        e -= 1;         /* a in [2^e, 2^(e+1)) */
+    }
+    const double r = rint(ldexp(a, 3 - e));   /* units of the spacing; ties to even */
+    int field, mant;
+    if (e == -6 && r < 8.0) {
+        field = 0;
+        mant = (int)r;
+    } else if (r >= 16.0) {
+        field = e + 1 + 7;
+        mant = 0;
+    } else {
+        field = e + 7;
+        mant = (int)r - 8;
+    }
+    if (field > 15 || (field == 15 && mant == 7)) return (uint8_t)((sign << 7) | 0x7E);
+    return (uint8_t)((sign << 7) | (field << 3) | mant);
+}
+
+/*
+ * Block-scaled E4M3 quantisation of x [B, N, H, d] (fp64): one scale per
+ * (b, h, block of `block` tokens), scales [B, H, ceil(N / block)] fp32.
+ */
+int oracle_quantize_e4m3_blocks(const double *x, int B, int N, int H, int d, int block,
+                                uint8_t *codes, float *scales)
+{
+    if (B < 0 || N < 0 || H <= 0 || d <= 0 || block <= 0) return -1;
+    const int nblk = (N + block - 1) / block;
+#pragma omp parallel for schedule(static)
+    for (int64_t task = 0; task < (int64_t)B * H * nblk; ++task) {
+        const int b = (int)(task / ((int64_t)H * nblk));
+        const int h = (int)((task / nblk) % H);
+        const int blk = (int)(task % nblk);
+        const int n0 = blk * block, n1 = (n0 + block < N) ? n0 + block : N;
+        double amax = 0.0;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                const double v = fabs(x[(((int64_t)b * N + n) * H + h) * d + c]);
+                if (v > amax) amax = v;
+            }
+        const float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+        scales[((int64_t)b * H + h) * nblk + blk] = sc;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                const int64_t i = (((int64_t)b * N + n) * H + h) * d + c;
+                codes[i] = oracle_e4m3_encode(x[i] / (double)sc);
+            }
+    }
+    return 0;
+}
+
+/*
+ * Attention over E4M3 codes: q8 [B, N, Hq, d] with q_scale [B, Hq, ceil(N /
+ * qblock)], k8 [B, N, Hkv, d] with k_scale [B, Hkv, ceil(N / kblock)], v8
+ * [B, N, Hkv, d] with v_scale [B, Hkv].  Each value is code * its scale;
+ * then the definition with causal / window masks as in oracle_attn.
+ *   o [B, N, Hq, d], lse [B, Hq, N] (fp64)
+ */
+int oracle_attn_fp8(const uint8_t *q8, const float *q_scale, int qblock,
+                    const uint8_t *k8, const float *k_scale, int kblock,
+                    const uint8_t *v8, const float *v_scale,
+                    int B, int N, int Hq, int Hkv, int d, int causal, int window,
+                    double scale, double *o, double *lse)
+{
+    if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv || qblock <= 0 ||
+        kblock <= 0)
+        return -1;
+    const int group = Hq / Hkv;
+    const int nbq = (N + qblock - 1) / qblock, nbk = (N + kblock - 1) / kblock;
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(N > 0 ? N : 1);
+        double *sb = (double *)malloc(sizeof(double) * n);
+        double *ksr = (double *)malloc(sizeof(double) * n);
+        double *vsr = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint8_t **kp = (const uint8_t **)malloc(sizeof(void *) * n);
+        const uint8_t **vp = (const uint8_t **)malloc(sizeof(void *) * n);
+        if (!sb || !ksr || !vsr || !qd || !orow || !kp || !vp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t task = 0; task < (int64_t)B * N * Hq; ++task) {
+                const int b = (int)(task / ((int64_t)N * Hq));
+                const int i = (int)((task / Hq) % N);
+                const int h = (int)(task % Hq), g = h / group;
+                const double qs = (double)q_scale[((int64_t)b * Hq + h) * nbq + i / qblock];
+                for (int c = 0; c < d; ++c)
+                    qd[c] = oracle_e4m3_value(q8[(((int64_t)b * N + i) * Hq + h) * d + c]) * qs;
+                /* the allowed keys are one contiguous range */
+                int j0 = 0, j1 = N;
+                if (causal) {
+                    j1 = i + 1;
+                    if (window > 0 && i - window + 1 > 0) j0 = i - window + 1;
+                }
+                int nk = 0;
+                for (int j = j0; j < j1; ++j, ++nk) {
+                    kp[nk] = k8 + (((int64_t)b * N + j) * Hkv + g) * d;
+                    vp[nk] = v8 + (((int64_t)b * N + j) * Hkv + g) * d;
+                    ksr[nk] = (double)k_scale[((int64_t)b * Hkv + g) * nbk + j / kblock];
+                    vsr[nk] = (double)v_scale[(int64_t)b * Hkv + g];
+                }
+                double l;
+                attend_row_fp8(qd, d, nk, kp, vp, ksr, vsr, scale, -INFINITY, sb, orow, &l);
+                for (int c = 0; c < d; ++c) o[task * d + c] = orow[c];
+                lse[((int64_t)b * Hq + h) * N + i] = l;
+            }
+        }
+        free(sb); free(ksr); free(vsr); free(qd); free(orow); free(kp); free(vp);
     }
     return bad ? -2 : 0;
 }
