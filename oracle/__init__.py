@@ -94,11 +94,13 @@ def lib():
         L.oracle_hadamard_rotate.restype = ctypes.c_int
         L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_block_scale.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_block_scale.restype = ctypes.c_float
         L.oracle_quantize_e4m3_blocks.argtypes = [_f64p] + [ctypes.c_int] * 5 + [_u8p, _f32p]
         L.oracle_quantize_e4m3_blocks.restype = ctypes.c_int
         L.oracle_attn_fp8.argtypes = [_u8p, _f32p, ctypes.c_int, _u8p, _f32p, ctypes.c_int,
                                       _u8p, _f32p] + [ctypes.c_int] * 7 + [
-            ctypes.c_double, _f64p, _f64p]
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
         L.oracle_attn_fp8.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -449,8 +451,9 @@ def attn_doc(q, k, v, doc_ids, causal=False, window=0, scale=None, rows=None):
 # ---------------------------------------------------------------- FP8 prefill
 # Incoherent processing ("FlashAttention-3", samanvya.dev "Attention Is the
 # Bottleneck"): Q and K rotated by diag(signs) H / sqrt(d) (H Sylvester
-# Hadamard), then E4M3 with a scale per (batch, head, 128-token block); V
-# unrotated with one scale per (batch, KV head).  oracle.c states the readings.
+# Hadamard), then E4M3 with a power-of-two scale per (batch, head, 128-token
+# block); V unrotated with one scale per (batch, KV head).  oracle.c states the
+# readings.
 FP8_BLOCK = 128
 
 
@@ -471,6 +474,12 @@ def hadamard_rotate(x, signs=None) -> np.ndarray:
 def e4m3_encode(y: float) -> int:
     """The E4M3 code nearest to y (ties to even, saturating at 448)."""
     return int(lib().oracle_e4m3_encode(float(y)))
+
+
+def e4m3_block_scale(amax: float) -> float:
+    """The scale of a block with largest magnitude amax: the smallest power of
+    two 2^k (k >= -126) with amax / 2^k <= 448; 1 for amax = 0."""
+    return float(lib().oracle_e4m3_block_scale(float(amax)))
 
 
 def quantize_e4m3_blocks(x, block):
@@ -498,8 +507,9 @@ def fp8_prepare(q, k, v, signs=None):
 
 
 def attn_fp8(q8, q_scale, k8, k_scale, v8, v_scale, causal=False, window=0, scale=None,
-             qblock=FP8_BLOCK, kblock=FP8_BLOCK):
-    """Attention over E4M3 codes [B, N, H, d] and their scales -> O [B,N,Hq,d], LSE [B,Hq,N]."""
+             qblock=FP8_BLOCK, kblock=FP8_BLOCK, rows=None):
+    """Attention over E4M3 codes [B, N, H, d] and their scales -> O [B,R,Hq,d], LSE [B,Hq,R]
+    for the query positions ``rows`` of every batch (default: all N)."""
     q8, k8, v8 = _u8(q8), _u8(k8), _u8(v8)
     B, N, Hq, d = q8.shape
     Hkv = k8.shape[2]
@@ -508,10 +518,14 @@ def attn_fp8(q8, q_scale, k8, k_scale, v8, v_scale, causal=False, window=0, scal
     vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float32))
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o = np.empty((B, N, Hq, d), np.float64)
-    lse = np.empty((B, Hq, N), np.float64)
+    rp, R = None, N
+    if rows is not None:
+        ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        rp, R = ra.ctypes.data_as(ctypes.c_void_p), ra.size
+    o = np.empty((B, R, Hq, d), np.float64)
+    lse = np.empty((B, Hq, R), np.float64)
     _check(lib().oracle_attn_fp8(q8, qs, int(qblock), k8, ks, int(kblock), v8, vs, B, N, Hq,
-                                 Hkv, d, int(causal), int(window), float(scale), o, lse),
+                                 Hkv, d, int(causal), int(window), float(scale), rp, R, o, lse),
            "attn_fp8")
     return o, lse
 

@@ -871,9 +871,13 @@ int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_cache, const uint1
  *   - Q and K get one scale per (batch, head, block of 128 tokens), V (not
  *     rotated) one per (batch, KV head): V's contraction runs over all keys,
  *     so its scale has to factor out of the whole sum;
- *   - scale = amax / 448 of the block (448 = largest finite E4M3), stored as
- *     fp32 (1 when the block is all zero); code = the E4M3 value nearest to
- *     x / scale, ties to the even code, saturated to +-448.
+ *   - the pages do not say how a block's scale is chosen: here it is the
+ *     smallest power of two 2^k with amax / 2^k <= 448 (448 = largest finite
+ *     E4M3; k >= -126 so that 1 / scale is a finite fp32), 1 for an all-zero
+ *     block -- the power-of-two scales of the OCP microscaling formats.  Then
+ *     x / scale is exact and the code is decided on the exact value: the
+ *     E4M3 value nearest to x / scale, ties to the even code, saturated to
+ *     +-448.
  * The attention is then the plain definition applied to the dequantised
  * values code * scale.
  */
@@ -946,6 +950,17 @@ uint8_t oracle_e4m3_encode(double y)
     return (uint8_t)((sign << 7) | (field << 3) | mant);
 }
 
+/* The scale of a block whose largest magnitude is amax (see above). */
+float oracle_e4m3_block_scale(double amax)
+{
+    if (!(amax > 0.0)) return 1.0f;
+    int e;
+    const double f = frexp(amax, &e);          /* amax = f * 2^e, f in [0.5, 1) */
+    int k = (f <= 0.875) ? e - 9 : e - 8;       /* 448 = 0.875 * 2^9 */
+    if (k < -126) k = -126;
+    return (float)ldexp(1.0, k);
+}
+
 /*
  * Block-scaled E4M3 quantisation of x [B, N, H, d] (fp64): one scale per
  * (b, h, block of `block` tokens), scales [B, H, ceil(N / block)] fp32.
@@ -967,7 +982,7 @@ int oracle_quantize_e4m3_blocks(const double *x, int B, int N, int H, int d, int
                 const double v = fabs(x[(((int64_t)b * N + n) * H + h) * d + c]);
                 if (v > amax) amax = v;
             }
-        const float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+        const float sc = oracle_e4m3_block_scale(amax);
         scales[((int64_t)b * H + h) * nblk + blk] = sc;
         for (int n = n0; n < n1; ++n)
             for (int c = 0; c < d; ++c) {
@@ -983,17 +998,21 @@ int oracle_quantize_e4m3_blocks(const double *x, int B, int N, int H, int d, int
  * qblock)], k8 [B, N, Hkv, d] with k_scale [B, Hkv, ceil(N / kblock)], v8
  * [B, N, Hkv, d] with v_scale [B, Hkv].  Each value is code * its scale;
  * then the definition with causal / window masks as in oracle_attn.
- *   o [B, N, Hq, d], lse [B, Hq, N] (fp64)
+ *   rows: the query positions to compute in every batch (NULL = all N, in order)
+ *   o [B, nrows, Hq, d], lse [B, Hq, nrows] (fp64)
  */
 int oracle_attn_fp8(const uint8_t *q8, const float *q_scale, int qblock,
                     const uint8_t *k8, const float *k_scale, int kblock,
                     const uint8_t *v8, const float *v_scale,
                     int B, int N, int Hq, int Hkv, int d, int causal, int window,
-                    double scale, double *o, double *lse)
+                    double scale, const int64_t *rows, int64_t nrows, double *o, double *lse)
 {
     if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv || qblock <= 0 ||
         kblock <= 0)
         return -1;
+    if (!rows) nrows = N;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows && (rows[r] < 0 || rows[r] >= N)) return -1;
     const int group = Hq / Hkv;
     const int nbq = (N + qblock - 1) / qblock, nbk = (N + kblock - 1) / kblock;
     int bad = 0;
@@ -1012,9 +1031,10 @@ int oracle_attn_fp8(const uint8_t *q8, const float *q_scale, int qblock,
             bad = 1;
         } else {
 #pragma omp for schedule(dynamic, 1)
-            for (int64_t task = 0; task < (int64_t)B * N * Hq; ++task) {
-                const int b = (int)(task / ((int64_t)N * Hq));
-                const int i = (int)((task / Hq) % N);
+            for (int64_t task = 0; task < (int64_t)B * nrows * Hq; ++task) {
+                const int b = (int)(task / (nrows * Hq));
+                const int64_t r = (task / Hq) % nrows;
+                const int i = (int)(rows ? rows[r] : r);
                 const int h = (int)(task % Hq), g = h / group;
                 const double qs = (double)q_scale[((int64_t)b * Hq + h) * nbq + i / qblock];
                 for (int c = 0; c < d; ++c)
@@ -1035,7 +1055,7 @@ int oracle_attn_fp8(const uint8_t *q8, const float *q_scale, int qblock,
                 double l;
                 attend_row_fp8(qd, d, nk, kp, vp, ksr, vsr, scale, -INFINITY, sb, orow, &l);
                 for (int c = 0; c < d; ++c) o[task * d + c] = orow[c];
-                lse[((int64_t)b * Hq + h) * N + i] = l;
+                lse[((int64_t)b * Hq + h) * nrows + r] = l;
             }
         }
         free(sb); free(ksr); free(vsr); free(qd); free(orow); free(kp); free(vp);

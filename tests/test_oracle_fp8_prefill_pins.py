@@ -10,8 +10,9 @@ precision").  Pins, none produced by the oracle itself:
     invariants of an orthogonal map (norms and Q.K dot products kept);
   - E4M3 rounding against torch's float8_e4m3fn cast (a library routine) and
     a brute-force nearest-code search over all 254 finite codes;
-  - block scales: each block's largest magnitude lands on code 448, blocks are
-    independent, an all-zero block gets scale 1;
+  - block scales: the smallest power of two that brings the block's largest
+    magnitude to at most 448 (checked against a search over powers of two),
+    blocks independent, an all-zero block at scale 1;
   - the attention over codes against the pinned bf16 oracle on values both
     can hold exactly;
   - the pages' claim: with outlier channels the rotated FP8 attention is
@@ -113,15 +114,30 @@ def test_block_scales():
                 if amax == 0:
                     assert scales[b, h, j] == 1.0 and np.all(cs == 0)
                     continue
-                assert scales[b, h, j] == np.float32(amax / 448.0)
-                # the block's largest magnitude is the largest code
+                sc = float(scales[b, h, j])
+                # a power of two, the smallest with amax / scale <= 448
+                assert sc == 2.0 ** round(math.log2(sc))
+                assert amax / sc <= 448.0 < amax / (sc / 2.0)
+                # the block's largest magnitude lands in the top binade
                 i = np.unravel_index(np.abs(xs).argmax(), xs.shape)
-                assert cs[i] & 0x7F == 0x7E
+                assert 224.0 <= oracle.e4m3_value(int(cs[i]) & 0x7F) <= 448.0
                 # every value within half a grid step (relative 2^-4) of its code
                 deq = np.vectorize(oracle.e4m3_value)(cs) * float(scales[b, h, j])
                 tol = np.maximum(np.abs(xs) * 2.0 ** -4, 2.0 ** -10 * float(scales[b, h, j]))
                 assert np.all(np.abs(deq - xs) <= tol * (1 + 1e-12))
-    assert scales[1, 0, 1] == np.float32(37.0 / 448.0)
+    assert scales[1, 0, 1] == 0.125          # 37 / 0.125 = 296 <= 448 < 592
+
+
+def test_block_scale_by_search():
+    rng = np.random.default_rng(15)
+    amaxes = np.concatenate([np.exp2(rng.uniform(-130, 120, 2000)),
+                             [448.0, 449.0, 224.0, 223.9, 1.0, 3.5, 7.0, 448.0 * 2 ** -20]])
+    for a in amaxes:
+        k = -126
+        while a / 2.0 ** k > 448.0:
+            k += 1
+        assert oracle.e4m3_block_scale(a) == np.float32(2.0 ** k), a
+    assert oracle.e4m3_block_scale(0.0) == 1.0
 
 
 @pytest.mark.parametrize("causal,window", [(0, 0), (1, 0), (1, 40)])
@@ -188,3 +204,20 @@ def test_incoherent_processing_reduces_error_with_outliers():
     e_plain = np.sqrt(((o_plain - ref) ** 2).mean())
     e_rot = np.sqrt(((o_rot - ref) ** 2).mean())
     assert e_rot * 2.0 < e_plain, (e_rot, e_plain)
+
+
+def test_attn_fp8_rows_are_a_selection():
+    B, N, Hq, Hkv, d = 2, 200, 2, 1, 16
+    rng = np.random.default_rng(41)
+    finite = np.array([c for c in range(256) if (c & 0x7F) <= 0x58])
+    q8 = rng.choice(finite, (B, N, Hq, d)).astype(np.uint8)
+    k8 = rng.choice(finite, (B, N, Hkv, d)).astype(np.uint8)
+    v8 = rng.choice(finite, (B, N, Hkv, d)).astype(np.uint8)
+    qs = rng.uniform(0.01, 0.1, (B, Hq, 2)).astype(np.float32)
+    ks = rng.uniform(0.01, 0.1, (B, Hkv, 2)).astype(np.float32)
+    vs = rng.uniform(0.5, 2.0, (B, Hkv)).astype(np.float32)
+    rows = [0, 5, 127, 128, 199]
+    for causal, window in ((0, 0), (1, 0), (1, 30)):
+        o, lse = oracle.attn_fp8(q8, qs, k8, ks, v8, vs, causal, window, 0.2)
+        os_, ls = oracle.attn_fp8(q8, qs, k8, ks, v8, vs, causal, window, 0.2, rows=rows)
+        assert np.array_equal(os_, o[:, rows]) and np.array_equal(ls, lse[:, :, rows])
