@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--no-next", action="store_true",
                     help="skip the extension rows (backward, FP8-cache decode)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "bwd", "decode_fp8",
-                                       "prefill_paged"],
+                                       "prefill_paged", "prefill_fp8"],
                     default="all",
                     help="time one kernel family only (for profiler captures)")
     ap.add_argument("--prefill-workload", default=PREFILL,
@@ -237,9 +237,9 @@ def bench_ours(args):
     pk, pk_src = peaks()
 
     # ---- inputs (seeded per rank; resident in HBM before timing)
-    do_p = args.only in ("all", "prefill", "bwd")
+    do_p = args.only in ("all", "prefill", "bwd", "prefill_fp8")
     do_d = args.only in ("all", "decode", "decode_fp8")
-    if args.only in ("bwd", "decode_fp8", "prefill_paged"):
+    if args.only in ("bwd", "decode_fp8", "prefill_paged", "prefill_fp8"):
         return bench_only_next(fa_import(), args, do_p, do_d)
     pname = args.prefill_workload
     seed = rank_seed(args.seed, rank)
@@ -459,7 +459,12 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
       bwd        -- fa_bwd on the prefill workload: FLOPs = 2.5 x the forward's
                     (five GEMMs of the forward's size per tile against two);
       decode_fp8 -- fa_decode_paged_fp8 over the decode workload's cache stored
-                    as FP8 E4M3 with a scale per (page, KV head): KV bytes halve.
+                    as FP8 E4M3 with a scale per (page, KV head): KV bytes halve;
+      prefill_paged -- fa_fwd_paged on a chunked-prefill workload;
+      prefill_fp8 -- fa_fp8_prepare (Hadamard rotation + E4M3 operands) and
+                    fa_fwd_fp8 on the prefill workload: the attention's FLOPs
+                    against the FP8 tensor peak, the preparation's bytes
+                    against HBM.
     """
     K = args.steps
     out = {}
@@ -486,6 +491,9 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
                        dout, dlse, out)
     if which in ("all", "prefill_paged"):
         bench_next_paged(fa, args, dev, timed, pk, traffic_all, out)
+    if which in ("all", "prefill_fp8"):
+        bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse,
+                               flops, out)
     err = fa.check_device_error()
     if err:
         raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
@@ -511,6 +519,45 @@ def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, 
                                "kernel": "bwd_kernel (+ bwd_prep_kernel, bwd_convert_kernel)",
                                "traffic": traffic_all.get("bwd_gqa4k")}}
     del g, gq, gk, gv, wsb
+
+
+def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, flops,
+                           out):
+    signs = workloads.hadamard_signs(q.shape[3], seed=args.seed).to(dev)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    ws = torch.empty(max(fa.fp8_workspace_bytes(B, N, Hkv), 4), dtype=torch.uint8, device=dev)
+    prep = fa.fp8_prepare(q, k, v, signs, workspace=ws)
+    ms_prep = timed(lambda: fa.fp8_prepare(q, k, v, signs, out=prep, workspace=ws))
+    ms = timed(lambda: fa.fwd_fp8(prep, True, pin.window, pin.scale, out=o, lse=lse))
+    ach = flops / (ms * 1e-3) / 1e12
+    peak8 = 2.0 * pk["bf16_tflops"]          # FP8 dense = 2 x bf16 (nominal ratio)
+    # preparation: bf16 Q, K, V read, E4M3 codes written (V read twice: its
+    # block maxima, then its codes)
+    elems = q.numel() + k.numel() + v.numel()
+    prep_bytes = 3.0 * elems
+    prep_gbs = prep_bytes / (ms_prep * 1e-3) / 1e9
+    out["prefill_fp8"] = {
+        "value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+        "flop_per_call": flops, "launches_per_call": 1,
+        "with_prepare": {"value": round(flops / ((ms + ms_prep) * 1e-3) / 1e12, 2),
+                         "unit": "TFLOP/s", "ms_per_call": round(ms + ms_prep, 4),
+                         "launches_per_call": 3},
+        "workload": "FP8 prefill of the prefill workload: Q, K rotated by a random-sign "
+                    "Hadamard matrix, E4M3 with 128-token block scales (V per head), causal",
+        "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak8, 1),
+                     "unit": "TFLOP/s", "frac": round(ach / peak8, 4),
+                     "peak_source": "measured bf16 burst x 2 (nominal FP8:bf16 ratio)",
+                     "kernel": "prefill_kernel<128> (FP8 mode)",
+                     "traffic": traffic_all.get("prefill_fp8_gqa4k")},
+        "prepare": {"ms_per_call": round(ms_prep, 4), "bytes_per_call": prep_bytes,
+                    "launches_per_call": 2,
+                    "roofline": {"bound": "hbm", "achieved": round(prep_gbs, 1),
+                                 "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                 "frac": round(prep_gbs / pk["hbm_gbs"], 4),
+                                 "kernel": "fp8_quant_qk_kernel + fp8_quant_vt_kernel",
+                                 "traffic": traffic_all.get("fp8_prepare_gqa4k")}}}
+    del prep, ws
 
 
 def paged_prefill_workload(seed):

@@ -12,6 +12,8 @@ Functions mirror the C entry points:
     bwd            -> fa_bwd            (dense backward: dQ, dK, dV)
     bwd_varlen     -> fa_bwd_varlen     (packed-sequence backward)
     decode_paged   -> fa_decode_paged   (paged split-KV decode)
+    fp8_prepare    -> fa_fp8_prepare    (Hadamard rotation + E4M3 operands)
+    fwd_fp8        -> fa_fwd_fp8        (FP8 prefill on those operands)
     decode_paged_noalloc, decode_workspace_bytes, bwd_workspace_bytes,
     check_device_error, selftest_watchdog, status_string, version
 """
@@ -41,7 +43,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa
            "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen", "fa_bwd_sinks",
            "fa_bwd_varlen_sinks",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
-           "fa_decode_paged_fp8",
+           "fa_decode_paged_fp8", "fa_fp8_workspace_bytes", "fa_fp8_prepare", "fa_fwd_fp8",
            "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
            "fa_selftest_watchdog", "fa_version")
 
@@ -75,6 +77,12 @@ def _load():
     lib.fa_fwd_paged.restype = i
     lib.fa_decode_paged_fp8.argtypes = [vp] * 10 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged_fp8.restype = i
+    lib.fa_fp8_workspace_bytes.argtypes = [i] * 3
+    lib.fa_fp8_workspace_bytes.restype = sz
+    lib.fa_fp8_prepare.argtypes = [vp] * 10 + [i] * 5 + [vp, sz, vp]
+    lib.fa_fp8_prepare.restype = i
+    lib.fa_fwd_fp8.argtypes = [vp] * 8 + [i] * 7 + [f, i, vp]
+    lib.fa_fwd_fp8.restype = i
     lib.fa_bwd_workspace_bytes.argtypes = [i] * 3
     lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_bwd.argtypes = [vp] * 9 + [i] * 7 + [f, vp, sz, vp]
@@ -180,6 +188,75 @@ def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
         return out, lse
     _check(_lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
                        int(causal), int(window), float(scale), od, _stream(stream)), "fa_fwd")
+    return out, lse
+
+
+FP8_BLOCK = 128   # tokens per Q / K scale block
+
+
+def fp8_workspace_bytes(B, N, Hkv) -> int:
+    return int(_lib.fa_fp8_workspace_bytes(int(B), int(N), int(Hkv)))
+
+
+def fp8_prepare(q, k, v, signs=None, out=None, workspace=None, stream=None):
+    """E4M3 operands of the FP8 prefill.  q [B,N,Hq,128], k/v [B,N,Hkv,128] bf16;
+    signs fp32 [128] of +-1 (device) or None (no rotation).  Returns a dict with
+    q8 [B,N,Hq,128], k8 [B,N,Hkv,128] uint8 codes, vt8 [B,Hkv,128,vt_stride]
+    uint8 (V transposed), q_scale [B,Hq,nblk], k_scale [B,Hkv,nblk], v_scale
+    [B,Hkv] fp32.  ``out`` may be such a dict to fill in place."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, 4, n)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
+        raise FAError(FA_ERR_INVALID_ARG, "k/v shape")
+    if signs is not None:
+        _need(signs, torch.float32, 1, "signs")
+        if signs.numel() != d:
+            raise FAError(FA_ERR_INVALID_ARG, "signs shape")
+    nblk = (N + FP8_BLOCK - 1) // FP8_BLOCK
+    vts = (N + 15) // 16 * 16
+    dev = q.device
+    if out is None:
+        out = {"q8": torch.empty((B, N, Hq, d), dtype=torch.uint8, device=dev),
+               "k8": torch.empty((B, N, Hkv, d), dtype=torch.uint8, device=dev),
+               "vt8": torch.empty((B, Hkv, d, vts), dtype=torch.uint8, device=dev),
+               "q_scale": torch.empty((B, Hq, nblk), dtype=torch.float32, device=dev),
+               "k_scale": torch.empty((B, Hkv, nblk), dtype=torch.float32, device=dev),
+               "v_scale": torch.empty((B, Hkv), dtype=torch.float32, device=dev)}
+    ws_need = fp8_workspace_bytes(B, N, Hkv)
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 4), dtype=torch.uint8, device=dev)
+    _check(_lib.fa_fp8_prepare(_ptr(q), _ptr(k), _ptr(v), _ptr(signs), _ptr(out["q8"]),
+                               _ptr(out["k8"]), _ptr(out["vt8"]), _ptr(out["q_scale"]),
+                               _ptr(out["k_scale"]), _ptr(out["v_scale"]), B, N, Hq, Hkv, d,
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)), "fa_fp8_prepare")
+    return out
+
+
+def fwd_fp8(prep, causal=False, window=0, scale=None, out_dtype=torch.bfloat16, out=None,
+            lse=None, return_lse=True, stream=None):
+    """FP8 prefill on fp8_prepare's operands -> (O [B,N,Hq,128], LSE [B,Hq,N])."""
+    q8, k8, vt8 = prep["q8"], prep["k8"], prep["vt8"]
+    _need(q8, torch.uint8, 4, "q8")
+    _need(k8, torch.uint8, 4, "k8")
+    _need(vt8, torch.uint8, 4, "vt8")
+    B, N, Hq, d = q8.shape
+    Hkv = k8.shape[2]
+    if tuple(k8.shape) != (B, N, Hkv, d) or tuple(vt8.shape) != (B, Hkv, d, (N + 15) // 16 * 16):
+        raise FAError(FA_ERR_INVALID_ARG, "k8/vt8 shape")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, N, Hq, d), dtype=out_dtype, device=q8.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q8.device)
+    od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    _check(_lib.fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(prep["q_scale"]),
+                           _ptr(prep["k_scale"]), _ptr(prep["v_scale"]), _ptr(out), _ptr(lse),
+                           B, Hq, Hkv, N, d, int(causal), int(window), float(scale), od,
+                           _stream(stream)), "fa_fwd_fp8")
     return out, lse
 
 

@@ -517,6 +517,71 @@ int fa_decode_paged_sinks(const void *q, const void *k_cache, const void *v_cach
                             scale, workspace, workspace_bytes, stream);
 }
 
+size_t fa_fp8_workspace_bytes(int B, int N, int Hkv) {
+    if (B <= 0 || N <= 0 || Hkv <= 0) return 0;
+    return (size_t)B * Hkv * (size_t)((N + 127) / 128) * sizeof(float);
+}
+
+int fa_fp8_prepare(const void *q, const void *k, const void *v, const float *signs,
+                   void *q8, void *k8, void *vt8, float *q_scale, float *k_scale,
+                   float *v_scale, int B, int N, int Hq, int Hkv, int d, void *workspace,
+                   size_t workspace_bytes, void *stream) {
+    if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (d != 128) return (d == 64) ? FA_ERR_UNSUPPORTED : FA_ERR_INVALID_ARG;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q || !k || !v || !q8 || !k8 || !vt8 || !q_scale || !k_scale || !v_scale)
+        return FA_ERR_INVALID_ARG;
+    if ((long long)B * N > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    const size_t need = fa_fp8_workspace_bytes(B, N, Hkv);
+    if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q8) || !aligned16(k8) ||
+        !aligned16(vt8) || (signs && !aligned16(signs)) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3) || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3) || (reinterpret_cast<uintptr_t>(workspace) & 3))
+        return FA_ERR_ALIGNMENT;
+    fa::Fp8PrepArgs a{};
+    a.q = q; a.k = k; a.v = v; a.signs = signs;
+    a.q8 = q8; a.k8 = k8; a.vt8 = vt8;
+    a.q_scale = q_scale; a.k_scale = k_scale; a.v_scale = v_scale;
+    a.v_block_max = static_cast<float *>(workspace);
+    a.B = B; a.N = N; a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.vt_stride = (N + 15) / 16 * 16;
+    return map_rc(fa::launch_fp8_prepare(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_fp8(const void *q8, const void *k8, const void *vt8, const float *q_scale,
+               const float *k_scale, const float *v_scale, void *o, float *lse, int B,
+               int Hq, int Hkv, int N, int d, int causal, int window, float scale,
+               int o_dtype, void *stream) {
+    if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
+    int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
+    if (rc) return rc;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (B == 0 || N == 0) return FA_OK;
+    if (!q8 || !k8 || !vt8 || !o || !q_scale || !k_scale || !v_scale) return FA_ERR_INVALID_ARG;
+    if ((long long)B * N > INT32_MAX / 2) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(vt8) || !aligned16(o) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3) || (reinterpret_cast<uintptr_t>(k_scale) & 3) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3))
+        return FA_ERR_ALIGNMENT;
+    fa::PrefillArgs a{};
+    a.q = q8; a.k = k8; a.v = vt8; a.o = o; a.lse = lse;
+    a.cu_seqlens = nullptr;
+    a.num_seqs = B;
+    a.seqlen = N;
+    a.total_tokens = B * N;
+    a.max_seqlen = N;
+    a.Hq = Hq; a.Hkv = Hkv; a.d = d;
+    a.causal = causal;
+    a.window = window > 0 ? window : 0;
+    a.scale = scale;
+    a.o_fp32 = o_dtype == FA_OUT_FP32;
+    a.q_scale = q_scale; a.k_scale = k_scale; a.v_scale = v_scale;
+    a.vt_stride = (N + 15) / 16 * 16;
+    return map_rc(fa::launch_prefill_fp8(a, static_cast<cudaStream_t>(stream)));
+}
+
 const char *fa_status_string(int status) {
     switch (status) {
     case FA_OK: return "ok";

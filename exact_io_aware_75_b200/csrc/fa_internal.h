@@ -28,9 +28,27 @@ struct PrefillArgs {
     int max_pages, num_pages;
     // document mask: one id per token; nullptr = none
     const int *doc;
+    // FP8 operands (launch_prefill_fp8): q, k hold E4M3 codes, v the
+    // transposed V codes [B, Hkv, d, vt_stride]; scales per (sequence, head,
+    // 128-token block) for Q and K, per (sequence, KV head) for V
+    const float *q_scale, *k_scale, *v_scale;
+    int vt_stride;
 };
 
 int launch_prefill(const PrefillArgs &a, cudaStream_t stream);
+int launch_prefill_fp8(const PrefillArgs &a, cudaStream_t stream);
+
+// Rotation and E4M3 quantisation of the FP8 prefill's operands.
+struct Fp8PrepArgs {
+    const void *q, *k, *v;      // bf16 [B*N, H, d]
+    const float *signs;         // [d] +-1, or nullptr: no rotation
+    void *q8, *k8, *vt8;        // codes; vt8 [B, Hkv, d, vt_stride]
+    float *q_scale, *k_scale, *v_scale;
+    float *v_block_max;         // workspace [B, Hkv, nblk]
+    int B, N, Hq, Hkv, d, vt_stride;
+};
+
+int launch_fp8_prepare(const Fp8PrepArgs &a, cudaStream_t stream);
 
 struct DecodeArgs {
     const void *q, *k_cache, *v_cache;

@@ -5,3 +5,4 @@
 #include "decode_sm100.cu"
 #include "decode_noalloc.cu"
 #include "bwd_sm100.cu"
+#include "fp8_prep.cu"

@@ -68,12 +68,16 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kPageRows = 16;                 // tokens per cache page (paged mode)
 constexpr int kPagesPerTile = 128 / kPageRows;
 
-template <int D, bool DOC = false>
+template <int D, bool DOC = false, bool F8 = false>
 struct Cfg {
-    static constexpr int kBoxBytes = kBlockM * 64 * 2;             // 128 rows x 64 bf16
-    static constexpr int kTileBytes = kBlockM * D * 2;             // Q tile or K/V tile
-    // K/V ring slots (one fewer with a document mask, for its key-id buffers)
-    static constexpr int kStages = (D == 128) ? (DOC ? 4 : 5) : 6;
+    static constexpr int kElem = F8 ? 1 : 2;                       // bytes per element
+    static constexpr int kBoxCols = 128 / kElem;                   // elements per 128-byte row
+    static constexpr int kBoxes = D / kBoxCols;                    // TMA boxes per tile
+    static constexpr int kBoxBytes = kBlockM * 128;                // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kBlockM * D * kElem;         // Q tile or K/V tile
+    // K/V ring slots (one fewer with a document mask, for its key-id buffers;
+    // FP8 tiles are half the size)
+    static constexpr int kStages = F8 ? 8 : (D == 128) ? (DOC ? 4 : 5) : 6;
     static constexpr int kDocBytes = DOC ? 8 * 2 * 128 * 4 : 0;   // [warp][parity][key]
     static constexpr int kSmemBytes = 2 * kTileBytes + kStages * kTileBytes + kDocBytes + 1024;
     static constexpr uint32_t kColO = 256;                         // O_t at 256 + t*D
@@ -101,6 +105,10 @@ struct Params {
     // Document mask: one id per token (packed order); key j is visible from
     // query i only if both ids are equal.
     const int *doc;
+    // FP8 operands (dense batches): E4M3 codes with scales per (sequence,
+    // head, 128-token block) for Q and K, per (sequence, KV head) for V.
+    const float *q_scale, *k_scale, *v_scale;
+    int nblk;   // 128-token blocks per sequence
 };
 
 struct Unit {
@@ -185,10 +193,12 @@ struct Shared {
 
 // ------------------------------------------------------------- TMA producer
 // Dense and packed batches: one thread issues every copy.
-template <int D, bool DOC>
+// FP8: one 128-byte box per tile row; V comes transposed (d rows of 128
+// keys), so its tile is read at (key, 0, sequence * Hkv + KV head).
+template <int D, bool DOC, bool F8>
 __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                          const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
-    using C = Cfg<D, DOC>;
+    using C = Cfg<D, DOC, F8>;
     volatile int *abort = &sh.abort;
     uint32_t q_uses[2] = {0, 0};
     uint32_t kv_it = 0;
@@ -199,9 +209,9 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
             if (w.lo[t] >= w.hi[t]) continue;
             if (!mbar_wait(&sh.q_empty[t], (q_uses[t] & 1) ^ 1, abort)) goto out;
             mbar_arrive_expect_tx(&sh.q_full[t], C::kTileBytes);
-            for (int b = 0; b < D / 64; ++b)
+            for (int b = 0; b < C::kBoxes; ++b)
                 tma_load_3d(sQ + t * C::kTileBytes + b * C::kBoxBytes, tmQ, &sh.q_full[t],
-                            b * 64, w.h, w.tok0 + w.q0 + t * kBlockM);
+                            b * C::kBoxCols, w.h, w.tok0 + w.q0 + t * kBlockM);
             ++q_uses[t];
         }
         for (int j = w.lo_all; j < w.hi_all; ++j) {
@@ -210,9 +220,15 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
                 const uint32_t use = kv_it / C::kStages;
                 if (!mbar_wait(&sh.kv_empty[slot], (use & 1) ^ 1, abort)) goto out;
                 mbar_arrive_expect_tx(&sh.kv_full[slot], C::kTileBytes);
-                for (int b = 0; b < D / 64; ++b)
-                    tma_load_3d(sKV + slot * C::kTileBytes + b * C::kBoxBytes, kv ? tmV : tmK,
-                                &sh.kv_full[slot], b * 64, w.kvh, w.tok0 + j * kBlockN);
+                if (F8 && kv) {
+                    tma_load_3d(sKV + slot * C::kTileBytes, tmV, &sh.kv_full[slot], j * kBlockN,
+                                0, w.seq * p.Hkv + w.kvh);
+                } else {
+                    for (int b = 0; b < C::kBoxes; ++b)
+                        tma_load_3d(sKV + slot * C::kTileBytes + b * C::kBoxBytes, kv ? tmV : tmK,
+                                    &sh.kv_full[slot], b * C::kBoxCols, w.kvh,
+                                    w.tok0 + j * kBlockN);
+                }
                 ++kv_it;
             }
         }
@@ -339,13 +355,14 @@ out:
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <int D, bool PAGED, bool DOC>
+template <int D, bool PAGED, bool DOC, bool F8>
 __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
-    using C = Cfg<D, DOC>;
+    using C = Cfg<D, DOC, F8>;
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
-    const uint32_t idS = idesc_bf16_f32(kBlockM, kBlockN, false);
-    const uint32_t idPV = idesc_bf16_f32(kBlockM, D, true);
+    const uint32_t idS = F8 ? idesc_e4m3_f32(kBlockM, kBlockN)
+                            : idesc_bf16_f32(kBlockM, kBlockN, false);
+    const uint32_t idPV = F8 ? idesc_e4m3_f32(kBlockM, D) : idesc_bf16_f32(kBlockM, D, true);
     const uint32_t q_addr = smem_u32(sQ), kv_addr = smem_u32(sKV);
     uint32_t q_uses[2] = {0, 0}, p_cnt[2] = {0, 0}, oe_uses[2] = {0, 0};
     uint32_t kv_it = 0;
@@ -353,30 +370,45 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
     // S_t = Q_t K^T: d/16 MMAs of K=16; K-major, 128-byte swizzle, atoms of
     // 8 rows x 128 bytes (SBO 1024), 64 columns per TMA box.  Descriptors
     // are precomputed; a k-step adds its byte offset >> 4 to the low half.
+    // (FP8: K = 32 per MMA, the same 32 bytes per k-step.)
     const uint32_t q_lo = desc_lo(q_addr, 16), kv_lo = desc_lo(kv_addr, 16);
-    const uint32_t v_lo = desc_lo(kv_addr, C::kBoxBytes);
+    const uint32_t v_lo = desc_lo(kv_addr, F8 ? 16 : C::kBoxBytes);
     constexpr uint32_t kTileStep = C::kTileBytes >> 4;
     auto issue_s = [&](int t, int kslot) {
         const uint32_t qa = q_lo + t * kTileStep;
         const uint32_t ka = kv_lo + kslot * kTileStep;
         const uint32_t dt = tmem + t * kBlockN;
         #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
+        for (int ks = 0; ks < D * C::kElem / 32; ++ks) {
             const uint32_t off = ((ks >> 2) * C::kBoxBytes + (ks & 3) * 32) >> 4;
-            mma_ss_lo(dt, qa + off, ka + off, idS, ks > 0 ? 1u : 0u);
+            if constexpr (F8)
+                mma_ss_lo_f8(dt, qa + off, ka + off, idS, ks > 0 ? 1u : 0u);
+            else
+                mma_ss_lo(dt, qa + off, ka + off, idS, ks > 0 ? 1u : 0u);
         }
     };
     // O_t += P_t V: 128/16 MMAs of K=16 keys; V is MN-major (d contiguous):
     // 16 keys = two 8-row groups (SBO 1024), d split in 64-column boxes (LBO).
+    // FP8: V^T is K-major (keys contiguous), 32 keys per MMA; P holds four
+    // codes per TMEM column, so 64 keys are 16 columns.
     auto issue_pv_half = [&](int t, int vslot, bool first, int half) {
         const uint32_t va = v_lo + vslot * kTileStep;
         const uint32_t dt = tmem + C::kColO + t * D;
         const uint32_t pa = tmem + t * kBlockN;
-        #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int ks = half * 4 + k;
-            mma_ts_lo(dt, pa + half * kHalf + k * 8, va + ((ks * 2048) >> 4), idPV,
-                      (ks > 0 || !first) ? 1u : 0u);
+        if constexpr (F8) {
+            #pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int ks = half * 2 + k;
+                mma_ts_lo_f8(dt, pa + ks * 8, va + ((ks * 32) >> 4), idPV,
+                             (ks > 0 || !first) ? 1u : 0u);
+            }
+        } else {
+            #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int ks = half * 4 + k;
+                mma_ts_lo(dt, pa + half * kHalf + k * 8, va + ((ks * 2048) >> 4), idPV,
+                          (ks > 0 || !first) ? 1u : 0u);
+            }
         }
     };
     // P_t V in two halves of 64 keys, each issued as soon as the softmax
@@ -491,10 +523,32 @@ __device__ __forceinline__ void exp_half(const float (&v)[kHalf], float sl2, flo
     acc = f2add(a2[0], a2[1]);
 }
 
+// The same for the FP8 kernel: P as E4M3 codes, four per 32-bit word (P is
+// at most 2^8 under the conditional rescale, inside E4M3's range of 448).
+// The running sum takes the fp32 values.
+__device__ __forceinline__ void exp_half_f8(const float (&v)[kHalf], float sl2, float mb,
+                                            uint32_t (&pk)[kHalf / 4], uint64_t &acc) {
+    const uint64_t c2 = f2pack(sl2, sl2), nm2 = f2pack(-mb, -mb);
+    uint64_t a2[2] = {acc, f2pack(0.f, 0.f)};
+    #pragma unroll
+    for (int c = 0; c < kHalf / 4; ++c) {
+        const uint64_t x = f2fma(f2pack(v[4 * c], v[4 * c + 1]), c2, nm2);
+        const uint64_t y = f2fma(f2pack(v[4 * c + 2], v[4 * c + 3]), c2, nm2);
+        float x0, x1, y0, y1;
+        f2unpack(x, x0, x1);
+        f2unpack(y, y0, y1);
+        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(y0), p3 = ex2(y1);
+        a2[0] = f2add(a2[0], f2pack(p0, p1));
+        a2[1] = f2add(a2[1], f2pack(p2, p3));
+        pk[c] = pack_e4m3x4(p0, p1, p2, p3);
+    }
+    acc = f2add(a2[0], a2[1]);
+}
+
 // ---------------------------------------------------------------- softmax
-template <int D, bool PAGED, bool DOC>
+template <int D, bool PAGED, bool DOC, bool F8>
 __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
-    using C = Cfg<D, DOC>;
+    using C = Cfg<D, DOC, F8>;
     volatile int *abort = &sh.abort;
     const int warp = warp_id(), lane = lane_id();
     const int t = warp >> 2;                 // tile of this warpgroup
@@ -502,7 +556,6 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
     const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = sh.tmem_base + lanes + t * kBlockN;
     const uint32_t tO = sh.tmem_base + lanes + C::kColO + t * D;
-    const float sl2 = p.scale_log2;
     uint32_t s_cnt = 0, pv_cnt = 0;
 
     FOR_EACH_UNIT(u) {
@@ -529,8 +582,19 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             mydoc = (row < w.L) ? __ldg(p.doc + w.tok0 + row) : INT_MIN + 1;
             load_key_docs(lo);
         }
+        // FP8: scores come out in units of q_scale * k_scale; both fold into
+        // the exponent's factor, per key block.  V's scale divides O at the end.
+        float sq = 1.f, sv = 1.f;
+        const float *ksc = nullptr;
+        if constexpr (F8) {
+            sq = __ldg(p.q_scale + ((size_t)w.seq * p.Hq + w.h) * p.nblk + (w.q0 >> 7) + t);
+            sv = __ldg(p.v_scale + (size_t)w.seq * p.Hkv + w.kvh);
+            ksc = p.k_scale + ((size_t)w.seq * p.Hkv + w.kvh) * p.nblk;
+        }
         float m_ref = -INFINITY, l = 0.f;
         for (int j = lo; j < hi; ++j) {
+            float sl2 = p.scale_log2;
+            if constexpr (F8) sl2 *= sq * __ldg(ksc + j);
             if (!mbar_wait_warp(&sh.s_full[t], s_cnt & 1, abort)) return;
             // the block's key ids, staged per warp (no cross-warp barrier)
             const int *kd = nullptr;
@@ -582,9 +646,16 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             // conditional rescale) the first half's P needs no block max:
             // start its exponentials while the block max is still unknown.
             float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-            uint32_t pkA[kHalf / 2];
+            uint32_t pkA[F8 ? kHalf / 4 : kHalf / 2];
             uint64_t accA = f2pack(0.f, 0.f);
-            if (!first) exp_half(sA, sl2, mb, pkA, accA);
+            auto exp_any = [&](const float (&v)[kHalf], uint32_t (&pk)[F8 ? kHalf / 4 : kHalf / 2],
+                               uint64_t &acc) {
+                if constexpr (F8)
+                    exp_half_f8(v, sl2, mb, pk, acc);
+                else
+                    exp_half(v, sl2, mb, pk, acc);
+            };
+            if (!first) exp_any(sA, pkA, accA);
             tmem_wait_ld();
             #pragma unroll
             for (int c = 0; c < kHalf; ++c) sB[c] = __uint_as_float(rawB[c]);
@@ -626,20 +697,26 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             if (redo) {
                 mb = (m_ref == -INFINITY) ? 0.f : m_ref;
                 accA = f2pack(0.f, 0.f);
-                exp_half(sA, sl2, mb, pkA, accA);
+                exp_any(sA, pkA, accA);
             }
-            // publish P for keys 0-63 (bf16 pairs in S columns 0-31): the MMA
-            // warp starts that half of P V
-            tmem_st32(tS + 0, pkA);
+            // publish P for keys 0-63 (bf16 pairs in S columns 0-31; FP8:
+            // codes in columns 0-15): the MMA warp starts that half of P V
+            if constexpr (F8)
+                tmem_st16(tS + 0, pkA);
+            else
+                tmem_st32(tS + 0, pkA);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.p_lo[t]);
-            // keys 64-127 (S columns 64-95)
-            uint32_t pkB[kHalf / 2];
+            // keys 64-127 (S columns 64-95; FP8: 16-31)
+            uint32_t pkB[F8 ? kHalf / 4 : kHalf / 2];
             uint64_t accB = f2pack(0.f, 0.f);
-            exp_half(sB, sl2, mb, pkB, accB);
-            tmem_st32(tS + kHalf, pkB);
+            exp_any(sB, pkB, accB);
+            if constexpr (F8)
+                tmem_st16(tS + kHalf / 4, pkB);
+            else
+                tmem_st32(tS + kHalf, pkB);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -669,7 +746,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                 m_ref = m_new;
             }
         }
-        const float inv_l = (l > 0.f) ? inv_scale_o / l : 0.f;
+        const float inv_l = (l > 0.f) ? inv_scale_o * sv / l : 0.f;
         const size_t orow = ((size_t)(w.tok0 + row) * p.Hq + w.h) * D;
         #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -714,11 +791,12 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
     }
 }
 
-template <int D, bool PAGED, bool DOC>
+template <int D, bool PAGED, bool DOC, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
-    using C = Cfg<D, DOC>;
+    static_assert(!F8 || (D == 128 && !PAGED && !DOC), "FP8: dense batches, d = 128");
+    using C = Cfg<D, DOC, F8>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Shared sh;
     const uint32_t base = smem_u32(smem_raw);
@@ -757,16 +835,17 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (warp < kSoftmaxWarps) {
         regs_increase<kRegsSoftmax>();
-        softmax_wg<D, PAGED, DOC>(p, sh, reinterpret_cast<int *>(sKV + C::kStages * C::kTileBytes));
+        softmax_wg<D, PAGED, DOC, F8>(p, sh,
+                                      reinterpret_cast<int *>(sKV + C::kStages * C::kTileBytes));
     } else {
         regs_decrease<kRegsControl>();
         if (warp == kWarpTma) {
             if constexpr (PAGED)
                 producer_paged<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
             else if (lane_id() == 0)
-                producer<D, DOC>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+                producer<D, DOC, F8>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
         } else if (warp == kWarpMma) {
-            if (lane_id() == 0) mma_issuer<D, PAGED, DOC>(p, sh, sQ, sKV);
+            if (lane_id() == 0) mma_issuer<D, PAGED, DOC, F8>(p, sh, sQ, sKV);
         }
     }
     __syncwarp();
@@ -784,38 +863,25 @@ static_assert(Cfg<128>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 static_assert(Cfg<64>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 static_assert(Cfg<128, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 static_assert(Cfg<64, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
+static_assert(Cfg<128, false, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 
-template <int D, bool PAGED, bool DOC>
+template <int D, bool PAGED, bool DOC, bool F8 = false>
 int launch_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                   const Params &p, long long units, cudaStream_t stream) {
-    using C = Cfg<D, DOC>;
+    using C = Cfg<D, DOC, F8>;
     // Setting the attribute is idempotent and cheap; do it on every call so
     // that any device the caller switches to is covered.
-    if (cudaFuncSetAttribute(prefill_kernel<D, PAGED, DOC>,
+    if (cudaFuncSetAttribute(prefill_kernel<D, PAGED, DOC, F8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return -5;
     const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
-    prefill_kernel<D, PAGED, DOC><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    prefill_kernel<D, PAGED, DOC, F8><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 
-template <int D>
-int launch_d(const PrefillArgs &a, cudaStream_t stream) {
-    alignas(64) CUtensorMap tq, tk, tv;
-    const uint64_t T = (uint64_t)a.total_tokens;
-    // K/V: the packed tokens (dense, varlen), or the cache's num_pages * 16
-    // rows read one 16-row page box at a time (paged)
-    const uint64_t TK = a.paged ? (uint64_t)a.num_pages * kPageRows : T;
-    const uint32_t kv_box = a.paged ? kPageRows : kBlockN;
-    if (encode_tensor_map_3d(&tq, a.q, 2, D, a.Hq, T, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2,
-                             64, 1, kBlockM, 128) ||
-        encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kv_box, 128) ||
-        encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
-                             64, 1, kv_box, 128))
-        return -5;
-    Params p;
+Params make_params(const PrefillArgs &a) {
+    Params p{};
     p.o = a.o;
     p.lse = a.lse;
     p.cu_seqlens = a.cu_seqlens;
@@ -839,6 +905,25 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.max_pages = a.max_pages;
     p.num_pages = a.num_pages;
     p.num_mblocks = (a.max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM);
+    return p;
+}
+
+template <int D>
+int launch_d(const PrefillArgs &a, cudaStream_t stream) {
+    alignas(64) CUtensorMap tq, tk, tv;
+    const uint64_t T = (uint64_t)a.total_tokens;
+    // K/V: the packed tokens (dense, varlen), or the cache's num_pages * 16
+    // rows read one 16-row page box at a time (paged)
+    const uint64_t TK = a.paged ? (uint64_t)a.num_pages * kPageRows : T;
+    const uint32_t kv_box = a.paged ? kPageRows : kBlockN;
+    if (encode_tensor_map_3d(&tq, a.q, 2, D, a.Hq, T, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2,
+                             64, 1, kBlockM, 128) ||
+        encode_tensor_map_3d(&tk, a.k, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kv_box, 128) ||
+        encode_tensor_map_3d(&tv, a.v, 2, D, a.Hkv, TK, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2,
+                             64, 1, kv_box, 128))
+        return -5;
+    Params p = make_params(a);
     const long long units = (long long)p.num_mblocks * a.num_seqs * a.Hq;
     if (units <= 0) return 0;
     if (units > (1ll << 30)) return -2;
@@ -848,12 +933,44 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     return launch_kernel<D, false, false>(tq, tk, tv, p, units, stream);
 }
 
+// FP8 operands, dense batches, d = 128: Q and K codes [B*N, H, 128] read in
+// one 128-byte box per row; V^T codes [B, Hkv, 128, vt_stride] read as boxes
+// of 128 keys x 128 rows of d.  Keys past N (the last block's tail) lie past
+// the tensor's extent and arrive as zeros.
+int launch_fp8(const PrefillArgs &a, cudaStream_t stream) {
+    constexpr int D = 128;
+    if (a.d != D || a.cu_seqlens || a.paged || a.doc || a.sinks) return -2;
+    alignas(64) CUtensorMap tq, tk, tv;
+    const uint64_t T = (uint64_t)a.total_tokens;
+    if (encode_tensor_map_3d(&tq, a.q, 1, D, a.Hq, T, D, (uint64_t)a.Hq * D, 128, 1, kBlockM,
+                             128) ||
+        encode_tensor_map_3d(&tk, a.k, 1, D, a.Hkv, T, D, (uint64_t)a.Hkv * D, 128, 1, kBlockN,
+                             128) ||
+        encode_tensor_map_3d(&tv, a.v, 1, (uint64_t)a.seqlen, D, (uint64_t)a.num_seqs * a.Hkv,
+                             (uint64_t)a.vt_stride, (uint64_t)D * a.vt_stride, kBlockN, D, 1, 128))
+        return -5;
+    Params p = make_params(a);
+    p.q_scale = a.q_scale;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.nblk = (a.seqlen + kBlockN - 1) / kBlockN;
+    const long long units = (long long)p.num_mblocks * a.num_seqs * a.Hq;
+    if (units <= 0) return 0;
+    if (units > (1ll << 30)) return -2;
+    p.num_units = (int)units;
+    return launch_kernel<D, false, false, true>(tq, tk, tv, p, units, stream);
+}
+
 }  // namespace prefill_impl
 
 int launch_prefill(const PrefillArgs &a, cudaStream_t stream) {
     if (a.d == 128) return prefill_impl::launch_d<128>(a, stream);
     if (a.d == 64) return prefill_impl::launch_d<64>(a, stream);
     return -2;
+}
+
+int launch_prefill_fp8(const PrefillArgs &a, cudaStream_t stream) {
+    return prefill_impl::launch_fp8(a, stream);
 }
 
 }  // namespace fa

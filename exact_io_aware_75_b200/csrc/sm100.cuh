@@ -306,6 +306,41 @@ __device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
+// The same two MMA forms with kind::f8f6f4: 8-bit E4M3 A and B, fp32
+// accumulate, K = 32 per instruction (32 bytes of each operand row, as for
+// kind::f16).  In TMEM, A holds four 8-bit values per 32-bit column, the
+// lowest byte at the lowest K index.
+__device__ __forceinline__ void mma_ss_lo_f8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %5};\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate),
+          "n"(kDescHiSw128Sbo1024)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_lo_f8(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate),
+          "n"(kDescHiSw128Sbo1024)
+        : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4 with E4M3 A and B (format 0 in bits
+// 7-9 and 10-12), fp32 D, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // TMEM loads/stores, shape 32x32b: thread t of the warp touches TMEM lane
 // (warp's lane quarter base + t); x32 = 32 consecutive 32-bit columns.
 #define FA_R32(a) "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), \
@@ -447,6 +482,18 @@ __device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &r0, fl
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Four fp32 values to E4M3 codes (round to nearest even, saturating at
+// +-448), packed with p0 in bits 0-7 (the lowest K index) up to p3 in 24-31.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(r) : "f"(p0), "f"(p1), "f"(p2), "f"(p3));
     return r;
 }
 

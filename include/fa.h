@@ -294,6 +294,54 @@ int fa_decode_paged_fp8(const void *q, const void *k_cache, const void *v_cache,
                         size_t workspace_bytes, void *stream);
 
 /*
+ * FP8 prefill with incoherent processing ("FlashAttention-3" in samanvya.dev
+ * "Attention Is the Bottleneck", "FlashAttention: same math, different IO":
+ * Q and K multiplied by a random orthogonal Hadamard matrix before FP8
+ * quantisation; "Low precision" in the same post: per-block scales).  Two
+ * calls: fa_fp8_prepare makes the E4M3 operands from bf16 Q, K, V, and
+ * fa_fwd_fp8 runs the attention on them.  Dense batches, d = 128.
+ *
+ * fa_fp8_prepare:
+ *   q [B*N, Hq, 128], k and v [B*N, Hkv, 128] bf16 (token-major, as fa_fwd)
+ *   signs [128] fp32, each +1 or -1 (a random draw the caller makes once and
+ *     keeps), or NULL for no rotation (plain FP8)
+ *   -> q8 [B*N, Hq, 128] and k8 [B*N, Hkv, 128] E4M3 codes of
+ *        Q' = Q diag(signs) H / sqrt(128), K' likewise (H the Sylvester
+ *        Hadamard matrix, entry (i, k) = (-1)^popcount(i & k)), so that
+ *        Q' K'^T = Q K^T;
+ *      q_scale [B, Hq, nblk], k_scale [B, Hkv, nblk] fp32, nblk = ceil(N/128):
+ *        one scale per (batch, head, block of 128 tokens);
+ *      vt8 [B, Hkv, 128, vt_stride] E4M3 codes of V transposed (row c of
+ *        (b, h) holds channel c of keys 0..N-1; vt_stride = N rounded up to a
+ *        multiple of 16; bytes N..vt_stride-1 of each row are not written);
+ *      v_scale [B, Hkv] fp32: one scale per (batch, KV head).
+ *   A scale is the smallest power of two 2^k (k >= -126) with amax / 2^k <=
+ *   448 over its block (1 for an all-zero block); a code is x / scale (exact)
+ *   rounded to the nearest E4M3 value (ties to even), saturated at +-448.  workspace: fa_fp8_workspace_bytes(B, N, Hkv) bytes of device
+ *   memory, 4-byte aligned (scratch; contents need no initialisation).
+ *   Alignment: q, k, v, q8, k8, vt8 and signs 16 bytes; scales 4 bytes.
+ *   Errors: FA_ERR_UNSUPPORTED for d != 128; FA_ERR_WORKSPACE if the
+ *   workspace is missing or small; otherwise as fa_fwd.
+ *
+ * fa_fwd_fp8:
+ *   The outputs of fa_fp8_prepare in; O [B*N, Hq, 128] (bf16 or fp32) and
+ *   LSE [B, Hq, N] out, for softmax(Q'K'^T * scale + mask) V with every
+ *   operand read as code * scale.  P is rounded to E4M3 for the P V product
+ *   (so the result is that of FP8 attention, not bit-close to fa_fwd); the
+ *   softmax statistics stay fp32.  Masks, scale, o_dtype, alignment and
+ *   errors as fa_fwd (q8, k8, vt8: 16 bytes; scales: 4 bytes).
+ */
+size_t fa_fp8_workspace_bytes(int B, int N, int Hkv);
+int fa_fp8_prepare(const void *q, const void *k, const void *v, const float *signs,
+                   void *q8, void *k8, void *vt8, float *q_scale, float *k_scale,
+                   float *v_scale, int B, int N, int Hq, int Hkv, int d, void *workspace,
+                   size_t workspace_bytes, void *stream);
+int fa_fwd_fp8(const void *q8, const void *k8, const void *vt8, const float *q_scale,
+               const float *k_scale, const float *v_scale, void *o, float *lse, int B,
+               int Hq, int Hkv, int N, int d, int causal, int window, float scale,
+               int o_dtype, void *stream);
+
+/*
  * fa_decode_paged without a workspace argument, for callers that cannot
  * allocate device memory: code running under a host framework whose memory
  * pool owns the device and forbids raw cudaMalloc, latency-critical serving

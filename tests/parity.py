@@ -40,3 +40,68 @@ def compare(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
         assert lmx <= TOL_LSE_MAX, f"{what}: max |dLSE| = {lmx:.3e}"
         out["lse_max"] = lmx
     return out
+
+
+# FP8 prefill.  The kernel rounds P (at most 2^8 under the conditional
+# rescale) to E4M3 before P V: relative error at most 2^-4 for P in E4M3's
+# normal range, at most 2^-10 absolute below it (where, for N(0,1)-like
+# scores, the weights are small and the errors random).  Against the oracle on
+# the same codes, element (i, c) of O may therefore differ by
+#   2^-4 * sum_j w_ij |v_jc|   (worst case: every weight rounded the same way)
+# plus the output rounding (bf16: 2^-9 relative, 2^-7 allowed) and 1e-3 for
+# the sub-normal weights.  sum_j w_ij |v_jc| is the oracle's attention with
+# |V| in place of V.  LSE comes from fp32 P: the bf16 tolerance holds.
+FP8_P_REL = 2.0 ** -4
+FP8_OUT_REL = 2.0 ** -7
+FP8_ABS = 1e-3
+
+
+def compare_fp8(o_gpu, o_ref, abs_v_ref, lse_gpu=None, lse_ref=None, what=""):
+    og = to64(o_gpu)
+    assert og.shape == o_ref.shape, (what, og.shape, o_ref.shape)
+    assert np.all(np.isfinite(og)), f"{what}: non-finite output"
+    err = np.abs(og - o_ref)
+    bound = FP8_P_REL * abs_v_ref + FP8_OUT_REL * np.abs(o_ref) + FP8_ABS
+    worst = float((err / bound).max()) if err.size else 0.0
+    assert worst <= 1.0, f"{what}: error {worst:.3f} x the FP8 bound (max |dO| {err.max():.3e})"
+    out = {"o_max": float(err.max()) if err.size else 0.0,
+           "o_mean": float(err.mean()) if err.size else 0.0, "bound_frac": worst}
+    if lse_ref is not None:
+        lg = to64(lse_gpu)
+        assert lg.shape == lse_ref.shape, (what, lg.shape, lse_ref.shape)
+        le = np.abs(lg - lse_ref)
+        assert float(le.max()) <= TOL_LSE_MAX, f"{what}: max |dLSE| = {le.max():.3e}"
+        out["lse_max"] = float(le.max())
+    return out
+
+
+def e4m3_table():
+    """Values of all 256 E4M3 codes (NaN for the two NaN codes), for comparisons."""
+    import oracle
+    return np.array([oracle.e4m3_value(c) for c in range(256)])
+
+
+def compare_codes(gpu, ref, exact, what="", rel_tie=2.0 ** -16, max_frac=1e-3):
+    """E4M3 codes from the GPU against the oracle's.  A code may differ only
+    where the exact pre-rounding value lies within `rel_tie` (relative) of
+    the midpoint between the two codes' values -- fp32 arithmetic on the GPU
+    against fp64 in the oracle may round such a value either way -- and then
+    only to the neighbouring code."""
+    g = np.asarray(gpu, dtype=np.uint8)
+    r = np.asarray(ref, dtype=np.uint8)
+    assert g.shape == r.shape, (what, g.shape, r.shape)
+    diff = g != r
+    n = int(diff.sum())
+    if n == 0:
+        return 0
+    assert n <= max_frac * g.size + 1, f"{what}: {n} of {g.size} codes differ"
+    t = e4m3_table()
+    gv, rv, y = t[g[diff]], t[r[diff]], np.asarray(exact, dtype=np.float64)[diff]
+    mid = (gv + rv) / 2.0
+    near = np.abs(y - mid) <= rel_tie * np.maximum(np.abs(y), 2.0 ** -9)
+    # neighbours on the grid: no representable value strictly between them
+    lo, hi = np.minimum(gv, rv), np.maximum(gv, rv)
+    fin = t[np.isfinite(t)]
+    between = np.array([np.any((fin > a) & (fin < b)) for a, b in zip(lo, hi)])
+    assert np.all(near) and not np.any(between), f"{what}: codes differ away from a tie"
+    return n

@@ -228,6 +228,56 @@ def test_fwd_doc_rejects(fa):
     assert lib.fa_fwd_doc(P, P, P, P, 0, P, 0, 2, 2, 128, 64, 1, 0, 0.1, 0, None) == 0
 
 
+def fp8_prep(fa, **kw):
+    a = dict(q=P, k=P, v=P, signs=P, q8=P, k8=P, vt8=P, qs=P, ks=P, vs=P, B=1, N=300, Hq=4,
+             Hkv=2, d=128, ws=P, wsb=1 << 20)
+    a.update(kw)
+    return fa.library().fa_fp8_prepare(a["q"], a["k"], a["v"], a["signs"], a["q8"], a["k8"],
+                                       a["vt8"], a["qs"], a["ks"], a["vs"], a["B"], a["N"],
+                                       a["Hq"], a["Hkv"], a["d"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), -1), (dict(Hkv=0), -1), (dict(d=64), -2), (dict(d=96), -1), (dict(B=-1), -1),
+    (dict(q=0), -1), (dict(vt8=0), -1), (dict(vs=0), -1), (dict(ws=0), -4), (dict(wsb=8), -4),
+    (dict(q=P + 8), -3), (dict(vt8=P + 4), -3), (dict(signs=P + 4), -3), (dict(qs=P + 2), -3),
+    (dict(ws=P + 2), -3)])
+def test_fp8_prepare_rejects(fa, kw, status):
+    assert fp8_prep(fa, **kw) == status
+
+
+def test_fp8_prepare_empty_and_workspace(fa):
+    assert fp8_prep(fa, N=0, q=0) == 0
+    assert fp8_prep(fa, B=0, ws=0) == 0
+    # one fp32 block maximum per (batch, KV head, 128-token block)
+    assert fa.fp8_workspace_bytes(3, 300, 2) == 3 * 2 * 3 * 4
+    assert fa.fp8_workspace_bytes(1, 128, 8) == 8 * 4
+    assert fa.fp8_workspace_bytes(0, 128, 8) == 0
+
+
+def fwd8(fa, **kw):
+    a = dict(q8=P, k8=P, vt8=P, qs=P, ks=P, vs=P, o=P, lse=0, B=1, Hq=4, Hkv=2, N=300, d=128,
+             causal=1, window=0, scale=0.1, od=0)
+    a.update(kw)
+    return fa.library().fa_fwd_fp8(a["q8"], a["k8"], a["vt8"], a["qs"], a["ks"], a["vs"],
+                                   a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                                   a["causal"], a["window"], a["scale"], a["od"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Hq=3), -1), (dict(d=64), -2), (dict(d=96), -2), (dict(window=5, causal=0), -2),
+    (dict(scale=0.0), -1), (dict(od=3), -1), (dict(q8=0), -1), (dict(ks=0), -1),
+    (dict(o=0), -1), (dict(k8=P + 8), -3), (dict(vt8=P + 1), -3), (dict(vs=P + 2), -3),
+    (dict(lse=P + 2), -3), (dict(B=-1), -1)])
+def test_fwd_fp8_rejects(fa, kw, status):
+    assert fwd8(fa, **kw) == status
+
+
+def test_fwd_fp8_empty_is_noop(fa):
+    assert fwd8(fa, B=0, q8=0) == 0
+    assert fwd8(fa, N=0, q8=0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """Importing the binding with the shared library absent raises, rather
     than falling back to anything else."""

@@ -270,6 +270,13 @@ def grad_out(shape, seed=0) -> torch.Tensor:
     return randn_bf16(tuple(shape), g)
 
 
+def hadamard_signs(d: int, seed=0) -> torch.Tensor:
+    """The random +-1 per channel of the FP8 prefill's rotation (fp32 [d]),
+    from a generator of its own seeded with ``seed + 4``."""
+    g = torch.Generator("cpu").manual_seed(seed + 4)
+    return torch.where(torch.rand(d, generator=g) < 0.5, -1.0, 1.0).to(torch.float32)
+
+
 def bf16_bits(t: torch.Tensor):
     """The raw bf16 bit patterns of a CPU bf16 tensor as a numpy uint16 array."""
     import numpy as np
