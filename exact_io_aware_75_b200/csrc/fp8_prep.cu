@@ -121,18 +121,24 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
         sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
     }
     const int n0 = blk * kBlock + warp * kRowsPerWarp;
+    // all 16 row loads in flight before any arithmetic (8 bytes per lane,
+    // 256 contiguous bytes per row)
+    uint2 raw[kRowsPerWarp];
+    #pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i)
+        raw[i] = (n0 + i < a.N) ? __ldg(reinterpret_cast<const uint2 *>(
+                                      src + (((size_t)b * a.N + n0 + i) * H + h) * kD) + lane)
+                                : make_uint2(0u, 0u);
     float x[kRowsPerWarp][4];
     float amax = 0.f;
     #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         const int n = n0 + i;                    // warp-uniform
         if (n < a.N) {
-            const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(
-                src + (((size_t)b * a.N + n) * H + h) * kD) + lane);
-            x[i][0] = bf16_lo(raw.x);
-            x[i][1] = bf16_hi(raw.x);
-            x[i][2] = bf16_lo(raw.y);
-            x[i][3] = bf16_hi(raw.y);
+            x[i][0] = bf16_lo(raw[i].x);
+            x[i][1] = bf16_hi(raw[i].x);
+            x[i][2] = bf16_lo(raw[i].y);
+            x[i][3] = bf16_hi(raw[i].y);
             if (rotate) {
                 #pragma unroll
                 for (int e = 0; e < 4; ++e) x[i][e] *= sg[e];
@@ -173,6 +179,18 @@ fp8_quant_vt_kernel(const Fp8PrepArgs a, int nblk) {
     __shared__ float red[kWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
+    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const int n0 = blk * kBlock;
+    const uint16_t *src = static_cast<const uint16_t *>(a.v);
+    // the block's rows in flight while the (b, h) maximum is reduced
+    uint2 raw[kRowsPerWarp];
+    #pragma unroll
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int n = n0 + warp * kRowsPerWarp + i;
+        raw[i] = (n < a.N) ? __ldg(reinterpret_cast<const uint2 *>(
+                                 src + (((size_t)b * a.N + n) * a.Hkv + h) * kD) + lane)
+                           : make_uint2(0u, 0u);
+    }
     float amax = 0.f;
     for (int i = threadIdx.x; i < nblk; i += kThreads)
         amax = fmaxf(amax, a.v_block_max[(size_t)bh * nblk + i]);
@@ -180,19 +198,11 @@ fp8_quant_vt_kernel(const Fp8PrepArgs a, int nblk) {
     const int kexp = amax > 0.f ? scale_exp(amax) : 0;
     const float inv = ldexpf(1.f, -kexp);
     if (threadIdx.x == 0 && blk == 0) a.v_scale[bh] = ldexpf(1.f, kexp);
-    const int b = bh / a.Hkv, h = bh % a.Hkv;
-    const int n0 = blk * kBlock;
-    const uint16_t *src = static_cast<const uint16_t *>(a.v);
-    #pragma unroll 4
+    #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int nl = warp * kRowsPerWarp + i, n = n0 + nl;
-        uint32_t w = 0;
-        if (n < a.N) {
-            const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(
-                src + (((size_t)b * a.N + n) * a.Hkv + h) * kD) + lane);
-            w = pack_e4m3x4(bf16_lo(raw.x) * inv, bf16_hi(raw.x) * inv, bf16_lo(raw.y) * inv,
-                            bf16_hi(raw.y) * inv);
-        }
+        const int nl = warp * kRowsPerWarp + i;
+        const uint32_t w = pack_e4m3x4(bf16_lo(raw[i].x) * inv, bf16_hi(raw[i].x) * inv,
+                                       bf16_lo(raw[i].y) * inv, bf16_hi(raw[i].y) * inv);
         #pragma unroll
         for (int e = 0; e < 4; ++e) sT[4 * lane + e][nl] = (uint8_t)(w >> (8 * e));
     }

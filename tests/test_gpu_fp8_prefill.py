@@ -18,7 +18,7 @@ import torch
 
 import oracle
 import workloads
-from parity import compare_codes, compare_fp8, to64
+from parity import code_flip_score_bound, compare_codes, compare_fp8, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -119,19 +119,35 @@ def test_fwd_fp8_on_oracle_codes(fa, B, N, Hq, Hkv, causal, window, out_dtype):
     compare_fp8(o, o_ref, a_ref, lse, lse_ref, f"fp8 N={N} causal={causal} W={window}")
 
 
-def test_fp8_end_to_end(fa):
-    """fa_fp8_prepare then fa_fwd_fp8 against the oracle's whole FP8 prefill."""
+@pytest.mark.parametrize("rot", [False, True])
+def test_fp8_end_to_end(fa, rot):
+    """fa_fp8_prepare then fa_fwd_fp8 against the oracle's whole FP8 prefill.
+    Without the rotation the GPU's codes are the oracle's, bit for bit; with
+    it a code may differ at a rounding tie (test_prepare_matches_oracle), and
+    the tolerance widens by the score shift those codes can cause."""
     B, N, Hq, Hkv = 1, 700, 8, 2
     q, k, v = inputs(B, N, Hq, Hkv, seed=71)
-    s = signs(128, 72)
-    o_ref, lse_ref, p = oracle.fp8_prefill(q, k, v, s, causal=True)
+    s = signs(128, 72) if rot else None
+    scale = 1.0 / math.sqrt(128)
+    o_ref, lse_ref, p = oracle.fp8_prefill(q, k, v, s, causal=True, scale=scale)
     a_ref, _ = oracle.attn_fp8(p["q8"], p["q_scale"], p["k8"], p["k_scale"], abs_v(p),
-                               p["v_scale"], True, 0)
-    prep = fa.fp8_prepare(q.cuda(), k.cuda(), v.cuda(), torch.tensor(s, dtype=torch.float32).cuda())
-    o, lse = fa.fwd_fp8(prep, True, 0)
+                               p["v_scale"], True, 0, scale)
+    sg = torch.tensor(s, dtype=torch.float32).cuda() if rot else None
+    prep = fa.fp8_prepare(q.cuda(), k.cuda(), v.cuda(), sg)
+    o, lse = fa.fwd_fp8(prep, True, 0, scale)
     torch.cuda.synchronize()
     assert fa.check_device_error() == 0
-    compare_fp8(o, o_ref, a_ref, lse, lse_ref, "fp8 end to end")
+    q8, k8 = prep["q8"].cpu().numpy(), prep["k8"].cpu().numpy()
+    if not rot:
+        assert np.array_equal(q8, p["q8"]) and np.array_equal(k8, p["k8"])
+        compare_fp8(o, o_ref, a_ref, lse, lse_ref, "fp8 end to end")
+        return
+    assert (q8 != p["q8"]).mean() <= 1e-3 and (k8 != p["k8"]).mean() <= 1e-3
+    ds = code_flip_score_bound(q8, p["q8"], p["q_scale"], k8, p["k8"], p["k_scale"], scale,
+                               True, 0)
+    vmax = float(np.abs(np.array([oracle.e4m3_value(c) for c in range(256)])[p["v8"]]).max()
+                 * p["v_scale"].max())
+    compare_fp8(o, o_ref, a_ref, lse, lse_ref, "fp8 end to end, rotated", ds=ds, vmax=vmax)
 
 
 def test_rotation_lowers_gpu_error_with_outliers(fa):
@@ -150,15 +166,26 @@ def test_rotation_lowers_gpu_error_with_outliers(fa):
     assert errs[1] * 2.0 < errs[0], errs
 
 
-def test_fp8_gqa4k_sampled_rows(fa):
+def test_fp8_gqa4k_full_size(fa):
     """The benchmark's shape (B=1, Hq=32, Hkv=8, N=4096, d=128, causal) in the
-    benchmark's launch: all outputs finite, sampled rows against the oracle."""
+    benchmark's launch: fa_fp8_prepare's scales and codes against the
+    oracle's in full, fa_fwd_fp8 on the oracle's codes on sampled rows."""
     inp = workloads.make("gqa4k", seed=0)
-    s = signs(128, 0)
-    p = oracle.fp8_prepare(inp.q, inp.k, inp.v, s)
-    prep = fa.fp8_prepare(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(),
-                          torch.tensor(s, dtype=torch.float32).cuda())
-    o, lse = fa.fwd_fp8(prep, True, 0, inp.scale)
+    s = workloads.hadamard_signs(128, seed=0)
+    p = oracle.fp8_prepare(inp.q, inp.k, inp.v, s.numpy().astype(np.float64))
+    prep = fa.fp8_prepare(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), s.cuda())
+    torch.cuda.synchronize()
+    assert fa.check_device_error() == 0
+    N = inp.q.shape[1]
+    for name, x in (("q", inp.q), ("k", inp.k)):
+        assert np.array_equal(prep[name + "_scale"].cpu().numpy(), p[name + "_scale"]), name
+        sc = np.repeat(p[name + "_scale"].transpose(0, 2, 1), 128, axis=1)[:, :N, :, None]
+        compare_codes(prep[name + "8"].cpu().numpy(), p[name + "8"],
+                      oracle.hadamard_rotate(x, s.numpy().astype(np.float64)) / sc,
+                      f"gqa4k {name} codes")
+    assert np.array_equal(prep["v_scale"].cpu().numpy(), p["v_scale"])
+    assert np.array_equal(prep["vt8"].cpu().numpy()[..., :N].transpose(0, 3, 1, 2), p["v8"])
+    o, lse = fa.fwd_fp8(to_device_prep(p, N), True, 0, inp.scale)
     torch.cuda.synchronize()
     assert fa.check_device_error() == 0
     assert torch.isfinite(o.float()).all()
