@@ -16,19 +16,21 @@
 //   product and the code -- nearest E4M3 value, ties to even, saturating --
 //   is decided on the exact value.
 //
-// How: HBM-bound elementwise work, two launches.
+// How: HBM-bound work in three launches.
+//   * fp8_rot_kernel (with a rotation): Q and K blocks on the tensor core, see
+//     its comment.
 //   * fp8_quant_qk_kernel: one CTA per (tensor, batch, head, block) of 128
 //     tokens x 128 channels.  A warp holds 16 rows, four channels per lane
-//     (8-byte coalesced loads), rotates each row with an in-warp fast
-//     Walsh-Hadamard transform (two butterfly levels in registers, five by
-//     lane shuffles), reduces the block maximum, and writes the codes (128
-//     contiguous bytes per row) and the scale.  V blocks only record their
-//     maximum.
+//     (8-byte coalesced loads, all in flight at once), reduces the block
+//     maximum, and writes the codes (128 contiguous bytes per row) and the
+//     scale: Q and K without a rotation.  V blocks only record their maximum.
 //   * fp8_quant_vt_kernel: one CTA per V block: the (batch, KV head) maximum
-//     over its blocks, the codes, and a transpose through shared memory into
-//     the [B, Hkv, d, vt_stride] layout whose rows of keys the attention
-//     kernel reads as the K-major operand of P V.
+//     over its blocks, the codes, and a transpose (32-bit words through
+//     shared memory, 4 x 4 bytes in registers) into the [B, Hkv, d,
+//     vt_stride] layout whose rows of keys the attention kernel reads as the
+//     K-major operand of P V.
 #include <climits>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fa_internal.h"
@@ -44,28 +46,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kRowsPerWarp = kBlock / kWarps;  // 16
 constexpr float kInvSqrtD = 0.08838834764831845f;   // 1 / sqrt(128)
-
-// H x for one 128-vector held as x[e] = element 4 * lane + e: butterflies
-// (a, b) -> (a + b, a - b) over index bits 0-1 in registers and bits 2-6
-// across lanes.  H is the Sylvester Hadamard matrix, (i, k) entry
-// (-1)^popcount(i & k).
-__device__ __forceinline__ void fwht128(float (&x)[4], int lane) {
-    const float a0 = x[0] + x[1], a1 = x[0] - x[1];
-    const float a2 = x[2] + x[3], a3 = x[2] - x[3];
-    x[0] = a0 + a2;
-    x[2] = a0 - a2;
-    x[1] = a1 + a3;
-    x[3] = a1 - a3;
-    #pragma unroll
-    for (int m = 1; m < 32; m <<= 1) {
-        const bool upper = (lane & m) != 0;
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float p = __shfl_xor_sync(0xffffffffu, x[e], m);
-            x[e] = upper ? p - x[e] : x[e] + p;
-        }
-    }
-}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -90,14 +70,15 @@ __device__ __forceinline__ float block_max(float v, float *red) {
     return r;
 }
 
-// Q and K blocks: rotate, scale, quantise.  V blocks: their maximum only.
-// blockIdx.x runs over the Q blocks, then K, then V, each (b, h, blk) with
-// blk fastest.
+// Without a rotation: Q and K blocks scaled and quantised; V blocks: their
+// maximum only.  blockIdx.x + first runs over the Q blocks, then K, then V,
+// each (b, h, blk) with blk fastest.  (With a rotation, Q and K go to
+// fp8_rot_kernel and this kernel takes the V blocks only.)
 __global__ void __launch_bounds__(kThreads)
-fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
+fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk, int first) {
     __shared__ float red[kWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int idx = blockIdx.x;
+    int idx = blockIdx.x + first;
     const int nq = a.B * a.Hq * nblk, nk = a.B * a.Hkv * nblk;
     int which, H;
     if (idx < nq) {
@@ -114,12 +95,6 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
     }
     const int blk = idx % nblk, h = (idx / nblk) % H, b = idx / (nblk * H);
     const uint16_t *src = static_cast<const uint16_t *>(which == 0 ? a.q : which == 1 ? a.k : a.v);
-    const bool rotate = which < 2 && a.signs != nullptr;
-    float sg[4] = {1.f, 1.f, 1.f, 1.f};
-    if (rotate) {
-        const float4 s4 = __ldg(reinterpret_cast<const float4 *>(a.signs) + lane);
-        sg[0] = s4.x; sg[1] = s4.y; sg[2] = s4.z; sg[3] = s4.w;
-    }
     const int n0 = blk * kBlock + warp * kRowsPerWarp;
     // all 16 row loads in flight before any arithmetic (8 bytes per lane,
     // 256 contiguous bytes per row)
@@ -132,24 +107,11 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
     float x[kRowsPerWarp][4];
     float amax = 0.f;
     #pragma unroll
-    for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int n = n0 + i;                    // warp-uniform
-        if (n < a.N) {
-            x[i][0] = bf16_lo(raw[i].x);
-            x[i][1] = bf16_hi(raw[i].x);
-            x[i][2] = bf16_lo(raw[i].y);
-            x[i][3] = bf16_hi(raw[i].y);
-            if (rotate) {
-                #pragma unroll
-                for (int e = 0; e < 4; ++e) x[i][e] *= sg[e];
-                fwht128(x[i], lane);
-                #pragma unroll
-                for (int e = 0; e < 4; ++e) x[i][e] *= kInvSqrtD;
-            }
-        } else {
-            #pragma unroll
-            for (int e = 0; e < 4; ++e) x[i][e] = 0.f;
-        }
+    for (int i = 0; i < kRowsPerWarp; ++i) {              // rows past N are zeros
+        x[i][0] = bf16_lo(raw[i].x);
+        x[i][1] = bf16_hi(raw[i].x);
+        x[i][2] = bf16_lo(raw[i].y);
+        x[i][3] = bf16_hi(raw[i].y);
         #pragma unroll
         for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
     }
@@ -159,7 +121,7 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
         return;
     }
     const int kexp = amax > 0.f ? scale_exp(amax) : 0;
-    const float inv = ldexpf(1.f, -kexp);
+    const float mult = ldexpf(1.f, -kexp);
     if (threadIdx.x == 0) (which == 0 ? a.q_scale : a.k_scale)[idx] = ldexpf(1.f, kexp);
     uint8_t *dst = static_cast<uint8_t *>(which == 0 ? a.q8 : a.k8);
     #pragma unroll
@@ -167,15 +129,215 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
         const int n = n0 + i;
         if (n < a.N)
             reinterpret_cast<uint32_t *>(dst + (((size_t)b * a.N + n) * H + h) * kD)[lane] =
-                pack_e4m3x4(x[i][0] * inv, x[i][1] * inv, x[i][2] * inv, x[i][3] * inv);
+                pack_e4m3x4(x[i][0] * mult, x[i][1] * mult, x[i][2] * mult, x[i][3] * mult);
     }
 }
 
+// ------------------------------------------------ rotation on the tensor core
+// Q' = Q diag(signs) H is a dense 128 x 128 contraction per token: each
+// 128-token block of one head is one M = N = K = 128 bf16 MMA against the
+// +-1 matrix B[c][k] = signs[k] (-1)^popcount(k & c), which the CTA writes
+// once into shared memory in the 128-byte-swizzled K-major layout a TMA tile
+// has.  Persistent CTAs of 128 threads (two per SM): thread 0 keeps the TMA
+// loads two blocks ahead in a double buffer and issues the MMAs into two TMEM
+// buffers; every thread owns one token row of the accumulator for the
+// epilogue (block maximum, power-of-two scale, E4M3 codes, 128-byte row
+// stores).  fp32 accumulation of +-x terms: within a few ulp of the exact
+// sums.
+constexpr int kRotThreads = 128;
+constexpr int kRotTile = kBlock * kD * 2;          // one bf16 block: 32 KiB
+constexpr int kRotBox = kBlock * 128;              // 128 rows x 64 bf16
+constexpr int kRotSmem = 3 * kRotTile + 1024;      // B, two A buffers, alignment slack
+constexpr uint32_t kRotTmemCols = 256;             // two 128-column accumulators
+
+struct RotShared {
+    uint64_t a_full[2], mma_done[2], drain;
+    uint32_t tmem_base;
+    int abort;
+    float red[kRotThreads / 32];
+    float sgn[kD];
+};
+
+__global__ void __launch_bounds__(kRotThreads, 2)
+fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const Fp8PrepArgs a, int nblk) {
+    extern __shared__ uint8_t rot_smem_raw[];
+    __shared__ RotShared sh;
+    const uint32_t base = smem_u32(rot_smem_raw);
+    uint8_t *smem = rot_smem_raw + ((1024 - (base & 1023)) & 1023);
+    uint8_t *sB = smem;
+    uint8_t *sA = smem + kRotTile;                 // buffer j at sA + j * kRotTile
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nq = a.B * a.Hq * nblk;
+    const int units = nq + a.B * a.Hkv * nblk;
+    int my_units = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) ++my_units;
+    volatile int *abort = &sh.abort;
+
+    if (tid == 0) {
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&sh.a_full[j], 1);
+            mbar_init(&sh.mma_done[j], 1);
+        }
+        mbar_init(&sh.drain, 1);
+        sh.abort = 0;
+        fence_barrier_init();
+    }
+    sh.sgn[tid] = __ldg(a.signs + tid);
+    if (warp == 0) tmem_alloc(&sh.tmem_base, kRotTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // B: two boxes of 64 k-columns; row c, 16-byte chunk j (k = 64 box + 8 j ..)
+    // at chunk position j ^ (c & 7)
+    for (int ch = tid; ch < 2 * kD * 8; ch += kRotThreads) {
+        const int box = ch >> 10, c = (ch >> 3) & (kD - 1), j = ch & 7;
+        uint32_t w[4];
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int k0 = box * 64 + j * 8 + 2 * e, k1 = k0 + 1;
+            const bool n0 = (sh.sgn[k0] < 0.f) != ((__popc(k0 & c) & 1) != 0);
+            const bool n1 = (sh.sgn[k1] < 0.f) != ((__popc(k1 & c) & 1) != 0);
+            w[e] = (n0 ? 0xBF80u : 0x3F80u) | ((n1 ? 0xBF80u : 0x3F80u) << 16);
+        }
+        *reinterpret_cast<uint4 *>(sB + box * kRotBox + c * 128 + ((j ^ (c & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    const uint32_t tmem = sh.tmem_base;
+    const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
+    const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
+    // unit -> (Q or K, batch, head, block)
+    auto decode = [&](int u, int &which, int &b, int &h, int &blk) {
+        which = u >= nq;
+        const int H = which ? a.Hkv : a.Hq;
+        const int v = which ? u - nq : u;
+        blk = v % nblk;
+        h = (v / nblk) % H;
+        b = v / (nblk * H);
+    };
+    int issued = 0, waited = 0;                    // TMA loads (thread 0)
+    auto load = [&](int it) {
+        const int buf = it & 1;
+        int which, b, h, blk;
+        decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        mbar_arrive_expect_tx(&sh.a_full[buf], kRotTile);
+        for (int bx = 0; bx < 2; ++bx)
+            tma_load_3d(sA + buf * kRotTile + bx * kRotBox, which ? &tmK : &tmQ, &sh.a_full[buf],
+                        bx * 64, h, b * a.N + blk * kBlock);
+        ++issued;
+    };
+    auto mma = [&](int it) -> bool {
+        const int buf = it & 1;
+        if (!mbar_wait(&sh.a_full[buf], (it >> 1) & 1, abort)) return false;
+        ++waited;
+        tc_fence_after();
+        const uint32_t aa = a_lo + buf * (kRotTile >> 4);
+        #pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
+            mma_ss_lo(tmem + buf * kD, aa + off, b_lo + off, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(&sh.mma_done[buf]);
+        return true;
+    };
+    bool ok = true;
+    if (tid == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        if (my_units > 0) load(0);
+        if (my_units > 1) load(1);
+        if (my_units > 0) ok = mma(0);
+    }
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int it = 0; it < my_units; ++it) {
+        const int buf = it & 1;
+        // unit it's accumulator is ready and its A buffer free
+        ok = ok && mbar_wait(&sh.mma_done[buf], (it >> 1) & 1, abort);
+        if (tid == 0 && ok) {
+            if (it + 2 < my_units) load(it + 2);
+            if (it + 1 < my_units) ok = mma(it + 1);
+        }
+        tc_fence_after();
+        int which, b, h, blk;
+        decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        const int n = blk * kBlock + tid;          // this thread's token (rows past N: the
+        const bool valid = n < a.N;                // next batch or zeros -- left out)
+        float m = 0.f;
+        if (ok) {
+            #pragma unroll
+            for (int q = 0; q < kD / 32; ++q) {
+                uint32_t r[32];
+                tmem_ld32(trow + buf * kD + q * 32, r);
+                tmem_wait_ld();
+                #pragma unroll
+                for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(__uint_as_float(r[e])));
+            }
+        }
+        if (!valid) m = 0.f;
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) sh.red[warp] = m;
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        float amax = sh.red[0];
+        #pragma unroll
+        for (int w = 1; w < kRotThreads / 32; ++w) amax = fmaxf(amax, sh.red[w]);
+        // the accumulator is H diag(signs) x; Q' = that / sqrt(128)
+        const float amax_c = amax * kInvSqrtD;
+        const int kexp = amax_c > 0.f ? scale_exp(amax_c) : 0;
+        const float mult = kInvSqrtD * ldexpf(1.f, -kexp);
+        const int H = which ? a.Hkv : a.Hq;
+        const int sidx = (b * H + h) * nblk + blk;
+        if (tid == 0) (which ? a.k_scale : a.q_scale)[sidx] = ldexpf(1.f, kexp);
+        uint8_t *dst = static_cast<uint8_t *>(which ? a.k8 : a.q8) +
+                       (((size_t)b * a.N + n) * H + h) * kD;
+        #pragma unroll
+        for (int q = 0; q < kD / 32; ++q) {
+            uint32_t r[32];
+            tmem_ld32(trow + buf * kD + q * 32, r);
+            tmem_wait_ld();
+            uint32_t cw[8];
+            #pragma unroll
+            for (int e = 0; e < 8; ++e)
+                cw[e] = pack_e4m3x4(__uint_as_float(r[4 * e]) * mult,
+                                    __uint_as_float(r[4 * e + 1]) * mult,
+                                    __uint_as_float(r[4 * e + 2]) * mult,
+                                    __uint_as_float(r[4 * e + 3]) * mult);
+            if (valid) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + q * 32);
+                d4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                d4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            }
+        }
+        // every row read from this TMEM buffer (and sh.red) before the MMA of
+        // unit it + 2 and the next reduction reuse them
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (tid == 0) {
+        // leave no copy or MMA in flight
+        for (int l = waited; l < issued; ++l) mbar_drain_wait(&sh.a_full[l & 1], (l >> 1) & 1);
+        tc_commit(&sh.drain);
+        mbar_drain_wait(&sh.drain, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kRotTmemCols);
+}
+
 // V codes, transposed: CTA (b * Hkv + h) * nblk + blk writes rows c = 0..127
-// of keys blk * 128 .. + 127 (those below N).
+// of keys blk * 128 .. + 127 (those below N).  The block goes through shared
+// memory as 32-bit words (four channels of one token), column-swizzled by
+// token / 4 so that both phases are free of bank conflicts; each lane then
+// turns a 4 x 4 byte block (four tokens x four channels) around in registers
+// and stores four 4-byte pieces of four V^T rows, a warp 128 bytes per row.
 __global__ void __launch_bounds__(kThreads)
 fp8_quant_vt_kernel(const Fp8PrepArgs a, int nblk) {
-    __shared__ uint8_t sT[kD][kBlock + 1];   // [channel][token]; odd row length: no bank conflicts
+    __shared__ uint32_t sW[kBlock][kD / 4];   // [token][channel group ^ (token / 4)]
     __shared__ float red[kWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
@@ -201,26 +363,34 @@ fp8_quant_vt_kernel(const Fp8PrepArgs a, int nblk) {
     #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         const int nl = warp * kRowsPerWarp + i;
-        const uint32_t w = pack_e4m3x4(bf16_lo(raw[i].x) * inv, bf16_hi(raw[i].x) * inv,
-                                       bf16_lo(raw[i].y) * inv, bf16_hi(raw[i].y) * inv);
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) sT[4 * lane + e][nl] = (uint8_t)(w >> (8 * e));
+        sW[nl][lane ^ ((nl >> 2) & 31)] =
+            pack_e4m3x4(bf16_lo(raw[i].x) * inv, bf16_hi(raw[i].x) * inv,
+                        bf16_lo(raw[i].y) * inv, bf16_hi(raw[i].y) * inv);
     }
     __syncthreads();
     const int nvalid = min(kBlock, a.N - n0);
     uint8_t *dst = static_cast<uint8_t *>(a.vt8) + (size_t)bh * kD * a.vt_stride + n0;
-    const int t0 = 4 * lane;
-    #pragma unroll 4
-    for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int c = warp * kRowsPerWarp + i;
-        uint8_t *row = dst + (size_t)c * a.vt_stride;
-        if (t0 + 4 <= nvalid) {
-            const uint32_t w = (uint32_t)sT[c][t0] | ((uint32_t)sT[c][t0 + 1] << 8) |
-                               ((uint32_t)sT[c][t0 + 2] << 16) | ((uint32_t)sT[c][t0 + 3] << 24);
-            *reinterpret_cast<uint32_t *>(row + t0) = w;
-        } else {
-            for (int e = 0; e < 4; ++e)
-                if (t0 + e < nvalid) row[t0 + e] = sT[c][t0 + e];
+    const int t0 = 4 * lane;                    // tokens t0 .. t0 + 3 of the block
+    #pragma unroll
+    for (int g = 0; g < kD / 4 / kWarps; ++g) {
+        const int cg = warp * (kD / 4 / kWarps) + g;   // channels 4 cg .. 4 cg + 3
+        const int col = cg ^ lane;
+        const uint32_t w0 = sW[t0][col], w1 = sW[t0 + 1][col];
+        const uint32_t w2 = sW[t0 + 2][col], w3 = sW[t0 + 3][col];
+        // byte e of word r = channel 4 cg + e of token t0 + r  ->  o[e]
+        const uint32_t u0 = __byte_perm(w0, w1, 0x5140), u1 = __byte_perm(w0, w1, 0x7362);
+        const uint32_t u2 = __byte_perm(w2, w3, 0x5140), u3 = __byte_perm(w2, w3, 0x7362);
+        const uint32_t o[4] = {__byte_perm(u0, u2, 0x5410), __byte_perm(u0, u2, 0x7632),
+                               __byte_perm(u1, u3, 0x5410), __byte_perm(u1, u3, 0x7632)};
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint8_t *row = dst + (size_t)(4 * cg + e) * a.vt_stride;
+            if (t0 + 4 <= nvalid) {
+                *reinterpret_cast<uint32_t *>(row + t0) = o[e];
+            } else {
+                for (int k = 0; k < 4; ++k)
+                    if (t0 + k < nvalid) row[t0 + k] = (uint8_t)(o[e] >> (8 * k));
+            }
         }
     }
 }
@@ -231,12 +401,30 @@ int launch_fp8_prepare(const Fp8PrepArgs &a, cudaStream_t stream) {
     using namespace fp8_impl;
     if (a.d != kD) return -2;
     const long long nblk = (a.N + kBlock - 1) / kBlock;
-    const long long grid_a = (long long)a.B * (a.Hq + 2 * a.Hkv) * nblk;
-    const long long grid_b = (long long)a.B * a.Hkv * nblk;
-    if (grid_a <= 0) return 0;
-    if (grid_a > INT_MAX) return -2;
-    fp8_quant_qk_kernel<<<(int)grid_a, kThreads, 0, stream>>>(a, (int)nblk);
-    fp8_quant_vt_kernel<<<(int)grid_b, kThreads, 0, stream>>>(a, (int)nblk);
+    const long long nq = (long long)a.B * a.Hq * nblk, nkv = (long long)a.B * a.Hkv * nblk;
+    if (nq <= 0) return 0;
+    if (nq + 2 * nkv > INT_MAX) return -2;
+    if (a.signs) {
+        // Q and K on the tensor core, then V's block maxima
+        alignas(64) CUtensorMap tq, tk;
+        const uint64_t T = (uint64_t)a.B * a.N;
+        if (encode_tensor_map_3d(&tq, a.q, 2, kD, a.Hq, T, (uint64_t)kD * 2,
+                                 (uint64_t)a.Hq * kD * 2, 64, 1, kBlock, 128) ||
+            encode_tensor_map_3d(&tk, a.k, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
+                                 (uint64_t)a.Hkv * kD * 2, 64, 1, kBlock, 128))
+            return -5;
+        if (cudaFuncSetAttribute(fp8_rot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kRotSmem) != cudaSuccess)
+            return -5;
+        const long long units = nq + nkv;
+        const long long cap = 2ll * device_sm_count();
+        const int grid = (int)(units < cap ? units : cap);
+        fp8_rot_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(tq, tk, a, (int)nblk);
+        fp8_quant_qk_kernel<<<(int)nkv, kThreads, 0, stream>>>(a, (int)nblk, (int)(nq + nkv));
+    } else {
+        fp8_quant_qk_kernel<<<(int)(nq + 2 * nkv), kThreads, 0, stream>>>(a, (int)nblk, 0);
+    }
+    fp8_quant_vt_kernel<<<(int)nkv, kThreads, 0, stream>>>(a, (int)nblk);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 

@@ -64,6 +64,11 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #endif
 // One score pair in kPolyPeriod takes the FMA-pipe exponential (0 = none).
 constexpr int kPolyPeriod = FA_POLY_PERIOD;
+#ifndef FA_POLY_F8
+#define FA_POLY_F8 0
+#endif
+// FP8 kernel: one group of four scores in kPolyPeriodF8 takes it (0 = none).
+constexpr int kPolyPeriodF8 = FA_POLY_F8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPageRows = 16;                 // tokens per cache page (paged mode)
 constexpr int kPagesPerTile = 128 / kPageRows;
@@ -537,7 +542,16 @@ __device__ __forceinline__ void exp_half_f8(const float (&v)[kHalf], float sl2, 
         float x0, x1, y0, y1;
         f2unpack(x, x0, x1);
         f2unpack(y, y0, y1);
-        const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(y0), p3 = ex2(y1);
+        float p0, p1, p2, p3;
+        if (kPolyPeriodF8 > 0 && (c % kPolyPeriodF8) == kPolyPeriodF8 - 1) {
+            exp2_poly_pair(x0, x1, p0, p1);
+            exp2_poly_pair(y0, y1, p2, p3);
+        } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+            p2 = ex2(y0);
+            p3 = ex2(y1);
+        }
         a2[0] = f2add(a2[0], f2pack(p0, p1));
         a2[1] = f2add(a2[1], f2pack(p2, p3));
         pk[c] = pack_e4m3x4(p0, p1, p2, p3);
