@@ -188,6 +188,33 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // unit -> (Q or K, batch, head, block)
+    auto decode = [&](int u, int &which, int &b, int &h, int &blk) {
+        which = u >= nq;
+        const int H = which ? a.Hkv : a.Hq;
+        const int v = which ? u - nq : u;
+        blk = v % nblk;
+        h = (v / nblk) % H;
+        b = v / (nblk * H);
+    };
+    int issued = 0, waited = 0;                    // TMA loads (thread 0)
+    auto load = [&](int it) {
+        const int buf = it & 1;
+        int which, b, h, blk;
+        decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        mbar_arrive_expect_tx(&sh.a_full[buf], kRotTile);
+        for (int bx = 0; bx < 2; ++bx)
+            tma_load_3d(sA + buf * kRotTile + bx * kRotBox, which ? &tmK : &tmQ, &sh.a_full[buf],
+                        bx * 64, h, b * a.N + blk * kBlock);
+        ++issued;
+    };
+    // the first two blocks' loads run while B is written
+    if (tid == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        if (my_units > 0) load(0);
+        if (my_units > 1) load(1);
+    }
     // B: two boxes of 64 k-columns; row c, 16-byte chunk j (k = 64 box + 8 j ..)
     // at chunk position j ^ (c & 7)
     for (int ch = tid; ch < 2 * kD * 8; ch += kRotThreads) {
@@ -209,26 +236,6 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tmem = sh.tmem_base;
     const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
     const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
-    // unit -> (Q or K, batch, head, block)
-    auto decode = [&](int u, int &which, int &b, int &h, int &blk) {
-        which = u >= nq;
-        const int H = which ? a.Hkv : a.Hq;
-        const int v = which ? u - nq : u;
-        blk = v % nblk;
-        h = (v / nblk) % H;
-        b = v / (nblk * H);
-    };
-    int issued = 0, waited = 0;                    // TMA loads (thread 0)
-    auto load = [&](int it) {
-        const int buf = it & 1;
-        int which, b, h, blk;
-        decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
-        mbar_arrive_expect_tx(&sh.a_full[buf], kRotTile);
-        for (int bx = 0; bx < 2; ++bx)
-            tma_load_3d(sA + buf * kRotTile + bx * kRotBox, which ? &tmK : &tmQ, &sh.a_full[buf],
-                        bx * 64, h, b * a.N + blk * kBlock);
-        ++issued;
-    };
     auto mma = [&](int it) -> bool {
         const int buf = it & 1;
         if (!mbar_wait(&sh.a_full[buf], (it >> 1) & 1, abort)) return false;
@@ -244,13 +251,7 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         return true;
     };
     bool ok = true;
-    if (tid == 0) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-        if (my_units > 0) load(0);
-        if (my_units > 1) load(1);
-        if (my_units > 0) ok = mma(0);
-    }
+    if (tid == 0 && my_units > 0) ok = mma(0);
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     for (int it = 0; it < my_units; ++it) {
         const int buf = it & 1;
