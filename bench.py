@@ -511,7 +511,7 @@ def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, 
     bflops = 2.5 * flops
     ach = bflops / (ms * 1e-3) / 1e12
     out["bwd"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
-                  "flop_per_call": bflops, "launches_per_call": 3,
+                  "flop_per_call": bflops, "launches_per_call": 2,
                   "workload": "backward of the prefill workload (dQ, dK, dV), causal",
                   "roofline": {"bound": "tensor", "achieved": round(ach, 2),
                                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -542,7 +542,7 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
         "flop_per_call": flops, "launches_per_call": 1,
         "with_prepare": {"value": round(flops / ((ms + ms_prep) * 1e-3) / 1e12, 2),
                          "unit": "TFLOP/s", "ms_per_call": round(ms + ms_prep, 4),
-                         "launches_per_call": 4},
+                         "launches_per_call": 3},
         "workload": "FP8 prefill of the prefill workload: Q, K rotated by a random-sign "
                     "Hadamard matrix, E4M3 with 128-token block scales (V per head), causal",
         "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak8, 1),
@@ -551,12 +551,11 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
                      "kernel": "prefill_kernel<128> (FP8 mode)",
                      "traffic": traffic_all.get("prefill_fp8_gqa4k")},
         "prepare": {"ms_per_call": round(ms_prep, 4), "bytes_per_call": prep_bytes,
-                    "launches_per_call": 3,
+                    "launches_per_call": 2,
                     "roofline": {"bound": "hbm", "achieved": round(prep_gbs, 1),
                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
                                  "frac": round(prep_gbs / pk["hbm_gbs"], 4),
-                                 "kernel": "fp8_rot_kernel + fp8_quant_qk_kernel (V maxima) "
-                                           "+ fp8_quant_vt_kernel",
+                                 "kernel": "fp8_rot_kernel + fp8_quant_vt_kernel",
                                  "traffic": traffic_all.get("fp8_prepare_gqa4k")}}}
     del prep, ws
 

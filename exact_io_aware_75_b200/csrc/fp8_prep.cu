@@ -16,9 +16,9 @@
 //   product and the code -- nearest E4M3 value, ties to even, saturating --
 //   is decided on the exact value.
 //
-// How: HBM-bound work in three launches.
-//   * fp8_rot_kernel (with a rotation): Q and K blocks on the tensor core, see
-//     its comment.
+// How: HBM-bound work in two launches.
+//   * fp8_rot_kernel (with a rotation): Q and K blocks on the tensor core and
+//     V's block maxima, see its comment.
 //   * fp8_quant_qk_kernel: one CTA per (tensor, batch, head, block) of 128
 //     tokens x 128 channels.  A warp holds 16 rows, four channels per lane
 //     (8-byte coalesced loads, all in flight at once), reduces the block
@@ -71,14 +71,14 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 // Without a rotation: Q and K blocks scaled and quantised; V blocks: their
-// maximum only.  blockIdx.x + first runs over the Q blocks, then K, then V,
-// each (b, h, blk) with blk fastest.  (With a rotation, Q and K go to
-// fp8_rot_kernel and this kernel takes the V blocks only.)
+// maximum only.  blockIdx.x runs over the Q blocks, then K, then V, each
+// (b, h, blk) with blk fastest.  (With a rotation, fp8_rot_kernel does all of
+// this.)
 __global__ void __launch_bounds__(kThreads)
-fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk, int first) {
+fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
     __shared__ float red[kWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int idx = blockIdx.x + first;
+    int idx = blockIdx.x;
     const int nq = a.B * a.Hq * nblk, nk = a.B * a.Hkv * nblk;
     int which, H;
     if (idx < nq) {
@@ -138,82 +138,87 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk, int first) {
 // 128-token block of one head is one M = N = K = 128 bf16 MMA against the
 // +-1 matrix B[c][k] = signs[k] (-1)^popcount(k & c), which the CTA writes
 // once into shared memory in the 128-byte-swizzled K-major layout a TMA tile
-// has.  Persistent CTAs of 128 threads (two per SM): thread 0 keeps the TMA
-// loads two blocks ahead in a double buffer and issues the MMAs into two TMEM
-// buffers; every thread owns one token row of the accumulator for the
-// epilogue (block maximum, power-of-two scale, E4M3 codes, 128-byte row
-// stores).  fp32 accumulation of +-x terms: within a few ulp of the exact
-// sums.
-constexpr int kRotThreads = 128;
+// has.  One persistent CTA per SM, 8 warps: thread 0 keeps TMA loads up to
+// four blocks ahead and issues each block's MMA one block ahead into one of
+// two TMEM accumulators; every thread owns half a token row (64 channels;
+// warps w and w + 4 share TMEM lanes 32 (w % 4) ..) for the epilogue: block
+// maximum, power-of-two scale, E4M3 codes, 64-byte stores.  The same CTAs
+// take V's blocks after their Q and K blocks, reading the tile from shared
+// memory for its maximum only.  fp32 accumulation of +-x terms: within a few
+// ulp of the exact sums.
+constexpr int kRotThreads = 256;
+constexpr int kRotWarps = kRotThreads / 32;
+constexpr int kRotStages = 4;
 constexpr int kRotTile = kBlock * kD * 2;          // one bf16 block: 32 KiB
 constexpr int kRotBox = kBlock * 128;              // 128 rows x 64 bf16
-constexpr int kRotSmem = 3 * kRotTile + 1024;      // B, two A buffers, alignment slack
+constexpr int kRotSmem = (1 + kRotStages) * kRotTile + 1024;   // B, A ring, alignment
 constexpr uint32_t kRotTmemCols = 256;             // two 128-column accumulators
 
 struct RotShared {
-    uint64_t a_full[2], mma_done[2], drain;
+    uint64_t a_full[kRotStages], mma_done[2], drain;
     uint32_t tmem_base;
     int abort;
-    float red[kRotThreads / 32];
+    float red[kRotWarps];
     float sgn[kD];
 };
 
-__global__ void __launch_bounds__(kRotThreads, 2)
+__global__ void __launch_bounds__(kRotThreads, 1)
 fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const Fp8PrepArgs a, int nblk) {
+               const __grid_constant__ CUtensorMap tmV, const Fp8PrepArgs a, int nblk) {
     extern __shared__ uint8_t rot_smem_raw[];
     __shared__ RotShared sh;
     const uint32_t base = smem_u32(rot_smem_raw);
     uint8_t *smem = rot_smem_raw + ((1024 - (base & 1023)) & 1023);
     uint8_t *sB = smem;
-    uint8_t *sA = smem + kRotTile;                 // buffer j at sA + j * kRotTile
+    uint8_t *sA = smem + kRotTile;                 // stage j at sA + j * kRotTile
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nq = a.B * a.Hq * nblk;
-    const int units = nq + a.B * a.Hkv * nblk;
+    const int row = (warp & 3) * 32 + lane;        // token row of the block
+    const int half = warp >> 2;                    // channels 64 half .. + 63
+    const int nq = a.B * a.Hq * nblk, nkv = a.B * a.Hkv * nblk;
+    const int units = nq + 2 * nkv;                // Q blocks, K blocks, V blocks
     int my_units = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) ++my_units;
     volatile int *abort = &sh.abort;
 
     if (tid == 0) {
-        for (int j = 0; j < 2; ++j) {
-            mbar_init(&sh.a_full[j], 1);
-            mbar_init(&sh.mma_done[j], 1);
-        }
+        for (int j = 0; j < kRotStages; ++j) mbar_init(&sh.a_full[j], 1);
+        for (int j = 0; j < 2; ++j) mbar_init(&sh.mma_done[j], 1);
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
         fence_barrier_init();
     }
-    sh.sgn[tid] = __ldg(a.signs + tid);
+    if (tid < kD) sh.sgn[tid] = __ldg(a.signs + tid);
     if (warp == 0) tmem_alloc(&sh.tmem_base, kRotTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // unit -> (Q or K, batch, head, block)
+    // unit -> tensor (0 Q, 1 K, 2 V), batch, head, block
     auto decode = [&](int u, int &which, int &b, int &h, int &blk) {
-        which = u >= nq;
+        which = u < nq ? 0 : (u < nq + nkv ? 1 : 2);
         const int H = which ? a.Hkv : a.Hq;
-        const int v = which ? u - nq : u;
+        const int v = u - (which == 0 ? 0 : (which == 1 ? nq : nq + nkv));
         blk = v % nblk;
         h = (v / nblk) % H;
         b = v / (nblk * H);
     };
     int issued = 0, waited = 0;                    // TMA loads (thread 0)
     auto load = [&](int it) {
-        const int buf = it & 1;
+        const int st = it % kRotStages;
         int which, b, h, blk;
         decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
-        mbar_arrive_expect_tx(&sh.a_full[buf], kRotTile);
+        mbar_arrive_expect_tx(&sh.a_full[st], kRotTile);
+        const CUtensorMap *m = which == 0 ? &tmQ : (which == 1 ? &tmK : &tmV);
         for (int bx = 0; bx < 2; ++bx)
-            tma_load_3d(sA + buf * kRotTile + bx * kRotBox, which ? &tmK : &tmQ, &sh.a_full[buf],
-                        bx * 64, h, b * a.N + blk * kBlock);
+            tma_load_3d(sA + st * kRotTile + bx * kRotBox, m, &sh.a_full[st], bx * 64, h,
+                        b * a.N + blk * kBlock);
         ++issued;
     };
-    // the first two blocks' loads run while B is written
+    // loads of the first blocks run while B is written
     if (tid == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
-        if (my_units > 0) load(0);
-        if (my_units > 1) load(1);
+        tma_prefetch_desc(&tmV);
+        for (int it = 0; it < my_units && it < kRotStages; ++it) load(it);
     }
     // B: two boxes of 64 k-columns; row c, 16-byte chunk j (k = 64 box + 8 j ..)
     // at chunk position j ^ (c & 7)
@@ -236,48 +241,62 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tmem = sh.tmem_base;
     const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
     const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
-    auto mma = [&](int it) -> bool {
-        const int buf = it & 1;
-        if (!mbar_wait(&sh.a_full[buf], (it >> 1) & 1, abort)) return false;
+    // A CTA's units run in increasing order, Q and K before V, so unit it of
+    // a Q or K block is its it-th MMA: accumulator it & 1.
+    auto is_qk = [&](int it) { return blockIdx.x + it * gridDim.x < nq + nkv; };
+    auto mma = [&](int it) -> bool {               // thread 0
+        const int st = it % kRotStages;
+        if (!mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort)) return false;
         ++waited;
+        if (!is_qk(it)) return true;               // V: read from shared memory
         tc_fence_after();
-        const uint32_t aa = a_lo + buf * (kRotTile >> 4);
+        const uint32_t aa = a_lo + st * (kRotTile >> 4);
         #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
             const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
-            mma_ss_lo(tmem + buf * kD, aa + off, b_lo + off, idesc, ks > 0 ? 1u : 0u);
+            mma_ss_lo(tmem + (it & 1) * kD, aa + off, b_lo + off, idesc, ks > 0 ? 1u : 0u);
         }
-        tc_commit(&sh.mma_done[buf]);
+        tc_commit(&sh.mma_done[it & 1]);
         return true;
     };
     bool ok = true;
     if (tid == 0 && my_units > 0) ok = mma(0);
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
     for (int it = 0; it < my_units; ++it) {
-        const int buf = it & 1;
-        // unit it's accumulator is ready and its A buffer free
-        ok = ok && mbar_wait(&sh.mma_done[buf], (it >> 1) & 1, abort);
-        if (tid == 0 && ok) {
-            if (it + 2 < my_units) load(it + 2);
-            if (it + 1 < my_units) ok = mma(it + 1);
-        }
+        const int st = it % kRotStages;
+        const bool qk = is_qk(it);
+        if (qk)
+            ok = ok && mbar_wait(&sh.mma_done[it & 1], (it >> 1) & 1, abort);
+        else
+            ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
+        if (tid == 0 && ok && it + 1 < my_units) ok = mma(it + 1);
         tc_fence_after();
         int which, b, h, blk;
         decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
-        const int n = blk * kBlock + tid;          // this thread's token (rows past N: the
-        const bool valid = n < a.N;                // next batch or zeros -- left out)
+        const int n = blk * kBlock + row;          // this thread's token (rows past N:
+        const bool valid = n < a.N;                // the next batch or zeros -- left out)
+        float v[64];
         float m = 0.f;
-        if (ok) {
+        if (ok && qk) {
+            tmem_ld32(trow + (it & 1) * kD, reinterpret_cast<uint32_t *>(v));
+            tmem_ld32(trow + (it & 1) * kD + 32, reinterpret_cast<uint32_t *>(v) + 32);
+            tmem_wait_ld();
+        } else if (ok) {
+            // V: this row's 64 bf16 of box `half`, chunks swizzled by row & 7
+            const uint8_t *src = sA + st * kRotTile + half * kRotBox + row * 128;
             #pragma unroll
-            for (int q = 0; q < kD / 32; ++q) {
-                uint32_t r[32];
-                tmem_ld32(trow + buf * kD + q * 32, r);
-                tmem_wait_ld();
-                #pragma unroll
-                for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(__uint_as_float(r[e])));
+            for (int c = 0; c < 8; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) << 4));
+                v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
+                v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
+                v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
+                v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
             }
         }
-        if (!valid) m = 0.f;
+        if (ok && valid) {
+            #pragma unroll
+            for (int e = 0; e < 64; ++e) m = fmaxf(m, fabsf(v[e]));
+        }
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) sh.red[warp] = m;
@@ -285,42 +304,39 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!ok) break;
         float amax = sh.red[0];
         #pragma unroll
-        for (int w = 1; w < kRotThreads / 32; ++w) amax = fmaxf(amax, sh.red[w]);
-        // the accumulator is H diag(signs) x; Q' = that / sqrt(128)
-        const float amax_c = amax * kInvSqrtD;
-        const int kexp = amax_c > 0.f ? scale_exp(amax_c) : 0;
-        const float mult = kInvSqrtD * ldexpf(1.f, -kexp);
-        const int H = which ? a.Hkv : a.Hq;
-        const int sidx = (b * H + h) * nblk + blk;
-        if (tid == 0) (which ? a.k_scale : a.q_scale)[sidx] = ldexpf(1.f, kexp);
-        uint8_t *dst = static_cast<uint8_t *>(which ? a.k8 : a.q8) +
-                       (((size_t)b * a.N + n) * H + h) * kD;
-        #pragma unroll
-        for (int q = 0; q < kD / 32; ++q) {
-            uint32_t r[32];
-            tmem_ld32(trow + buf * kD + q * 32, r);
-            tmem_wait_ld();
-            uint32_t cw[8];
-            #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                cw[e] = pack_e4m3x4(__uint_as_float(r[4 * e]) * mult,
-                                    __uint_as_float(r[4 * e + 1]) * mult,
-                                    __uint_as_float(r[4 * e + 2]) * mult,
-                                    __uint_as_float(r[4 * e + 3]) * mult);
+        for (int w = 1; w < kRotWarps; ++w) amax = fmaxf(amax, sh.red[w]);
+        if (which == 2) {
+            if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
+        } else {
+            // the accumulator is H diag(signs) x; Q' = that / sqrt(128)
+            const float amax_c = amax * kInvSqrtD;
+            const int kexp = amax_c > 0.f ? scale_exp(amax_c) : 0;
+            const float mult = kInvSqrtD * ldexpf(1.f, -kexp);
+            const int H = which ? a.Hkv : a.Hq;
+            if (tid == 0) (which ? a.k_scale : a.q_scale)[(b * H + h) * nblk + blk] = ldexpf(1.f, kexp);
             if (valid) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + q * 32);
-                d4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                d4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                uint32_t cw[16];
+                #pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    cw[e] = pack_e4m3x4(v[4 * e] * mult, v[4 * e + 1] * mult, v[4 * e + 2] * mult,
+                                        v[4 * e + 3] * mult);
+                uint4 *d4 = reinterpret_cast<uint4 *>(
+                    static_cast<uint8_t *>(which ? a.k8 : a.q8) +
+                    (((size_t)b * a.N + n) * H + h) * kD + half * 64);
+                #pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
             }
         }
-        // every row read from this TMEM buffer (and sh.red) before the MMA of
-        // unit it + 2 and the next reduction reuse them
+        // this block's accumulator, tile and sh.red are free after the barrier
         tc_fence_before();
         __syncthreads();
+        if (tid == 0 && it + kRotStages < my_units) load(it + kRotStages);
     }
     if (tid == 0) {
         // leave no copy or MMA in flight
-        for (int l = waited; l < issued; ++l) mbar_drain_wait(&sh.a_full[l & 1], (l >> 1) & 1);
+        for (int l = waited; l < issued; ++l)
+            mbar_drain_wait(&sh.a_full[l % kRotStages], (l / kRotStages) & 1);
         tc_commit(&sh.drain);
         mbar_drain_wait(&sh.drain, 0);
     }
@@ -406,24 +422,25 @@ int launch_fp8_prepare(const Fp8PrepArgs &a, cudaStream_t stream) {
     if (nq <= 0) return 0;
     if (nq + 2 * nkv > INT_MAX) return -2;
     if (a.signs) {
-        // Q and K on the tensor core, then V's block maxima
-        alignas(64) CUtensorMap tq, tk;
+        // Q and K on the tensor core, V's block maxima in the same kernel
+        alignas(64) CUtensorMap tq, tk, tv;
         const uint64_t T = (uint64_t)a.B * a.N;
         if (encode_tensor_map_3d(&tq, a.q, 2, kD, a.Hq, T, (uint64_t)kD * 2,
                                  (uint64_t)a.Hq * kD * 2, 64, 1, kBlock, 128) ||
             encode_tensor_map_3d(&tk, a.k, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
+                                 (uint64_t)a.Hkv * kD * 2, 64, 1, kBlock, 128) ||
+            encode_tensor_map_3d(&tv, a.v, 2, kD, a.Hkv, T, (uint64_t)kD * 2,
                                  (uint64_t)a.Hkv * kD * 2, 64, 1, kBlock, 128))
             return -5;
         if (cudaFuncSetAttribute(fp8_rot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kRotSmem) != cudaSuccess)
             return -5;
-        const long long units = nq + nkv;
-        const long long cap = 2ll * device_sm_count();
+        const long long units = nq + 2 * nkv;
+        const long long cap = device_sm_count();
         const int grid = (int)(units < cap ? units : cap);
-        fp8_rot_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(tq, tk, a, (int)nblk);
-        fp8_quant_qk_kernel<<<(int)nkv, kThreads, 0, stream>>>(a, (int)nblk, (int)(nq + nkv));
+        fp8_rot_kernel<<<grid, kRotThreads, kRotSmem, stream>>>(tq, tk, tv, a, (int)nblk);
     } else {
-        fp8_quant_qk_kernel<<<(int)(nq + 2 * nkv), kThreads, 0, stream>>>(a, (int)nblk, 0);
+        fp8_quant_qk_kernel<<<(int)(nq + 2 * nkv), kThreads, 0, stream>>>(a, (int)nblk);
     }
     fp8_quant_vt_kernel<<<(int)nkv, kThreads, 0, stream>>>(a, (int)nblk);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
