@@ -511,7 +511,7 @@ def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, 
     bflops = 2.5 * flops
     ach = bflops / (ms * 1e-3) / 1e12
     out["bwd"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
-                  "flop_per_call": bflops, "launches_per_call": 2,
+                  "flop_per_call": bflops, "launches_per_call": 3,
                   "workload": "backward of the prefill workload (dQ, dK, dV), causal",
                   "roofline": {"bound": "tensor", "achieved": round(ach, 2),
                                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
