@@ -158,9 +158,21 @@ struct RotShared {
     uint64_t a_full[kRotStages], mma_done[2], drain;
     uint32_t tmem_base;
     int abort;
-    float red[kRotWarps];
+    int4 info[kRotStages];           // (tensor, batch, head, block) of the block in each stage
+    float red[2][kRotWarps];         // per-warp maxima, alternating by iteration
     float sgn[kD];
 };
+
+// Maximum of |v| over 64 values: eight independent chains, then a tree.
+__device__ __forceinline__ float absmax64(const float (&v)[64]) {
+    float m[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fabsf(v[i]);
+    #pragma unroll
+    for (int e = 8; e < 64; ++e) m[e & 7] = fmaxf(m[e & 7], fabsf(v[e]));
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+                 fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
 
 __global__ void __launch_bounds__(kRotThreads, 1)
 fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -202,10 +214,13 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         b = v / (nblk * H);
     };
     int issued = 0, waited = 0;                    // TMA loads (thread 0)
+    // (thread 0; the block's indices go to shared memory for the epilogue,
+    // read after the barriers that follow)
     auto load = [&](int it) {
         const int st = it % kRotStages;
         int which, b, h, blk;
         decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        sh.info[st] = make_int4(which, b, h, blk);
         mbar_arrive_expect_tx(&sh.a_full[st], kRotTile);
         const CUtensorMap *m = which == 0 ? &tmQ : (which == 1 ? &tmK : &tmV);
         for (int bx = 0; bx < 2; ++bx)
@@ -271,8 +286,8 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
         if (tid == 0 && ok && it + 1 < my_units) ok = mma(it + 1);
         tc_fence_after();
-        int which, b, h, blk;
-        decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        const int4 inf = sh.info[st];
+        const int which = inf.x, b = inf.y, h = inf.z, blk = inf.w;
         const int n = blk * kBlock + row;          // this thread's token (rows past N:
         const bool valid = n < a.N;                // the next batch or zeros -- left out)
         float v[64];
@@ -293,18 +308,20 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
             }
         }
-        if (ok && valid) {
-            #pragma unroll
-            for (int e = 0; e < 64; ++e) m = fmaxf(m, fabsf(v[e]));
-        }
+        if (ok && valid) m = absmax64(v);
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) sh.red[warp] = m;
+        float *red = sh.red[it & 1];
+        if (lane == 0) red[warp] = m;
+        // After this barrier every thread holds its values in registers: the
+        // block's accumulator and tile are free for the next MMA and load, and
+        // red[] of this iteration is rewritten only two iterations on.
+        tc_fence_before();
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
-        float amax = sh.red[0];
-        #pragma unroll
-        for (int w = 1; w < kRotWarps; ++w) amax = fmaxf(amax, sh.red[w]);
+        if (tid == 0 && it + kRotStages < my_units) load(it + kRotStages);
+        float amax = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
+                           fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
         if (which == 2) {
             if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
         } else {
@@ -328,10 +345,6 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
             }
         }
-        // this block's accumulator, tile and sh.red are free after the barrier
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && it + kRotStages < my_units) load(it + kRotStages);
     }
     if (tid == 0) {
         // leave no copy or MMA in flight
