@@ -146,18 +146,20 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
 // 128-token block of one head is one M = N = K = 128 bf16 MMA against the
 // +-1 matrix B[c][k] = signs[k] (-1)^popcount(k & c), which the CTA writes
 // once into shared memory in the 128-byte-swizzled K-major layout a TMA tile
-// has.  One persistent CTA per SM, 16 warps: thread 0 keeps TMA loads up to
+// has.  One persistent CTA per SM, 8 warps: thread 0 keeps TMA loads up to
 // four blocks ahead and issues each block's MMA one block ahead into one of
-// two TMEM accumulators; every thread owns a quarter of a token row (32
-// channels; warps w, w + 4, w + 8, w + 12 share TMEM lanes 32 (w % 4) ..)
-// for the epilogue: block maximum, power-of-two scale, E4M3 codes, 32-byte
-// stores.  The same CTAs
+// two TMEM accumulators; every thread owns half a token row (64 channels;
+// warps w and w + 4 share TMEM lanes 32 (w % 4) ..) for the epilogue: block
+// maximum, power-of-two scale, E4M3 codes, 64-byte stores.  The same CTAs
 // take V's blocks after their Q and K blocks, reading the tile from shared
 // memory for its maximum only.  fp32 accumulation of +-x terms: within a few
 // ulp of the exact sums.
-constexpr int kRotThreads = 512;
+constexpr int kRotThreads = 256;
 constexpr int kRotWarps = kRotThreads / 32;
-constexpr int kRotStages = 4;
+#ifndef FA_ROT_STAGES
+#define FA_ROT_STAGES 4
+#endif
+constexpr int kRotStages = FA_ROT_STAGES;
 constexpr int kRotTile = kBlock * kD * 2;          // one bf16 block: 32 KiB
 constexpr int kRotBox = kBlock * 128;              // 128 rows x 64 bf16
 constexpr int kRotSmem = (1 + kRotStages) * kRotTile + 1024;   // B, A ring, alignment
@@ -172,13 +174,13 @@ struct RotShared {
     float sgn[kD];
 };
 
-// Maximum of |v| over 32 values: eight independent chains, then a tree.
-__device__ __forceinline__ float absmax32(const float (&v)[32]) {
+// Maximum of |v| over 64 values: eight independent chains, then a tree.
+__device__ __forceinline__ float absmax64(const float (&v)[64]) {
     float m[8];
     #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = fabsf(v[i]);
     #pragma unroll
-    for (int e = 8; e < 32; ++e) m[e & 7] = fmaxf(m[e & 7], fabsf(v[e]));
+    for (int e = 8; e < 64; ++e) m[e & 7] = fmaxf(m[e & 7], fabsf(v[e]));
     return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                  fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
@@ -194,7 +196,7 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     uint8_t *sA = smem + kRotTile;                 // stage j at sA + j * kRotTile
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = (warp & 3) * 32 + lane;        // token row of the block
-    const int quarter = warp >> 2;                 // channels 32 quarter .. + 31
+    const int half = warp >> 2;                    // channels 64 half .. + 63
     const int nq = a.B * a.Hq * nblk, nkv = a.B * a.Hkv * nblk;
     const int units = nq + 2 * nkv;                // Q blocks, K blocks, V blocks
     int my_units = 0;
@@ -285,7 +287,7 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     bool ok = true;
     if (tid == 0 && my_units > 0) ok = mma(0);
-    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + quarter * 32;
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
     for (int it = 0; it < my_units; ++it) {
         const int st = it % kRotStages;
         const bool qk = is_qk(it);
@@ -299,26 +301,25 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int which = inf.x, b = inf.y, h = inf.z, blk = inf.w;
         const int n = blk * kBlock + row;          // this thread's token (rows past N:
         const bool valid = n < a.N;                // the next batch or zeros -- left out)
-        float v[32];
+        float v[64];
         float m = 0.f;
         if (ok && qk) {
             tmem_ld32(trow + (it & 1) * kD, reinterpret_cast<uint32_t *>(v));
+            tmem_ld32(trow + (it & 1) * kD + 32, reinterpret_cast<uint32_t *>(v) + 32);
             tmem_wait_ld();
         } else if (ok) {
-            // V: this row's 32 bf16 (box quarter / 2, chunks 4 (quarter % 2) ..),
-            // chunks swizzled by row & 7
-            const uint8_t *src = sA + st * kRotTile + (quarter >> 1) * kRotBox + row * 128;
+            // V: this row's 64 bf16 of box `half`, chunks swizzled by row & 7
+            const uint8_t *src = sA + st * kRotTile + half * kRotBox + row * 128;
             #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int ch = (quarter & 1) * 4 + c;
-                const uint4 q = *reinterpret_cast<const uint4 *>(src + ((ch ^ (row & 7)) << 4));
+            for (int c = 0; c < 8; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) << 4));
                 v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
                 v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
                 v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
                 v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
             }
         }
-        if (ok && valid) m = absmax32(v);
+        if (ok && valid) m = absmax64(v);
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         float *red = sh.red[it & 1];
@@ -330,11 +331,8 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
         if (tid == 0 && it + kRotStages < my_units) load(it + kRotStages);
-        float r4[4];
-        #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            r4[i] = fmaxf(fmaxf(red[4 * i], red[4 * i + 1]), fmaxf(red[4 * i + 2], red[4 * i + 3]));
-        const float amax = fmaxf(fmaxf(r4[0], r4[1]), fmaxf(r4[2], r4[3]));
+        float amax = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
+                           fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
         if (which == 2) {
             if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
         } else {
@@ -345,16 +343,17 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const int H = which ? a.Hkv : a.Hq;
             if (tid == 0) (which ? a.k_scale : a.q_scale)[(b * H + h) * nblk + blk] = pow2f(kexp);
             if (valid) {
-                uint32_t cw[8];
+                uint32_t cw[16];
                 #pragma unroll
-                for (int e = 0; e < 8; ++e)
+                for (int e = 0; e < 16; ++e)
                     cw[e] = pack_e4m3x4(v[4 * e] * mult, v[4 * e + 1] * mult, v[4 * e + 2] * mult,
                                         v[4 * e + 3] * mult);
                 uint4 *d4 = reinterpret_cast<uint4 *>(
                     static_cast<uint8_t *>(which ? a.k8 : a.q8) +
-                    (((size_t)b * a.N + n) * H + h) * kD + quarter * 32);
-                d4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                d4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                    (((size_t)b * a.N + n) * H + h) * kD + half * 64);
+                #pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
             }
         }
     }
