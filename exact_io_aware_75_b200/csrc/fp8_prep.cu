@@ -146,16 +146,19 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
 // 128-token block of one head is one M = N = K = 128 bf16 MMA against the
 // +-1 matrix B[c][k] = signs[k] (-1)^popcount(k & c), which the CTA writes
 // once into shared memory in the 128-byte-swizzled K-major layout a TMA tile
-// has.  One persistent CTA per SM, 8 warps: thread 0 keeps TMA loads up to
-// four blocks ahead and issues each block's MMA one block ahead into one of
-// two TMEM accumulators; every thread owns half a token row (64 channels;
-// warps w and w + 4 share TMEM lanes 32 (w % 4) ..) for the epilogue: block
-// maximum, power-of-two scale, E4M3 codes, 64-byte stores.  The same CTAs
-// take V's blocks after their Q and K blocks, reading the tile from shared
-// memory for its maximum only.  fp32 accumulation of +-x terms: within a few
-// ulp of the exact sums.
-constexpr int kRotThreads = 256;
-constexpr int kRotWarps = kRotThreads / 32;
+// has.  One persistent CTA per SM, warp-specialised:
+//   * warp 8 (one thread): TMA loads into a ring of kRotStages tiles and the
+//     MMAs into two TMEM accumulators, paced by full / empty mbarriers only;
+//   * warps 0-7: the epilogue, half a token row (64 channels) per thread
+//     (warps w and w + 4 share TMEM lanes 32 (w % 4) ..): block maximum over
+//     the eight warps (a named barrier of their own), power-of-two scale,
+//     E4M3 codes, 64-byte stores.
+// After their Q and K blocks the same CTAs take V's blocks, reading the tile
+// from shared memory for its maximum only.  fp32 accumulation of +-x terms:
+// within a few ulp of the exact sums.
+constexpr int kRotEpiWarps = 8;
+constexpr int kRotEpiThreads = kRotEpiWarps * 32;
+constexpr int kRotThreads = kRotEpiThreads + 32;   // + the TMA / MMA warp
 #ifndef FA_ROT_STAGES
 #define FA_ROT_STAGES 4
 #endif
@@ -164,13 +167,14 @@ constexpr int kRotTile = kBlock * kD * 2;          // one bf16 block: 32 KiB
 constexpr int kRotBox = kBlock * 128;              // 128 rows x 64 bf16
 constexpr int kRotSmem = (1 + kRotStages) * kRotTile + 1024;   // B, A ring, alignment
 constexpr uint32_t kRotTmemCols = 256;             // two 128-column accumulators
+constexpr int kRotEpiBar = 1;                      // named barrier of the epilogue warps
 
 struct RotShared {
-    uint64_t a_full[kRotStages], mma_done[2], drain;
+    uint64_t a_full[kRotStages], a_empty[kRotStages];
+    uint64_t acc_full[2], acc_empty[2], drain;
     uint32_t tmem_base;
     int abort;
-    int4 info[kRotStages];           // (tensor, batch, head, block) of the block in each stage
-    float red[2][kRotWarps];         // per-warp maxima, alternating by iteration
+    float red[2][kRotEpiWarps];      // per-warp maxima, alternating by iteration
     float sgn[kD];
 };
 
@@ -195,8 +199,6 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     uint8_t *sB = smem;
     uint8_t *sA = smem + kRotTile;                 // stage j at sA + j * kRotTile
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int row = (warp & 3) * 32 + lane;        // token row of the block
-    const int half = warp >> 2;                    // channels 64 half .. + 63
     const int nq = a.B * a.Hq * nblk, nkv = a.B * a.Hkv * nblk;
     const int units = nq + 2 * nkv;                // Q blocks, K blocks, V blocks
     int my_units = 0;
@@ -204,8 +206,14 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     volatile int *abort = &sh.abort;
 
     if (tid == 0) {
-        for (int j = 0; j < kRotStages; ++j) mbar_init(&sh.a_full[j], 1);
-        for (int j = 0; j < 2; ++j) mbar_init(&sh.mma_done[j], 1);
+        for (int j = 0; j < kRotStages; ++j) {
+            mbar_init(&sh.a_full[j], 1);
+            mbar_init(&sh.a_empty[j], 1);
+        }
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&sh.acc_full[j], 1);
+            mbar_init(&sh.acc_empty[j], 1);
+        }
         mbar_init(&sh.drain, 1);
         sh.abort = 0;
         fence_barrier_init();
@@ -224,14 +232,15 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         h = (v / nblk) % H;
         b = v / (nblk * H);
     };
-    int issued = 0, waited = 0;                    // TMA loads (thread 0)
-    // (thread 0; the block's indices go to shared memory for the epilogue,
-    // read after the barriers that follow)
+    // A CTA's units run in increasing order, Q and K before V, so a Q or K
+    // unit it is this CTA's it-th MMA: accumulator it & 1.
+    auto is_qk = [&](int it) { return blockIdx.x + it * gridDim.x < nq + nkv; };
+    const bool ctrl = warp == kRotEpiWarps && lane == 0;
+    int issued = 0;                                // TMA loads (control thread)
     auto load = [&](int it) {
         const int st = it % kRotStages;
         int which, b, h, blk;
         decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
-        sh.info[st] = make_int4(which, b, h, blk);
         mbar_arrive_expect_tx(&sh.a_full[st], kRotTile);
         const CUtensorMap *m = which == 0 ? &tmQ : (which == 1 ? &tmK : &tmV);
         for (int bx = 0; bx < 2; ++bx)
@@ -239,8 +248,8 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                         b * a.N + blk * kBlock);
         ++issued;
     };
-    // loads of the first blocks run while B is written
-    if (tid == 0) {
+    // the first tiles' loads run while B is written
+    if (ctrl) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -263,106 +272,116 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     fence_proxy_async_smem();
     __syncthreads();
-
     const uint32_t tmem = sh.tmem_base;
-    const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
-    const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
-    // A CTA's units run in increasing order, Q and K before V, so unit it of
-    // a Q or K block is its it-th MMA: accumulator it & 1.
-    auto is_qk = [&](int it) { return blockIdx.x + it * gridDim.x < nq + nkv; };
-    auto mma = [&](int it) -> bool {               // thread 0
-        const int st = it % kRotStages;
-        if (!mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort)) return false;
-        ++waited;
-        if (!is_qk(it)) return true;               // V: read from shared memory
-        tc_fence_after();
-        const uint32_t aa = a_lo + st * (kRotTile >> 4);
-        #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
-            mma_ss_lo(tmem + (it & 1) * kD, aa + off, b_lo + off, idesc, ks > 0 ? 1u : 0u);
+
+    if (warp == kRotEpiWarps) {
+        // ---------------- control: MMAs and the loads that refill the ring
+        if (ctrl) {
+            const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
+            const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
+            for (int it = 0; it < my_units; ++it) {
+                const int st = it % kRotStages;
+                if (is_qk(it)) {
+                    if (!mbar_wait(&sh.acc_empty[it & 1], ((it >> 1) & 1) ^ 1, abort)) break;
+                    if (!mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort)) break;
+                    tc_fence_after();
+                    const uint32_t aa = a_lo + st * (kRotTile >> 4);
+                    #pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
+                        mma_ss_lo(tmem + (it & 1) * kD, aa + off, b_lo + off, idesc,
+                                  ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sh.acc_full[it & 1]);
+                    tc_commit(&sh.a_empty[st]);    // the tile is free once the MMA is done
+                }
+                if (it + kRotStages < my_units) {
+                    if (!mbar_wait(&sh.a_empty[st], (it / kRotStages) & 1, abort)) break;
+                    load(it + kRotStages);
+                }
+            }
+            // leave no copy or MMA in flight: the last load of every stage, then
+            // every MMA issued
+            for (int st = 0; st < kRotStages; ++st)
+                if (issued > st) mbar_drain_wait(&sh.a_full[st], ((issued - 1 - st) / kRotStages) & 1);
+            tc_commit(&sh.drain);
+            mbar_drain_wait(&sh.drain, 0);
         }
-        tc_commit(&sh.mma_done[it & 1]);
-        return true;
-    };
-    bool ok = true;
-    if (tid == 0 && my_units > 0) ok = mma(0);
-    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
-    for (int it = 0; it < my_units; ++it) {
-        const int st = it % kRotStages;
-        const bool qk = is_qk(it);
-        if (qk)
-            ok = ok && mbar_wait(&sh.mma_done[it & 1], (it >> 1) & 1, abort);
-        else
-            ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
-        if (tid == 0 && ok && it + 1 < my_units) ok = mma(it + 1);
-        tc_fence_after();
-        const int4 inf = sh.info[st];
-        const int which = inf.x, b = inf.y, h = inf.z, blk = inf.w;
-        const int n = blk * kBlock + row;          // this thread's token (rows past N:
-        const bool valid = n < a.N;                // the next batch or zeros -- left out)
-        float v[64];
-        float m = 0.f;
-        if (ok && qk) {
-            tmem_ld32(trow + (it & 1) * kD, reinterpret_cast<uint32_t *>(v));
-            tmem_ld32(trow + (it & 1) * kD + 32, reinterpret_cast<uint32_t *>(v) + 32);
-            tmem_wait_ld();
-        } else if (ok) {
-            // V: this row's 64 bf16 of box `half`, chunks swizzled by row & 7
-            const uint8_t *src = sA + st * kRotTile + half * kRotBox + row * 128;
+    } else {
+        // ---------------- epilogue
+        const int row = (warp & 3) * 32 + lane;    // token row of the block
+        const int half = warp >> 2;                // channels 64 half .. + 63
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
+        bool ok = true;
+        for (int it = 0; it < my_units; ++it) {
+            const int st = it % kRotStages;
+            const bool qk = is_qk(it);
+            if (qk)
+                ok = ok && mbar_wait(&sh.acc_full[it & 1], (it >> 1) & 1, abort);
+            else
+                ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
+            tc_fence_after();
+            int which, b, h, blk;
+            decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+            const int n = blk * kBlock + row;      // this thread's token (rows past N:
+            const bool valid = n < a.N;            // the next batch or zeros -- left out)
+            float v[64];
+            float m = 0.f;
+            if (ok && qk) {
+                tmem_ld32(trow + (it & 1) * kD, reinterpret_cast<uint32_t *>(v));
+                tmem_ld32(trow + (it & 1) * kD + 32, reinterpret_cast<uint32_t *>(v) + 32);
+                tmem_wait_ld();
+            } else if (ok) {
+                // V: this row's 64 bf16 of box `half`, chunks swizzled by row & 7
+                const uint8_t *src = sA + st * kRotTile + half * kRotBox + row * 128;
+                #pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 q = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) << 4));
+                    v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
+                    v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
+                    v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
+                    v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
+                }
+            }
+            if (ok && valid) m = absmax64(v);
             #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 q = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) << 4));
-                v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
-                v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
-                v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
-                v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float *red = sh.red[it & 1];
+            if (lane == 0) red[warp] = m;
+            // after this barrier every epilogue thread holds its values in
+            // registers: the accumulator (or tile) goes back to the control
+            // warp; red[] of this iteration is rewritten two iterations on
+            tc_fence_before();
+            ok = named_bar_and(kRotEpiBar, kRotEpiThreads, ok);
+            if (!ok) break;
+            if (tid == 0) mbar_arrive(qk ? &sh.acc_empty[it & 1] : &sh.a_empty[st]);
+            const float amax = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
+                                     fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+            if (which == 2) {
+                if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
+            } else {
+                // the accumulator is H diag(signs) x; Q' = that / sqrt(128)
+                const float amax_c = amax * kInvSqrtD;
+                const int kexp = amax_c > 0.f ? scale_exp(amax_c) : 0;
+                const float mult = kInvSqrtD * pow2f(-kexp);
+                const int H = which ? a.Hkv : a.Hq;
+                if (tid == 0) (which ? a.k_scale : a.q_scale)[(b * H + h) * nblk + blk] = pow2f(kexp);
+                if (valid) {
+                    uint32_t cw[16];
+                    #pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        cw[e] = pack_e4m3x4(v[4 * e] * mult, v[4 * e + 1] * mult,
+                                            v[4 * e + 2] * mult, v[4 * e + 3] * mult);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(
+                        static_cast<uint8_t *>(which ? a.k8 : a.q8) +
+                        (((size_t)b * a.N + n) * H + h) * kD + half * 64);
+                    #pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
+                }
             }
         }
-        if (ok && valid) m = absmax64(v);
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float *red = sh.red[it & 1];
-        if (lane == 0) red[warp] = m;
-        // After this barrier every thread holds its values in registers: the
-        // block's accumulator and tile are free for the next MMA and load, and
-        // red[] of this iteration is rewritten only two iterations on.
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (tid == 0 && it + kRotStages < my_units) load(it + kRotStages);
-        float amax = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
-                           fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
-        if (which == 2) {
-            if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
-        } else {
-            // the accumulator is H diag(signs) x; Q' = that / sqrt(128)
-            const float amax_c = amax * kInvSqrtD;
-            const int kexp = amax_c > 0.f ? scale_exp(amax_c) : 0;
-            const float mult = kInvSqrtD * pow2f(-kexp);
-            const int H = which ? a.Hkv : a.Hq;
-            if (tid == 0) (which ? a.k_scale : a.q_scale)[(b * H + h) * nblk + blk] = pow2f(kexp);
-            if (valid) {
-                uint32_t cw[16];
-                #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    cw[e] = pack_e4m3x4(v[4 * e] * mult, v[4 * e + 1] * mult, v[4 * e + 2] * mult,
-                                        v[4 * e + 3] * mult);
-                uint4 *d4 = reinterpret_cast<uint4 *>(
-                    static_cast<uint8_t *>(which ? a.k8 : a.q8) +
-                    (((size_t)b * a.N + n) * H + h) * kD + half * 64);
-                #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
-            }
-        }
-    }
-    if (tid == 0) {
-        // leave no copy or MMA in flight
-        for (int l = waited; l < issued; ++l)
-            mbar_drain_wait(&sh.a_full[l % kRotStages], (l / kRotStages) & 1);
-        tc_commit(&sh.drain);
-        mbar_drain_wait(&sh.drain, 0);
+        if (!ok) *abort = 1;
     }
     tc_fence_before();
     __syncthreads();
