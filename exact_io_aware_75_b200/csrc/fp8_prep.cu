@@ -147,16 +147,25 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
 // +-1 matrix B[c][k] = signs[k] (-1)^popcount(k & c), which the CTA writes
 // once into shared memory in the 128-byte-swizzled K-major layout a TMA tile
 // has.  One persistent CTA per SM, warp-specialised:
-//   * warp 8 (one thread): TMA loads into a ring of kRotStages tiles and the
-//     MMAs into two TMEM accumulators, paced by full / empty mbarriers only;
-//   * warps 0-7: the epilogue, half a token row (64 channels) per thread
-//     (warps w and w + 4 share TMEM lanes 32 (w % 4) ..): block maximum over
-//     the eight warps (a named barrier of their own), power-of-two scale,
-//     E4M3 codes, 64-byte stores.
+//   * the last warp (one thread): TMA loads into a ring of kRotStages tiles
+//     and the MMAs into two TMEM accumulators, paced by full / empty
+//     mbarriers only; it writes each block's indices beside its tile, so the
+//     epilogue reads them after the tile's full barrier (release / acquire);
+//   * the other kRotEpiWarps warps: the epilogue, kRotCols channels of one
+//     token row per thread (warps w, w + 4, .. share TMEM lanes 32 (w % 4)
+//     ..): block maximum over the epilogue warps (a named barrier of their
+//     own), power-of-two scale, E4M3 codes, kRotCols-byte stores.  A tile's
+//     stage is released by the epilogue (not by the MMA), so a block's
+//     indices stay in place until every epilogue thread has read them.
 // After their Q and K blocks the same CTAs take V's blocks, reading the tile
 // from shared memory for its maximum only.  fp32 accumulation of +-x terms:
 // within a few ulp of the exact sums.
-constexpr int kRotEpiWarps = 8;
+#ifndef FA_ROT_EPI_WARPS
+#define FA_ROT_EPI_WARPS 8
+#endif
+constexpr int kRotEpiWarps = FA_ROT_EPI_WARPS;        // 8 or 16
+constexpr int kRotCols = kD * 4 / kRotEpiWarps;        // channels per epilogue thread
+static_assert(kRotEpiWarps == 8 || kRotEpiWarps == 16, "epilogue warps");
 constexpr int kRotEpiThreads = kRotEpiWarps * 32;
 constexpr int kRotThreads = kRotEpiThreads + 32;   // + the TMA / MMA warp
 #ifndef FA_ROT_STAGES
@@ -174,17 +183,19 @@ struct RotShared {
     uint64_t acc_full[2], acc_empty[2], drain;
     uint32_t tmem_base;
     int abort;
+    int4 info[kRotStages];           // (tensor, batch, head, block) of each stage's tile
     float red[2][kRotEpiWarps];      // per-warp maxima, alternating by iteration
     float sgn[kD];
 };
 
-// Maximum of |v| over 64 values: eight independent chains, then a tree.
-__device__ __forceinline__ float absmax64(const float (&v)[64]) {
+// Maximum of |v| over N values: eight independent chains, then a tree.
+template <int N>
+__device__ __forceinline__ float absmax(const float (&v)[N]) {
     float m[8];
     #pragma unroll
     for (int i = 0; i < 8; ++i) m[i] = fabsf(v[i]);
     #pragma unroll
-    for (int e = 8; e < 64; ++e) m[e & 7] = fmaxf(m[e & 7], fabsf(v[e]));
+    for (int e = 8; e < N; ++e) m[e & 7] = fmaxf(m[e & 7], fabsf(v[e]));
     return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                  fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
@@ -241,6 +252,7 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int st = it % kRotStages;
         int which, b, h, blk;
         decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+        sh.info[st] = make_int4(which, b, h, blk);
         mbar_arrive_expect_tx(&sh.a_full[st], kRotTile);
         const CUtensorMap *m = which == 0 ? &tmQ : (which == 1 ? &tmK : &tmV);
         for (int bx = 0; bx < 2; ++bx)
@@ -275,29 +287,55 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tmem = sh.tmem_base;
 
     if (warp == kRotEpiWarps) {
-        // ---------------- control: MMAs and the loads that refill the ring
+        // ---------------- control: MMAs and the loads that refill the ring.
+        // Both wait on the epilogue (an accumulator, a stage), in different
+        // orders, so neither blocks the other: poll and issue whichever is
+        // ready, giving up after kWaitLimitCycles without progress.
         if (ctrl) {
             const uint32_t b_lo = desc_lo(smem_u32(sB), 16), a_lo = desc_lo(smem_u32(sA), 16);
             const uint32_t idesc = idesc_bf16_f32(kBlock, kD, false);
-            for (int it = 0; it < my_units; ++it) {
-                const int st = it % kRotStages;
-                if (is_qk(it)) {
-                    if (!mbar_wait(&sh.acc_empty[it & 1], ((it >> 1) & 1) ^ 1, abort)) break;
-                    if (!mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort)) break;
-                    tc_fence_after();
-                    const uint32_t aa = a_lo + st * (kRotTile >> 4);
-                    #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
-                        mma_ss_lo(tmem + (it & 1) * kD, aa + off, b_lo + off, idesc,
-                                  ks > 0 ? 1u : 0u);
+            int it_mma = 0;
+            long long t_progress = clock64();
+            for (uint32_t spin = 0; it_mma < my_units || issued < my_units; ++spin) {
+                bool progressed = false;
+                if (it_mma < my_units) {
+                    const int st = it_mma % kRotStages;
+                    if (!is_qk(it_mma)) {
+                        ++it_mma;                  // V: no MMA
+                        progressed = true;
+                    } else if (mbar_test(smem_u32(&sh.acc_empty[it_mma & 1]),
+                                         ((it_mma >> 1) & 1) ^ 1) &&
+                               mbar_test(smem_u32(&sh.a_full[st]), (it_mma / kRotStages) & 1)) {
+                        tc_fence_after();
+                        const uint32_t aa = a_lo + st * (kRotTile >> 4);
+                        #pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks) {
+                            const uint32_t off = ((ks >> 2) * kRotBox + (ks & 3) * 32) >> 4;
+                            mma_ss_lo(tmem + (it_mma & 1) * kD, aa + off, b_lo + off, idesc,
+                                      ks > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&sh.acc_full[it_mma & 1]);
+                        ++it_mma;
+                        progressed = true;
                     }
-                    tc_commit(&sh.acc_full[it & 1]);
-                    tc_commit(&sh.a_empty[st]);    // the tile is free once the MMA is done
                 }
-                if (it + kRotStages < my_units) {
-                    if (!mbar_wait(&sh.a_empty[st], (it / kRotStages) & 1, abort)) break;
-                    load(it + kRotStages);
+                if (issued < my_units) {
+                    // load `issued` reuses the stage of unit issued - kRotStages
+                    const int prev = issued - kRotStages;
+                    if (mbar_test(smem_u32(&sh.a_empty[prev % kRotStages]), (prev / kRotStages) & 1)) {
+                        load(issued);
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_progress = clock64();
+                } else if ((spin & 63) == 0) {
+                    if (*abort) break;
+                    if (clock64() - t_progress > kWaitLimitCycles) {
+                        *abort = 1;
+                        report_error(kDevErrTimeout);
+                        break;
+                    }
                 }
             }
             // leave no copy or MMA in flight: the last load of every stage, then
@@ -310,40 +348,41 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     } else {
         // ---------------- epilogue
         const int row = (warp & 3) * 32 + lane;    // token row of the block
-        const int half = warp >> 2;                // channels 64 half .. + 63
-        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 64;
+        const int col0 = (warp >> 2) * kRotCols;   // first channel of this thread
+        const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16) + col0;
         bool ok = true;
         for (int it = 0; it < my_units; ++it) {
             const int st = it % kRotStages;
             const bool qk = is_qk(it);
-            if (qk)
-                ok = ok && mbar_wait(&sh.acc_full[it & 1], (it >> 1) & 1, abort);
-            else
-                ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
+            ok = ok && mbar_wait(&sh.a_full[st], (it / kRotStages) & 1, abort);
+            if (qk) ok = ok && mbar_wait(&sh.acc_full[it & 1], (it >> 1) & 1, abort);
             tc_fence_after();
-            int which, b, h, blk;
-            decode(blockIdx.x + it * gridDim.x, which, b, h, blk);
+            const int4 inf = sh.info[st];
+            const int which = inf.x, b = inf.y, h = inf.z, blk = inf.w;
             const int n = blk * kBlock + row;      // this thread's token (rows past N:
             const bool valid = n < a.N;            // the next batch or zeros -- left out)
-            float v[64];
+            float v[kRotCols];
             float m = 0.f;
             if (ok && qk) {
-                tmem_ld32(trow + (it & 1) * kD, reinterpret_cast<uint32_t *>(v));
-                tmem_ld32(trow + (it & 1) * kD + 32, reinterpret_cast<uint32_t *>(v) + 32);
+                #pragma unroll
+                for (int q = 0; q < kRotCols / 32; ++q)
+                    tmem_ld32(trow + (it & 1) * kD + q * 32, reinterpret_cast<uint32_t *>(v) + 32 * q);
                 tmem_wait_ld();
             } else if (ok) {
-                // V: this row's 64 bf16 of box `half`, chunks swizzled by row & 7
-                const uint8_t *src = sA + st * kRotTile + half * kRotBox + row * 128;
+                // V: this row's bf16 channels col0 .. from box col0 / 64, chunks
+                // swizzled by row & 7
+                const uint8_t *src = sA + st * kRotTile + (col0 / 64) * kRotBox + row * 128;
                 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 q = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) << 4));
+                for (int c = 0; c < kRotCols / 8; ++c) {
+                    const int ch = (col0 % 64) / 8 + c;
+                    const uint4 q = *reinterpret_cast<const uint4 *>(src + ((ch ^ (row & 7)) << 4));
                     v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
                     v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
                     v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
                     v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
                 }
             }
-            if (ok && valid) m = absmax64(v);
+            if (ok && valid) m = absmax<kRotCols>(v);
             #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             float *red = sh.red[it & 1];
@@ -354,9 +393,17 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tc_fence_before();
             ok = named_bar_and(kRotEpiBar, kRotEpiThreads, ok);
             if (!ok) break;
-            if (tid == 0) mbar_arrive(qk ? &sh.acc_empty[it & 1] : &sh.a_empty[st]);
-            const float amax = fmaxf(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])),
-                                     fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+            if (tid == 0) {
+                if (qk) mbar_arrive(&sh.acc_empty[it & 1]);
+                mbar_arrive(&sh.a_empty[st]);
+            }
+            float r4[kRotEpiWarps / 4];
+            #pragma unroll
+            for (int i = 0; i < kRotEpiWarps / 4; ++i)
+                r4[i] = fmaxf(fmaxf(red[4 * i], red[4 * i + 1]), fmaxf(red[4 * i + 2], red[4 * i + 3]));
+            float amax = r4[0];
+            #pragma unroll
+            for (int i = 1; i < kRotEpiWarps / 4; ++i) amax = fmaxf(amax, r4[i]);
             if (which == 2) {
                 if (tid == 0) a.v_block_max[(b * a.Hkv + h) * nblk + blk] = amax;
             } else {
@@ -367,16 +414,16 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const int H = which ? a.Hkv : a.Hq;
                 if (tid == 0) (which ? a.k_scale : a.q_scale)[(b * H + h) * nblk + blk] = pow2f(kexp);
                 if (valid) {
-                    uint32_t cw[16];
+                    uint32_t cw[kRotCols / 4];
                     #pragma unroll
-                    for (int e = 0; e < 16; ++e)
+                    for (int e = 0; e < kRotCols / 4; ++e)
                         cw[e] = pack_e4m3x4(v[4 * e] * mult, v[4 * e + 1] * mult,
                                             v[4 * e + 2] * mult, v[4 * e + 3] * mult);
                     uint4 *d4 = reinterpret_cast<uint4 *>(
                         static_cast<uint8_t *>(which ? a.k8 : a.q8) +
-                        (((size_t)b * a.N + n) * H + h) * kD + half * 64);
+                        (((size_t)b * a.N + n) * H + h) * kD + col0);
                     #pragma unroll
-                    for (int e = 0; e < 4; ++e)
+                    for (int e = 0; e < kRotCols / 16; ++e)
                         d4[e] = make_uint4(cw[4 * e], cw[4 * e + 1], cw[4 * e + 2], cw[4 * e + 3]);
                 }
             }
