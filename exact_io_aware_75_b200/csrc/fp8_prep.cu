@@ -80,7 +80,8 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 
 // Without a rotation: Q and K blocks scaled and quantised; V blocks: their
 // maximum only.  blockIdx.x runs over the Q blocks, then K, then V, each
-// (b, h, blk) with blk fastest.  (With a rotation, fp8_rot_kernel does all of
+// (b, blk, h) with the head fastest, so CTAs running together read whole
+// token rows (all heads) rather than one head's slice of many rows.  (With a rotation, fp8_rot_kernel does all of
 // this.)
 __global__ void __launch_bounds__(kThreads)
 fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
@@ -101,7 +102,8 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
         H = a.Hkv;
         idx -= nq + nk;
     }
-    const int blk = idx % nblk, h = (idx / nblk) % H, b = idx / (nblk * H);
+    const int h = idx % H, blk = (idx / H) % nblk, b = idx / (H * nblk);
+    const int sidx = (b * H + h) * nblk + blk;   // [B, H, nblk] layout of the scales
     const uint16_t *src = static_cast<const uint16_t *>(which == 0 ? a.q : which == 1 ? a.k : a.v);
     const int n0 = blk * kBlock + warp * kRowsPerWarp;
     // all 16 row loads in flight before any arithmetic (8 bytes per lane,
@@ -125,12 +127,12 @@ fp8_quant_qk_kernel(const Fp8PrepArgs a, int nblk) {
     }
     amax = block_max(amax, red);
     if (which == 2) {
-        if (threadIdx.x == 0) a.v_block_max[idx] = amax;
+        if (threadIdx.x == 0) a.v_block_max[sidx] = amax;
         return;
     }
     const int kexp = amax > 0.f ? scale_exp(amax) : 0;
     const float mult = pow2f(-kexp);
-    if (threadIdx.x == 0) (which == 0 ? a.q_scale : a.k_scale)[idx] = pow2f(kexp);
+    if (threadIdx.x == 0) (which == 0 ? a.q_scale : a.k_scale)[sidx] = pow2f(kexp);
     uint8_t *dst = static_cast<uint8_t *>(which == 0 ? a.q8 : a.k8);
     #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
@@ -239,9 +241,9 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         which = u < nq ? 0 : (u < nq + nkv ? 1 : 2);
         const int H = which ? a.Hkv : a.Hq;
         const int v = u - (which == 0 ? 0 : (which == 1 ? nq : nq + nkv));
-        blk = v % nblk;
-        h = (v / nblk) % H;
-        b = v / (nblk * H);
+        h = v % H;
+        blk = (v / H) % nblk;
+        b = v / (H * nblk);
     };
     // A CTA's units run in increasing order, Q and K before V, so a Q or K
     // unit it is this CTA's it-th MMA: accumulator it & 1.
@@ -436,8 +438,9 @@ fp8_rot_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (warp == 0) tmem_dealloc(tmem, kRotTmemCols);
 }
 
-// V codes, transposed: CTA (b * Hkv + h) * nblk + blk writes rows c = 0..127
-// of keys blk * 128 .. + 127 (those below N).  The block goes through shared
+// V codes, transposed: CTA (b * nblk + blk) * Hkv + h (head fastest, as
+// above) writes rows c = 0..127 of (b, h) for keys blk * 128 .. + 127 (those
+// below N).  The block goes through shared
 // memory as 32-bit words (four channels of one token), column-swizzled by
 // token / 4 so that both phases are free of bank conflicts; each lane then
 // turns a 4 x 4 byte block (four tokens x four channels) around in registers
@@ -447,8 +450,8 @@ fp8_quant_vt_kernel(const Fp8PrepArgs a, int nblk) {
     __shared__ uint32_t sW[kBlock][kD / 4];   // [token][channel group ^ (token / 4)]
     __shared__ float red[kWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
-    const int b = bh / a.Hkv, h = bh % a.Hkv;
+    const int h = blockIdx.x % a.Hkv, blk = (blockIdx.x / a.Hkv) % nblk;
+    const int b = blockIdx.x / (a.Hkv * nblk), bh = b * a.Hkv + h;
     const int n0 = blk * kBlock;
     const uint16_t *src = static_cast<const uint16_t *>(a.v);
     // the block's rows in flight while the (b, h) maximum is reduced
