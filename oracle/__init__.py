@@ -89,6 +89,10 @@ def lib():
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
         L.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
+        L.oracle_attn_varlen_rows_sink_tokens.argtypes = [
+            _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
+        L.oracle_attn_varlen_rows_sink_tokens.restype = ctypes.c_int
         L.oracle_hadamard_rotate.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int,
                                              ctypes.c_void_p, _f64p]
         L.oracle_hadamard_rotate.restype = ctypes.c_int
@@ -443,6 +447,32 @@ def attn_doc(q, k, v, doc_ids, causal=False, window=0, scale=None, rows=None):
                                              vb.reshape(B * N, Hkv, d), cu, B, Hq, Hkv, d,
                                              int(causal), int(window), float(scale), doc, rp,
                                              nrows, o, lse), "attn_doc")
+    if rows is not None:
+        return o, lse
+    return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(B, N, Hq).transpose(0, 2, 1))
+
+
+def attn_sink_tokens(q, k, v, window, n_sink, scale=None, rows=None):
+    """Dense causal batch with a sliding window of W keys that also keeps the
+    first n_sink tokens visible (StreamingLLM's sink tokens).  -> O [B,N,Hq,d],
+    LSE [B,Hq,N]; with ``rows`` (list of (b, i)) only those: O [R,Hq,d], LSE [R,Hq]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, Hq, d = qb.shape
+    Hkv = kb.shape[2]
+    cu = np.arange(B + 1, dtype=np.int32) * N
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        nrows, rp = B * N, None
+    else:
+        r = np.ascontiguousarray(np.asarray([int(b) * N + int(i) for b, i in rows], dtype=np.int64))
+        nrows, rp = r.size, r.ctypes.data_as(ctypes.c_void_p)
+    o = np.empty((nrows, Hq, d), np.float64)
+    lse = np.empty((nrows, Hq), np.float64)
+    _check(lib().oracle_attn_varlen_rows_sink_tokens(
+        qb.reshape(B * N, Hq, d), kb.reshape(B * N, Hkv, d), vb.reshape(B * N, Hkv, d), cu, B,
+        Hq, Hkv, d, int(window), int(n_sink), float(scale), rp, nrows, o, lse),
+        "attn_sink_tokens")
     if rows is not None:
         return o, lse
     return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(B, N, Hq).transpose(0, 2, 1))

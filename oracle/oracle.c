@@ -46,6 +46,8 @@
  *   - oracle_prefill_paged: a chunk of new queries over a paged cache, the
  *     chunk holding each sequence's last positions;
  *   - oracle_attn_varlen_rows_doc: a document mask by per-token ids;
+ *   - oracle_attn_varlen_rows_sink_tokens: a sliding window that keeps the
+ *     first tokens of each sequence visible;
  *   - oracle_hadamard_rotate, oracle_e4m3_encode, oracle_quantize_e4m3_blocks,
  *     oracle_attn_fp8: the FP8 prefill with incoherent processing (rotation
  *     of Q and K, block-scaled E4M3 codes, attention over the codes).
@@ -168,6 +170,7 @@ static int attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const ui
                                   const int32_t *cu_seqlens, int num_seqs,
                                   int Hq, int Hkv, int d, int causal, int window,
                                   double scale, const double *sinks, const int32_t *doc,
+                                  int n_sink_tokens,
                                   const int64_t *rows, int64_t nrows, double *o, double *lse)
 {
     if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0) return -1;
@@ -213,7 +216,8 @@ static int attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const ui
                 for (int64_t j = 0; j < L; ++j) {
                     kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
                     vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
-                    vis[j] = (unsigned char)(allowed(i, j, causal, window) &&
+                    vis[j] = (unsigned char)((allowed(i, j, causal, window) ||
+                                              (causal && j <= i && j < n_sink_tokens)) &&
                                              (!doc || doc[start + i] == doc[start + j]));
                 }
                 attend_row_sink(qd, d, L, kp, vp, vis, scale, sinks ? sinks[h] : -INFINITY, s,
@@ -232,7 +236,7 @@ int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t
                             double *o, double *lse)
 {
     return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
-                                  scale, NULL, NULL, rows, nrows, o, lse);
+                                  scale, NULL, NULL, 0, rows, nrows, o, lse);
 }
 
 /*
@@ -249,7 +253,7 @@ int oracle_attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const ui
 {
     if (!sinks) return -1;
     return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
-                                  scale, sinks, NULL, rows, nrows, o, lse);
+                                  scale, sinks, NULL, 0, rows, nrows, o, lse);
 }
 
 /*
@@ -268,7 +272,26 @@ int oracle_attn_varlen_rows_doc(const uint16_t *q, const uint16_t *k, const uint
 {
     if (!doc) return -1;
     return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, causal, window,
-                                  scale, NULL, doc, rows, nrows, o, lse);
+                                  scale, NULL, doc, 0, rows, nrows, o, lse);
+}
+
+/*
+ * Sink tokens with a sliding window ("Sliding windows and local:global
+ * layers": StreamingLLM keeps a handful of sink tokens plus a recent
+ * window): with causal and window W > 0, key j is visible from query i if
+ * j <= i and (j > i - W or j < n_sink) -- the first n_sink tokens of each
+ * sequence stay visible to every later query.  Otherwise as
+ * oracle_attn_varlen_rows.
+ */
+int oracle_attn_varlen_rows_sink_tokens(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                        const int32_t *cu_seqlens, int num_seqs, int Hq,
+                                        int Hkv, int d, int window, int n_sink, double scale,
+                                        const int64_t *rows, int64_t nrows, double *o,
+                                        double *lse)
+{
+    if (window <= 0 || n_sink < 0) return -1;
+    return attn_varlen_rows_sinks(q, k, v, cu_seqlens, num_seqs, Hq, Hkv, d, 1, window,
+                                  scale, NULL, NULL, n_sink, rows, nrows, o, lse);
 }
 
 /* Dense batch: q [B,N,Hq,d], k/v [B,N,Hkv,d]; o [B,N,Hq,d]; lse [B,Hq,N]. */
