@@ -39,7 +39,7 @@ FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa_fwd_paged",
-           "fa_fwd_doc",
+           "fa_fwd_doc", "fa_fwd_sink_tokens",
            "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen", "fa_bwd_sinks",
            "fa_bwd_varlen_sinks",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
@@ -71,6 +71,8 @@ def _load():
     lib.fa_fwd_varlen_sinks.restype = i
     lib.fa_decode_paged_sinks.argtypes = [vp] * 8 + [i] * 7 + [f, vp, sz, vp]
     lib.fa_decode_paged_sinks.restype = i
+    lib.fa_fwd_sink_tokens.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp]
+    lib.fa_fwd_sink_tokens.restype = i
     lib.fa_fwd_doc.argtypes = [vp] * 6 + [i] * 7 + [f, i, vp]
     lib.fa_fwd_doc.restype = i
     lib.fa_fwd_paged.argtypes = [vp] * 9 + [i] * 11 + [f, i, vp]
@@ -153,10 +155,12 @@ def _need(t, dtype, ndim, name):
 
 
 def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
-        out=None, lse=None, return_lse=True, stream=None, sinks=None, doc_ids=None):
+        out=None, lse=None, return_lse=True, stream=None, sinks=None, doc_ids=None,
+        sink_tokens=None):
     """Dense prefill.  q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 -> (O [B,N,Hq,d], LSE [B,Hq,N]).
     ``sinks`` (fp32 [Hq], device) selects fa_fwd_sinks; ``doc_ids`` (int32 [B,N],
-    device) selects fa_fwd_doc."""
+    device) selects fa_fwd_doc; ``sink_tokens`` (an int, with causal and a window)
+    selects fa_fwd_sink_tokens."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, 4, n)
     B, N, Hq, d = q.shape
@@ -170,6 +174,13 @@ def fwd(q, k, v, causal=False, window=0, scale=None, out_dtype=torch.bfloat16,
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    if sink_tokens is not None:
+        if sinks is not None or doc_ids is not None or not causal:
+            raise FAError(FA_ERR_UNSUPPORTED, "sink_tokens with sinks, doc_ids or non-causal")
+        _check(_lib.fa_fwd_sink_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
+                                       Hkv, N, d, int(window), int(sink_tokens), float(scale),
+                                       od, _stream(stream)), "fa_fwd_sink_tokens")
+        return out, lse
     if doc_ids is not None:
         if sinks is not None:
             raise FAError(FA_ERR_UNSUPPORTED, "sinks with doc_ids")

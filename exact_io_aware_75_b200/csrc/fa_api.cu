@@ -127,7 +127,8 @@ namespace {
 
 int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
               const float *sinks, int B, int Hq, int Hkv, int N, int d, int causal, int window,
-              float scale, int o_dtype, void *stream, const int *doc = nullptr) {
+              float scale, int o_dtype, void *stream, const int *doc = nullptr,
+              int n_sink = 0) {
     if (B < 0 || N < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
     if (rc) return rc;
@@ -151,6 +152,7 @@ int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
     a.o_fp32 = o_dtype == FA_OUT_FP32;
     a.sinks = sinks;
     a.doc = doc;
+    a.n_sink = n_sink;
     return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -193,6 +195,14 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
            void *stream) {
     return fwd_dense(q, k, v, o, lse, nullptr, B, Hq, Hkv, N, d, causal, window, scale,
                      o_dtype, stream);
+}
+
+int fa_fwd_sink_tokens(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int N, int d, int window, int n_sink,
+                       float scale, int o_dtype, void *stream) {
+    if (window <= 0 || n_sink < 0) return FA_ERR_INVALID_ARG;
+    return fwd_dense(q, k, v, o, lse, nullptr, B, Hq, Hkv, N, d, 1, window, scale, o_dtype,
+                     stream, nullptr, n_sink);
 }
 
 int fa_fwd_sinks(const void *q, const void *k, const void *v, void *o, float *lse,

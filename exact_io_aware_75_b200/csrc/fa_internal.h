@@ -28,6 +28,8 @@ struct PrefillArgs {
     int max_pages, num_pages;
     // document mask: one id per token; nullptr = none
     const int *doc;
+    // sink tokens kept visible beside a causal window (0 = none)
+    int n_sink;
     // FP8 operands (launch_prefill_fp8): q, k hold E4M3 codes, v the
     // transposed V codes [B, Hkv, d, vt_stride]; scales per (sequence, head,
     // 128-token block) for Q and K, per (sequence, KV head) for V

@@ -114,6 +114,9 @@ struct Params {
     // head, 128-token block) for Q and K, per (sequence, KV head) for V.
     const float *q_scale, *k_scale, *v_scale;
     int nblk;   // 128-token blocks per sequence
+    // Sink tokens (with causal and a window): keys j < n_sink of a sequence
+    // stay visible to every later query; 0 = none.
+    int n_sink;
 };
 
 struct Unit {
@@ -125,9 +128,13 @@ struct Unit {
     int off;    // key position of query row 0 (Lk - L)
     int lo[2], hi[2];  // key-block range per tile, [lo, hi)
     int lo_all, hi_all;
+    // Sink tokens: tile t also takes key blocks [0, ns[t]) (ns[t] <= lo[t]);
+    // the unit walks blocks [0, A) then [lo_all, hi_all), A = the tiles'
+    // largest ns capped at lo_all.
+    int ns[2], A;
 };
 
-template <bool PAGED>
+template <bool PAGED, bool SINK = false>
 __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     const int per_mb = p.num_seqs * p.Hq;
     const int mb = p.num_mblocks - 1 - u / per_mb;
@@ -172,7 +179,20 @@ __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
         w.lo_all = min(w.lo_all, lo);
         w.hi_all = max(w.hi_all, hi);
     }
+    w.ns[0] = w.ns[1] = w.A = 0;
+    if (SINK && !PAGED && p.n_sink > 0 && p.causal && p.window > 0) {
+        const int sb = min((p.n_sink + kBlockN - 1) / kBlockN, nkb);
+        w.ns[0] = (w.lo[0] < w.hi[0]) ? min(sb, w.lo[0]) : 0;
+        w.ns[1] = (w.lo[1] < w.hi[1]) ? min(sb, w.lo[1]) : 0;
+        w.A = min(max(w.ns[0], w.ns[1]), w.lo_all);
+    }
     return true;
+}
+
+// The unit's key blocks in order: [0, A) (sink blocks), then [lo_all, hi_all).
+__device__ __forceinline__ int unit_first(const Unit &w) { return w.A > 0 ? 0 : w.lo_all; }
+__device__ __forceinline__ int unit_next(const Unit &w, int j) {
+    return (j + 1 == w.A) ? w.lo_all : j + 1;
 }
 
 // Unit `it` of this CTA: rows of G = gridDim.x units are walked in
@@ -200,7 +220,7 @@ struct Shared {
 // Dense and packed batches: one thread issues every copy.
 // FP8: one 128-byte box per tile row; V comes transposed (d rows of 128
 // keys), so its tile is read at (key, 0, sequence * Hkv + KV head).
-template <int D, bool DOC, bool F8>
+template <int D, bool DOC, bool F8, bool SINK>
 __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const CUtensorMap *tmV,
                          const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
     using C = Cfg<D, DOC, F8>;
@@ -209,7 +229,7 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
     uint32_t kv_it = 0;
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit<false>(u, p, w)) continue;
+        if (!get_unit<false, SINK>(u, p, w)) continue;
         for (int t = 0; t < 2; ++t) {
             if (w.lo[t] >= w.hi[t]) continue;
             if (!mbar_wait(&sh.q_empty[t], (q_uses[t] & 1) ^ 1, abort)) goto out;
@@ -219,7 +239,8 @@ __device__ void producer(const CUtensorMap *tmQ, const CUtensorMap *tmK, const C
                             b * C::kBoxCols, w.h, w.tok0 + w.q0 + t * kBlockM);
             ++q_uses[t];
         }
-        for (int j = w.lo_all; j < w.hi_all; ++j) {
+        for (int j = SINK ? unit_first(w) : w.lo_all; j < w.hi_all;
+             j = SINK ? unit_next(w, j) : j + 1) {
             for (int kv = 0; kv < 2; ++kv) {
                 const int slot = kv_it % C::kStages;
                 const uint32_t use = kv_it / C::kStages;
@@ -360,7 +381,7 @@ out:
 }
 
 // ------------------------------------------------------------ MMA issuer
-template <int D, bool PAGED, bool DOC, bool F8>
+template <int D, bool PAGED, bool DOC, bool F8, bool SINK>
 __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sKV) {
     using C = Cfg<D, DOC, F8>;
     volatile int *abort = &sh.abort;
@@ -437,7 +458,7 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
 
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit<PAGED>(u, p, w)) continue;
+        if (!get_unit<PAGED, SINK>(u, p, w)) continue;
         bool first_pv[2] = {true, true};
         for (int t = 0; t < 2; ++t) {
             if (w.lo[t] >= w.hi[t]) continue;
@@ -446,10 +467,12 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
         }
         tc_fence_after();
         int prev_v = -1;
-        for (int j = w.lo_all; j < w.hi_all; ++j) {
-            const bool in0 = j >= w.lo[0] && j < w.hi[0];
-            const bool in1 = j >= w.lo[1] && j < w.hi[1];
-            const bool prev1 = (j - 1) >= w.lo[1] && (j - 1) < w.hi[1];
+        bool last1 = false;       // (sink tokens) the previous block was one of tile 1's
+        for (int j = SINK ? unit_first(w) : w.lo_all; j < w.hi_all;
+             j = SINK ? unit_next(w, j) : j + 1) {
+            const bool in0 = (SINK && j < w.ns[0]) || (j >= w.lo[0] && j < w.hi[0]);
+            const bool in1 = (SINK && j < w.ns[1]) || (j >= w.lo[1] && j < w.hi[1]);
+            const bool prev1 = SINK ? last1 : ((j - 1) >= w.lo[1] && (j - 1) < w.hi[1]);
             const int kslot = kv_it % C::kStages;
             if (!mbar_wait(&sh.kv_full[kslot], (kv_it / C::kStages) & 1, abort)) goto out;
             ++kv_it;
@@ -479,8 +502,9 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *sQ, uint8_t *sK
             }
             if (!in1) tc_commit(&sh.kv_empty[vslot]);
             prev_v = vslot;
+            if (SINK) last1 = in1;
         }
-        if ((w.hi_all - 1) >= w.lo[1] && (w.hi_all - 1) < w.hi[1]) {
+        if (SINK ? last1 : ((w.hi_all - 1) >= w.lo[1] && (w.hi_all - 1) < w.hi[1])) {
             if (!issue_pv(1, prev_v, first_pv[1])) goto out;
             tc_commit(&sh.kv_empty[prev_v]);
         }
@@ -560,7 +584,7 @@ __device__ __forceinline__ void exp_half_f8(const float (&v)[kHalf], float sl2, 
 }
 
 // ---------------------------------------------------------------- softmax
-template <int D, bool PAGED, bool DOC, bool F8>
+template <int D, bool PAGED, bool DOC, bool F8, bool SINK>
 __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
     using C = Cfg<D, DOC, F8>;
     volatile int *abort = &sh.abort;
@@ -574,10 +598,11 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
 
     FOR_EACH_UNIT(u) {
         Unit w;
-        if (!get_unit<PAGED>(u, p, w)) continue;
+        if (!get_unit<PAGED, SINK>(u, p, w)) continue;
         // (selects, not w.lo[t]: a run-time index would keep the unit in
         // local memory)
         const int lo = t ? w.lo[1] : w.lo[0], hi = t ? w.hi[1] : w.hi[0];
+        const int ns = SINK ? (t ? w.ns[1] : w.ns[0]) : 0;   // sink blocks before lo
         if (lo >= hi) continue;
         const int row = w.q0 + t * kBlockM + r;    // row index within the sequence
         const int rmin = w.q0 + t * kBlockM, rmax = rmin + kBlockM - 1;
@@ -606,7 +631,8 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             ksc = p.k_scale + ((size_t)w.seq * p.Hkv + w.kvh) * p.nblk;
         }
         float m_ref = -INFINITY, l = 0.f;
-        for (int j = lo; j < hi; ++j) {
+        const int j0 = (SINK && ns > 0) ? 0 : lo;
+        for (int j = j0; j < hi; j = (SINK && j + 1 == ns) ? lo : j + 1) {
             float sl2 = p.scale_log2;
             if constexpr (F8) sl2 *= sq * __ldg(ksc + j);
             if (!mbar_wait_warp(&sh.s_full[t], s_cnt & 1, abort)) return;
@@ -621,7 +647,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             }
             ++s_cnt;
             tc_fence_after();
-            const bool first = (j == lo);
+            const bool first = (j == j0);
             const int k0 = j * kBlockN;
             // keys of the sequence and the key position of query row 0:
             // L and 0 for dense and packed batches
@@ -636,6 +662,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             int c_hi = Lk - k0;
             if (p.causal) c_hi = min(c_hi, pos + 1 - k0);
             const int c_lo = (p.window > 0) ? pos - p.window + 1 - k0 : 0;
+            const int c_sink = SINK ? p.n_sink - k0 : INT_MIN;   // keys c < c_sink: sink tokens
             // Scores in two halves of 64 keys: the second half's TMEM load is
             // in flight while the first half is masked and reduced.
             float sA[kHalf], sB[kHalf];
@@ -653,7 +680,8 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             if (DOC || edge) {
                 #pragma unroll
                 for (int c = 0; c < kHalf; ++c)
-                    if (c >= c_hi || c < c_lo || (DOC && kd[c] != mydoc)) sA[c] = -INFINITY;
+                    if (c >= c_hi || (c < c_lo && c >= c_sink) || (DOC && kd[c] != mydoc))
+                        sA[c] = -INFINITY;
             }
             const float mA = row_max64(sA);
             // With the reference max unchanged (the common case under the
@@ -676,7 +704,8 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             if (DOC || edge) {
                 #pragma unroll
                 for (int c = 0; c < kHalf; ++c)
-                    if (c + kHalf >= c_hi || c + kHalf < c_lo || (DOC && kd[c + kHalf] != mydoc))
+                    if (c + kHalf >= c_hi || (c + kHalf < c_lo && c + kHalf >= c_sink) ||
+                        (DOC && kd[c + kHalf] != mydoc))
                         sB[c] = -INFINITY;
             }
             const float m_blk = fmaxf(mA, row_max64(sB)) * sl2;
@@ -805,11 +834,12 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
     }
 }
 
-template <int D, bool PAGED, bool DOC, bool F8>
+template <int D, bool PAGED, bool DOC, bool F8, bool SINK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const Params p) {
     static_assert(!F8 || (D == 128 && !PAGED && !DOC), "FP8: dense batches, d = 128");
+    static_assert(!SINK || (!PAGED && !DOC && !F8), "sink tokens: bf16 dense and packed batches");
     using C = Cfg<D, DOC, F8>;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Shared sh;
@@ -849,7 +879,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
     if (warp < kSoftmaxWarps) {
         regs_increase<kRegsSoftmax>();
-        softmax_wg<D, PAGED, DOC, F8>(p, sh,
+        softmax_wg<D, PAGED, DOC, F8, SINK>(p, sh,
                                       reinterpret_cast<int *>(sKV + C::kStages * C::kTileBytes));
     } else {
         regs_decrease<kRegsControl>();
@@ -857,9 +887,9 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if constexpr (PAGED)
                 producer_paged<D>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
             else if (lane_id() == 0)
-                producer<D, DOC, F8>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
+                producer<D, DOC, F8, SINK>(&tmQ, &tmK, &tmV, p, sh, sQ, sKV);
         } else if (warp == kWarpMma) {
-            if (lane_id() == 0) mma_issuer<D, PAGED, DOC, F8>(p, sh, sQ, sKV);
+            if (lane_id() == 0) mma_issuer<D, PAGED, DOC, F8, SINK>(p, sh, sQ, sKV);
         }
     }
     __syncwarp();
@@ -879,18 +909,18 @@ static_assert(Cfg<128, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared mem
 static_assert(Cfg<64, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 static_assert(Cfg<128, false, true>::kSmemBytes + sizeof(Shared) <= 232448, "shared memory");
 
-template <int D, bool PAGED, bool DOC, bool F8 = false>
+template <int D, bool PAGED, bool DOC, bool F8 = false, bool SINK = false>
 int launch_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                   const Params &p, long long units, cudaStream_t stream) {
     using C = Cfg<D, DOC, F8>;
     // Setting the attribute is idempotent and cheap; do it on every call so
     // that any device the caller switches to is covered.
-    if (cudaFuncSetAttribute(prefill_kernel<D, PAGED, DOC, F8>,
+    if (cudaFuncSetAttribute(prefill_kernel<D, PAGED, DOC, F8, SINK>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return -5;
     const int grid = (int)(units < device_sm_count() ? units : device_sm_count());
-    prefill_kernel<D, PAGED, DOC, F8><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+    prefill_kernel<D, PAGED, DOC, F8, SINK><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 
@@ -919,6 +949,7 @@ Params make_params(const PrefillArgs &a) {
     p.max_pages = a.max_pages;
     p.num_pages = a.num_pages;
     p.num_mblocks = (a.max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM);
+    p.n_sink = a.n_sink;
     return p;
 }
 
@@ -944,6 +975,8 @@ int launch_d(const PrefillArgs &a, cudaStream_t stream) {
     p.num_units = (int)units;
     if (a.paged) return launch_kernel<D, true, false>(tq, tk, tv, p, units, stream);
     if (a.doc) return launch_kernel<D, false, true>(tq, tk, tv, p, units, stream);
+    if (a.n_sink > 0 && a.causal && a.window > 0)
+        return launch_kernel<D, false, false, false, true>(tq, tk, tv, p, units, stream);
     return launch_kernel<D, false, false>(tq, tk, tv, p, units, stream);
 }
 

@@ -294,6 +294,19 @@ int fa_decode_paged_fp8(const void *q, const void *k_cache, const void *v_cache,
                         size_t workspace_bytes, void *stream);
 
 /*
+ * Causal sliding-window prefill that keeps the first n_sink tokens of every
+ * sequence visible (samanvya.dev "Attention Is the Bottleneck", "Sliding
+ * windows and local:global layers": StreamingLLM's sink tokens plus a recent
+ * window).  Key j is visible from query i if j <= i and (j > i - window or
+ * j < n_sink).  Dense batches as fa_fwd, always causal; window >= 1 (else
+ * FA_ERR_INVALID_ARG), n_sink >= 0 (0: fa_fwd with the window).  Arguments,
+ * layouts, alignment and errors as fa_fwd.
+ */
+int fa_fwd_sink_tokens(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int N, int d, int window, int n_sink,
+                       float scale, int o_dtype, void *stream);
+
+/*
  * FP8 prefill with incoherent processing ("FlashAttention-3" in samanvya.dev
  * "Attention Is the Bottleneck", "FlashAttention: same math, different IO":
  * Q and K multiplied by a random orthogonal Hadamard matrix before FP8

@@ -278,6 +278,17 @@ def test_fwd_fp8_empty_is_noop(fa):
     assert fwd8(fa, N=0, q8=0) == 0
 
 
+def test_fwd_sink_tokens_rejects(fa):
+    lib = fa.library()
+    ok = [P, P, P, P, 0, 1, 4, 2, 300, 128]
+    assert lib.fa_fwd_sink_tokens(*ok, 0, 4, 0.1, 0, None) == -1        # no window
+    assert lib.fa_fwd_sink_tokens(*ok, 64, -1, 0.1, 0, None) == -1      # negative sinks
+    assert lib.fa_fwd_sink_tokens(P, P, P, P, 0, 1, 3, 2, 300, 128, 64, 4, 0.1, 0, None) == -1
+    assert lib.fa_fwd_sink_tokens(P, P, P, P, 0, 1, 4, 2, 300, 96, 64, 4, 0.1, 0, None) == -2
+    assert lib.fa_fwd_sink_tokens(P + 8, P, P, P, 0, 1, 4, 2, 300, 128, 64, 4, 0.1, 0, None) == -3
+    assert lib.fa_fwd_sink_tokens(0, P, P, P, 0, 0, 4, 2, 300, 128, 64, 4, 0.1, 0, None) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """Importing the binding with the shared library absent raises, rather
     than falling back to anything else."""
