@@ -124,17 +124,44 @@ def kernel_source_hash():
     return h.hexdigest()[:12]
 
 
-def recorded_traffic():
-    """DRAM bytes per launch from the committed ncu summary, keyed by kernel
-    source hash; None when the kernels changed since the capture."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+# The sources each recorded kernel is built from (its own file, the PTX
+# wrappers, and for the FP8 preparation the argument struct it takes).
+TRAFFIC_FAMILIES = {
+    "prefill": ("prefill_sm100.cu", "sm100.cuh"),
+    "decode": ("decode_sm100.cu", "sm100.cuh"),
+    "bwd": ("bwd_sm100.cu", "sm100.cuh"),
+    "fp8_prepare": ("fp8_prep.cu", "sm100.cuh", "fa_internal.h"),
+}
+
+
+def family_of(key):
+    for fam in ("fp8_prepare", "prefill", "decode", "bwd"):
+        if key.startswith(fam):
+            return fam
+    return None
+
+
+def family_hash(fam):
+    h = hashlib.sha256()
+    for f in TRAFFIC_FAMILIES[fam]:
+        h.update(open(os.path.join(ROOT, "exact_io_aware_75_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(path=None):
+    """DRAM bytes per launch from the committed ncu summary; a line counts
+    only while the sources its kernel is built from hash as they did at the
+    capture (otherwise the kernel's traffic is None)."""
+    path = path or os.path.join(ROOT, "profiles", "dram_traffic.txt")
     out = {}
     if not os.path.exists(path):
         return out
-    want = kernel_source_hash()
     for line in open(path):
         parts = line.split()
-        if len(parts) >= 4 and not line.startswith("#") and parts[1] == want:
+        if len(parts) < 4 or line.startswith("#"):
+            continue
+        fam = family_of(parts[0])
+        if fam is not None and parts[1] == family_hash(fam):
             out[parts[0]] = float(parts[3])
     return out
 
