@@ -15,7 +15,9 @@
  * Conventions shared by every call
  *   - q, k, v, o, caches: bf16 (o optionally fp32), innermost dimension
  *     contiguous, token-major:  dense [B, N, H, d], packed [total, H, d],
- *     cache [num_pages, page_size, Hkv, d].
+ *     cache [num_pages, page_size, Hkv, d].  The FP8 calls
+ *     (fa_decode_paged_fp8, fa_fp8_prepare, fa_fwd_fp8) take E4M3 codes with
+ *     fp32 scales instead; their comments give the layouts.
  *   - GQA ("MQA and GQA"): query head h reads KV head h / (Hq / Hkv);
  *     Hq must be a multiple of Hkv; Hkv == 1 is MQA.
  *   - Masks: causal (key j visible from query i iff j <= i; "every token can
