@@ -39,7 +39,7 @@ FA_OUT_BF16 = 0
 FA_OUT_FP32 = 1
 
 EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa_fwd_paged",
-           "fa_fwd_doc", "fa_fwd_sink_tokens",
+           "fa_fwd_doc", "fa_fwd_sink_tokens", "fa_fwd_varlen_sink_tokens",
            "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_varlen", "fa_bwd_sinks",
            "fa_bwd_varlen_sinks",
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
@@ -73,6 +73,8 @@ def _load():
     lib.fa_decode_paged_sinks.restype = i
     lib.fa_fwd_sink_tokens.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp]
     lib.fa_fwd_sink_tokens.restype = i
+    lib.fa_fwd_varlen_sink_tokens.argtypes = [vp] * 6 + [i] * 8 + [f, i, vp]
+    lib.fa_fwd_varlen_sink_tokens.restype = i
     lib.fa_fwd_doc.argtypes = [vp] * 6 + [i] * 7 + [f, i, vp]
     lib.fa_fwd_doc.restype = i
     lib.fa_fwd_paged.argtypes = [vp] * 9 + [i] * 11 + [f, i, vp]
@@ -273,9 +275,10 @@ def fwd_fp8(prep, causal=False, window=0, scale=None, out_dtype=torch.bfloat16, 
 
 def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=None,
                out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None,
-               sinks=None):
+               sinks=None, sink_tokens=None):
     """Packed prefill.  q [T,Hq,d], k/v [T,Hkv,d], cu_seqlens [S+1] int32 (device)
-    -> (O [T,Hq,d], LSE [Hq,T])."""
+    -> (O [T,Hq,d], LSE [Hq,T]).  ``sinks`` selects fa_fwd_varlen_sinks;
+    ``sink_tokens`` (an int, with causal and a window) fa_fwd_varlen_sink_tokens."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, 3, n)
     _need(cu_seqlens, torch.int32, 1, "cu_seqlens")
@@ -288,6 +291,15 @@ def fwd_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, window=0, scale=No
     if lse is None and return_lse:
         lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
     od = FA_OUT_FP32 if out.dtype == torch.float32 else FA_OUT_BF16
+    if sink_tokens is not None:
+        if sinks is not None or not causal:
+            raise FAError(FA_ERR_UNSUPPORTED, "sink_tokens with sinks or non-causal")
+        _check(_lib.fa_fwd_varlen_sink_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                              _ptr(cu_seqlens), cu_seqlens.numel() - 1, T,
+                                              int(max_seqlen), Hq, Hkv, d, int(window),
+                                              int(sink_tokens), float(scale), od,
+                                              _stream(stream)), "fa_fwd_varlen_sink_tokens")
+        return out, lse
     if sinks is not None:
         _need(sinks, torch.float32, 1, "sinks")
         _check(_lib.fa_fwd_varlen_sinks(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),

@@ -159,7 +159,7 @@ int fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
 int fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
                const float *sinks, const int *cu_seqlens, int num_seqs, int total_tokens,
                int max_seqlen, int Hq, int Hkv, int d, int causal, int window, float scale,
-               int o_dtype, void *stream) {
+               int o_dtype, void *stream, int n_sink = 0) {
     if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return FA_ERR_INVALID_ARG;
     int rc = check_common(Hq, Hkv, d, causal, window, scale, o_dtype);
     if (rc) return rc;
@@ -183,6 +183,7 @@ int fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
     a.scale = scale;
     a.o_fp32 = o_dtype == FA_OUT_FP32;
     a.sinks = sinks;
+    a.n_sink = n_sink;
     return map_rc(fa::launch_prefill(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -203,6 +204,15 @@ int fa_fwd_sink_tokens(const void *q, const void *k, const void *v, void *o, flo
     if (window <= 0 || n_sink < 0) return FA_ERR_INVALID_ARG;
     return fwd_dense(q, k, v, o, lse, nullptr, B, Hq, Hkv, N, d, 1, window, scale, o_dtype,
                      stream, nullptr, n_sink);
+}
+
+int fa_fwd_varlen_sink_tokens(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int *cu_seqlens, int num_seqs, int total_tokens,
+                              int max_seqlen, int Hq, int Hkv, int d, int window, int n_sink,
+                              float scale, int o_dtype, void *stream) {
+    if (window <= 0 || n_sink < 0) return FA_ERR_INVALID_ARG;
+    return fwd_varlen(q, k, v, o, lse, nullptr, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                      Hq, Hkv, d, 1, window, scale, o_dtype, stream, n_sink);
 }
 
 int fa_fwd_sinks(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -308,6 +308,13 @@ int fa_fwd_sink_tokens(const void *q, const void *k, const void *v, void *o, flo
                        int B, int Hq, int Hkv, int N, int d, int window, int n_sink,
                        float scale, int o_dtype, void *stream);
 
+/* The same for packed sequences (layouts as fa_fwd_varlen); the sink tokens
+ * are the first n_sink tokens of each sequence. */
+int fa_fwd_varlen_sink_tokens(const void *q, const void *k, const void *v, void *o, float *lse,
+                              const int *cu_seqlens, int num_seqs, int total_tokens,
+                              int max_seqlen, int Hq, int Hkv, int d, int window, int n_sink,
+                              float scale, int o_dtype, void *stream);
+
 /*
  * FP8 prefill with incoherent processing ("FlashAttention-3" in samanvya.dev
  * "Attention Is the Bottleneck", "FlashAttention: same math, different IO":

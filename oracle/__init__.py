@@ -478,6 +478,24 @@ def attn_sink_tokens(q, k, v, window, n_sink, scale=None, rows=None):
     return o.reshape(B, N, Hq, d), np.ascontiguousarray(lse.reshape(B, N, Hq).transpose(0, 2, 1))
 
 
+def attn_varlen_sink_tokens(q, k, v, cu_seqlens, window, n_sink, scale=None):
+    """Packed sequences with a causal window that keeps each sequence's first
+    n_sink tokens visible: q [T,Hq,d], k/v [T,Hkv,d] -> O [T,Hq,d], LSE [Hq,T]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((T, Hq, d), np.float64)
+    lse = np.empty((T, Hq), np.float64)
+    _check(lib().oracle_attn_varlen_rows_sink_tokens(qb, kb, vb, cu, cu.size - 1, Hq, Hkv, d,
+                                                     int(window), int(n_sink), float(scale),
+                                                     None, T, o, lse),
+           "attn_varlen_sink_tokens")
+    return o, np.ascontiguousarray(lse.T)
+
+
 # ---------------------------------------------------------------- FP8 prefill
 # Incoherent processing ("FlashAttention-3", samanvya.dev "Attention Is the
 # Bottleneck"): Q and K rotated by diag(signs) H / sqrt(d) (H Sylvester

@@ -289,6 +289,19 @@ def test_fwd_sink_tokens_rejects(fa):
     assert lib.fa_fwd_sink_tokens(0, P, P, P, 0, 0, 4, 2, 300, 128, 64, 4, 0.1, 0, None) == 0
 
 
+def test_fwd_varlen_sink_tokens_rejects(fa):
+    lib = fa.library()
+    ok = [P, P, P, P, 0, P, 3, 600, 300, 4, 2, 128]
+    assert lib.fa_fwd_varlen_sink_tokens(*ok, 0, 4, 0.1, 0, None) == -1      # no window
+    assert lib.fa_fwd_varlen_sink_tokens(*ok, 64, -2, 0.1, 0, None) == -1    # negative sinks
+    bad_cu = [P, P, P, P, 0, 0, 3, 600, 300, 4, 2, 128]
+    assert lib.fa_fwd_varlen_sink_tokens(*bad_cu, 64, 4, 0.1, 0, None) == -1
+    mis_cu = [P, P, P, P, 0, P + 2, 3, 600, 300, 4, 2, 128]
+    assert lib.fa_fwd_varlen_sink_tokens(*mis_cu, 64, 4, 0.1, 0, None) == -3
+    assert lib.fa_fwd_varlen_sink_tokens(P, P, P, P, 0, P, 0, 0, 0, 4, 2, 128, 64, 4, 0.1, 0,
+                                         None) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     """Importing the binding with the shared library absent raises, rather
     than falling back to anything else."""

@@ -65,3 +65,18 @@ def test_sink_tokens_long32k_sampled_rows(fa):
     o_ref, lse_ref = oracle.attn_sink_tokens(inp.q, inp.k, inp.v, inp.window, 4, inp.scale,
                                              rows=[(0, r) for r in rows])
     compare(o[0, rows], o_ref, lse[0][:, rows].T, lse_ref, "long32k_w4096 + 4 sink tokens")
+
+
+@pytest.mark.parametrize("W,S", [(64, 4), (200, 130)])
+def test_packed_sequences_match_oracle(fa, W, S):
+    """fa_fwd_varlen_sink_tokens: each sequence keeps its own first tokens."""
+    inp = workloads.varlen(lens=[300, 0, 517, 1, 129, 1000], Hq=8, Hkv=2, d=128, causal=True,
+                           seed=W + S)
+    cu = inp.cu_seqlens.cuda()
+    o, lse = fa.fwd_varlen(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), cu, inp.max_seqlen, True,
+                           W, inp.scale, out_dtype=torch.float32, sink_tokens=S)
+    torch.cuda.synchronize()
+    assert fa.check_device_error() == 0
+    o_ref, lse_ref = oracle.attn_varlen_sink_tokens(inp.q, inp.k, inp.v, inp.cu_seqlens, W, S,
+                                                    inp.scale)
+    compare(o, o_ref, lse, lse_ref, f"packed sink tokens W={W} S={S}")

@@ -70,3 +70,19 @@ def test_reductions_to_window_and_causal():
     for W, S in ((6, N), (N, 3)):
         d_ = oracle.attn_sink_tokens(q, k, v, W, S, 0.25)
         assert all(np.array_equal(x, y) for x, y in zip(d_, c))
+
+
+def test_packed_sequences_are_per_sequence():
+    """Packed form: each sequence's rows equal the pinned dense form on that
+    sequence alone (sink tokens are each sequence's own first tokens)."""
+    lens = [70, 0, 130, 5]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    q, k, v = rnd((T, 4, 16), 11), rnd((T, 2, 16), 12), rnd((T, 2, 16), 13)
+    o, lse = oracle.attn_varlen_sink_tokens(q, k, v, cu, 9, 3, 0.3)
+    for s, L in enumerate(lens):
+        if L == 0:
+            continue
+        a, b = int(cu[s]), int(cu[s + 1])
+        ro, rl = oracle.attn_sink_tokens(q[None, a:b], k[None, a:b], v[None, a:b], 9, 3, 0.3)
+        assert np.array_equal(o[a:b], ro[0]) and np.array_equal(lse[:, a:b], rl[0])
