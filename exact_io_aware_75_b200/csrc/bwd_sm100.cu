@@ -5,8 +5,8 @@
 // gradient dO, the gradients of sum(dO * O) with respect to Q, K and V.  The
 // attention matrix is never stored: it is recomputed from Q, K and the row
 // log-sum-exp the forward saved ("FlashAttention: same math, different IO" in
-// samanvya.dev's "Attention Is the Bottleneck": the backward pass recomputes
-// the matrix from Q, K, V and the saved softmax statistics).  With
+// samanvya.dev's "Attention Is the Bottleneck": the backward rebuilds the
+// matrix instead of keeping it, trading FLOPs for memory traffic).  With
 // D_i = dO_i . O_i, for each visible (query i, key j):
 //     P_ij  = 2^(S_ij * scale * log2e - LSE_i * log2e)
 //     dS_ij = P_ij (dO_i . V_j - D_i)

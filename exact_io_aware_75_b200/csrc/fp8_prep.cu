@@ -1,10 +1,10 @@
 // fp8_prep.cu -- operands of the FP8 prefill.
 //
 // What it computes ("FlashAttention-3" in samanvya.dev's "Attention Is the
-// Bottleneck", "FlashAttention: same math, different IO": Q and K are
-// multiplied by a random orthogonal Hadamard matrix before FP8 quantisation,
-// which spreads outlier channels over all dimensions; "Low precision" in the
-// same post: FP8 GEMMs carry per-block scales):
+// Bottleneck", "FlashAttention: same math, different IO": a random orthogonal
+// Hadamard transform of Q and K ahead of FP8 quantisation spreads outlier
+// channels over all dimensions; Ales Analytics "Attention and matrix kernels",
+// "How it works": FP8 GEMMs carry a scale per block):
 //   Q' = Q diag(signs) H / sqrt(d), K' = K diag(signs) H / sqrt(d), with H
 //   the Sylvester Hadamard matrix and signs a random +-1 per channel given by
 //   the caller, so Q' K'^T = Q K^T.  Q' and K' become E4M3 codes with one

@@ -22,7 +22,7 @@
  *     Hq must be a multiple of Hkv; Hkv == 1 is MQA.
  *   - Masks: causal (key j visible from query i iff j <= i; "every token can
  *     see every earlier token"), sliding window W > 0 (with causal only: keys
- *     i-W+1 .. i, i.e. the last W tokens including the query itself;
+ *     i-W+1 .. i, i.e. W keys ending at the query itself;
  *     "Sliding windows and local:global layers").  window <= 0: no window.
  *   - LSE is natural-log, in units of scaled scores; a row with no visible
  *     key (only possible for an empty sequence) has O = 0 and LSE = -inf.
@@ -100,9 +100,9 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                   float scale, int o_dtype, void *stream);
 
 /*
- * Chunked prefill over a paged cache ("Chunked-prefill serving in vLLM pairs
- * FlashAttention with KV paging", FlashAttention explainer, real-world
- * examples).  Sequence s has seq_lens_k[s] tokens in its pages -- the earlier
+ * Chunked prefill over a paged cache (zenaique's FlashAttention serving
+ * explainer, "Real-world examples": serving engines run long prompts in chunks
+ * over a paged KV cache with this kernel).  Sequence s has seq_lens_k[s] tokens in its pages -- the earlier
  * context plus this chunk, whose K/V the caller has already written -- and
  * its L_q = cu_seqlens_q[s+1] - cu_seqlens_q[s] queries are the LAST L_q of
  * them: query i of the chunk sits at position seq_lens_k[s] - L_q + i and,
@@ -175,9 +175,9 @@ int fa_fwd_varlen_sinks(const void *q, const void *k, const void *v, void *o, fl
  * Backward of dense prefill: the gradients of sum(dO * O) with respect to Q,
  * K and V, for O = fa_fwd(q, k, v, ...) with the same mask and scale.  The
  * attention matrix is recomputed tile by tile from Q, K and the LSE the
- * forward saved, never stored ("What attention costs", the FlashAttention
- * paragraph: the backward pass recomputes the matrix from Q, K, V and the
- * saved softmax statistics).  With grouped heads, dK and dV of a KV head sum
+ * forward saved, never stored (samanvya.dev "Attention Is the Bottleneck",
+ * "FlashAttention: same math, different IO": the backward rebuilds the
+ * matrix rather than keeping it).  With grouped heads, dK and dV of a KV head sum
  * over the query heads that read it.
  *   q, o, dout [B, N, Hq, d]  bf16, device (o as written by fa_fwd)
  *   k, v       [B, N, Hkv, d] bf16, device
@@ -319,7 +319,8 @@ int fa_fwd_varlen_sink_tokens(const void *q, const void *k, const void *v, void 
  * FP8 prefill with incoherent processing ("FlashAttention-3" in samanvya.dev
  * "Attention Is the Bottleneck", "FlashAttention: same math, different IO":
  * Q and K multiplied by a random orthogonal Hadamard matrix before FP8
- * quantisation; "Low precision" in the same post: per-block scales).  Two
+ * quantisation; Ales Analytics "Attention and matrix kernels", "How it
+ * works": FP8 GEMMs carry a scale per block).  Two
  * calls: fa_fp8_prepare makes the E4M3 operands from bf16 Q, K, V, and
  * fa_fwd_fp8 runs the attention on them.  Dense batches, d = 128.
  *

@@ -16,14 +16,14 @@
  *   The score row is materialised in full, one query row at a time.
  *
  *   LSE_i = M_i + log(l_i) in natural log, M_i = max_j S_ij,
- *   l_i = sum_j exp(S_ij - M_i): the "saved softmax statistics" the same post
- *   names for the backward pass.
+ *   l_i = sum_j exp(S_ij - M_i): the per-row softmax statistics the same post
+ *   says the backward keeps instead of the matrix.
  *
  * Allowed key sets A(i) (readings of the pages, each stated once here):
  *   non-causal : every key of the same sequence;
- *   causal     : keys j <= i ("every token can see every earlier token",
- *                "Attending to fewer tokens");
- *   window W>0 : causal and j > i - W, i.e. the last W tokens including the
+ *   causal     : keys j <= i (full causal attention: each token attends to
+ *                all tokens before it, "Attending to fewer tokens");
+ *   window W>0 : causal and j > i - W, i.e. the W keys ending at the
  *                token itself ("Sliding windows and local:global layers");
  *   decode     : the one query is the sequence's last token and sees all of
  *                its seq_len keys, gathered page by page through the block
@@ -243,7 +243,8 @@ int oracle_attn_varlen_rows(const uint16_t *q, const uint16_t *k, const uint16_t
  * The same with a learned sink logit per query head, sinks[Hq] (in units of
  * scaled scores), joining every row's softmax denominator as the score of
  * one extra key with a zero value ("Sliding windows and local:global
- * layers": gpt-oss's learned sink per head).  LSE includes the sink's term.
+ * layers": gpt-oss builds a learned sink into every head).  LSE includes the
+ * sink's term.
  */
 int oracle_attn_varlen_rows_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                   const int32_t *cu_seqlens, int num_seqs,
@@ -277,8 +278,8 @@ int oracle_attn_varlen_rows_doc(const uint16_t *q, const uint16_t *k, const uint
 
 /*
  * Sink tokens with a sliding window ("Sliding windows and local:global
- * layers": StreamingLLM keeps a handful of sink tokens plus a recent
- * window): with causal and window W > 0, key j is visible from query i if
+ * layers": StreamingLLM retains the first few tokens as sinks beside the
+ * recent window): with causal and window W > 0, key j is visible from query i if
  * j <= i and (j > i - W or j < n_sink) -- the first n_sink tokens of each
  * sequence stay visible to every later query.  Otherwise as
  * oracle_attn_varlen_rows.
@@ -459,9 +460,9 @@ int oracle_lse_combine(const double *o_parts, const double *lse_parts,
 }
 
 /*
- * Backward of packed-sequence attention (the gradients the backward pass
- * recomputes from Q, K, V and the saved statistics; "What attention costs",
- * the FlashAttention paragraph on not storing the attention matrix).  The
+ * Backward of packed-sequence attention (the backward rebuilds the attention
+ * matrix from the inputs and the forward's row statistics rather than
+ * storing it: "FlashAttention: same math, different IO").  The
  * pages give no formulas; these are the chain rule through the definition
  * above, with the upstream gradient dO = dLoss/dO:
  *   P_ij  = softmax_j(S_ij) over A(i)           (two-pass, as attend_row)
@@ -697,8 +698,8 @@ int oracle_attn_bwd_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t
 }
 
 /*
- * FP8 KV cache ("FP8 KV cache is a routine flag": the "Paging and prefix
- * sharing" neighbourhood of the same post stores the cache in fewer bits).
+ * FP8 KV cache ("Quantize what's left" in the same post: serving engines
+ * commonly store the cache in 8 bits).
  * Codes are OCP FP8 E4M3 in its "fn" form (no infinities): sign bit, 4
  * exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
  * subnormals m/8 * 2^-6; S.1111.111 is NaN.  A cached value is
@@ -808,9 +809,9 @@ int oracle_decode_paged_fp8(const uint16_t *q, const uint8_t *k_cache, const uin
 }
 
 /*
- * Chunked prefill over a paged cache ("Chunked-prefill serving ... pairs
- * FlashAttention with KV paging", FlashAttention explainer, real-world
- * examples): sequence s has seq_lens_k[s] tokens in its pages (earlier
+ * Chunked prefill over a paged cache (zenaique's FlashAttention serving
+ * explainer, "Real-world examples": serving engines run long prompts in
+ * chunks over a paged KV cache): sequence s has seq_lens_k[s] tokens in its pages (earlier
  * context plus this chunk's own keys), and its L_q = cu_seqlens_q[s+1] -
  * cu_seqlens_q[s] new query tokens are the last L_q of them: query i of the
  * chunk sits at position seq_lens_k[s] - L_q + i (the causal reading that
@@ -882,11 +883,11 @@ int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_cache, const uint1
 
 /*
  * FP8 prefill with incoherent processing ("FlashAttention-3" in the
- * "FlashAttention: same math, different IO" part of samanvya.dev's post: Q
- * and K are multiplied by a random orthogonal Hadamard matrix before E4M3
- * quantisation, which spreads outlier channels over all dimensions; "Low
- * precision" in the same post's introduction: FP8 GEMMs carry per-block
- * scales).  Readings, where the pages leave the step open:
+ * "FlashAttention: same math, different IO" part of samanvya.dev's post: a
+ * random orthogonal Hadamard transform of Q and K ahead of E4M3 quantisation
+ * spreads outlier channels over all dimensions; Ales Analytics "Attention and
+ * matrix kernels", "How it works": FP8 GEMMs carry a scale per block).
+ * Readings, where the pages leave the step open:
  *   - the orthogonal matrix is M = D H / sqrt(d): D = diag(signs), a random
  *     +-1 per channel drawn by the caller, H the Sylvester Hadamard matrix of
  *     order d (a power of two), entry (k, c) = (-1)^popcount(k & c).  Both Q

@@ -1,8 +1,9 @@
 """Pins for the oracle's attention backward (dQ, dK, dV for an upstream dO).
 
-The pages state only that the backward pass recomputes the attention matrix
-from Q, K, V and the saved softmax statistics (samanvya.dev "Attention Is the
-Bottleneck", "FlashAttention: same math, different IO"); the gradients
+The pages state only that the backward rebuilds the attention matrix from
+the inputs and the forward's row statistics rather than storing it
+(samanvya.dev "Attention Is the Bottleneck", "FlashAttention: same math,
+different IO"); the gradients
 themselves are fixed by calculus.  Pins, none produced by the oracle:
   - hand-worked gradients of the two-key case (tests/golden);
   - torch's automatic differentiation, in fp64, of the forward definition

@@ -1,11 +1,11 @@
 """Pins for the oracle's FP8 prefill with incoherent processing.
 
-The pages say only that Q and K are multiplied by a random orthogonal
-(Hadamard) matrix before FP8 quantisation, which spreads outliers and cut the
-error of FP8 attention 2.6x against plain FP8 (samanvya.dev "Attention Is the
-Bottleneck", "FlashAttention: same math, different IO", FlashAttention-3), and
-that FP8 GEMMs carry per-block scales (same post, introduction, "Low
-precision").  Pins, none produced by the oracle itself:
+The pages say only that a random orthogonal (Hadamard) transform of Q and K
+ahead of FP8 quantisation spreads outliers and lowered the error of FP8
+attention 2.6x against plain FP8 (samanvya.dev "Attention Is the Bottleneck",
+"FlashAttention: same math, different IO", FlashAttention-3), and that FP8
+GEMMs carry a scale per block (Ales Analytics "Attention and matrix kernels",
+"How it works").  Pins, none produced by the oracle itself:
   - the rotation against scipy's Hadamard matrix (a library routine) and the
     invariants of an orthogonal map (norms and Q.K dot products kept);
   - E4M3 rounding against torch's float8_e4m3fn cast (a library routine) and

@@ -1,6 +1,6 @@
-"""Pins for the oracle's chunked prefill over a paged cache (FlashAttention
-explainer, real-world examples: chunked-prefill serving pairs FlashAttention
-with KV paging).  The reading: a chunk's L_q queries are the last L_q of the
+"""Pins for the oracle's chunked prefill over a paged cache (zenaique's
+FlashAttention serving explainer, "Real-world examples": serving engines run
+long prompts in chunks over a paged KV cache).  The reading: a chunk's L_q queries are the last L_q of the
 sequence's seq_lens_k cached tokens.  Pins reduce it to the pinned dense
 definition: the chunk's rows equal the last rows of full causal attention over
 the whole sequence, whatever the page permutation; L_q = 1 is the decode."""

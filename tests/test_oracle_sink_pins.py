@@ -1,8 +1,8 @@
 """Pins for the oracle's learned attention sink: a per-head logit z_h that
 joins every row's softmax denominator as the score of one extra key whose
 value is zero (samanvya.dev "Attention Is the Bottleneck", "Sliding windows
-and local:global layers": gpt-oss's learned sink per head; the page gives no
-formula, this is the plain reading).  Pins, none produced by the oracle:
+and local:global layers": gpt-oss builds a learned sink into every head; the
+page gives no formula, this is the plain reading).  Pins, none produced by the oracle:
   - z = -inf is plain attention, bit for bit;
   - z equals a real extra key with score z and a zero value, built from the
     plain (pinned) oracle on an augmented input;

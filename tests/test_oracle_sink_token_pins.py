@@ -1,7 +1,8 @@
 """Pins for the oracle's sink tokens: a sliding window of W keys that also
 keeps the first n_sink tokens of each sequence visible (samanvya.dev
 "Attention Is the Bottleneck", "Sliding windows and local:global layers":
-StreamingLLM keeps a handful of sink tokens plus a recent window).  Pins, none
+StreamingLLM retains the first few tokens as sinks beside the recent
+window).  Pins, none
 produced by the oracle itself:
   - torch's softmax in fp64 over the explicitly masked score matrix (a
     library routine for the definition);
