@@ -154,7 +154,7 @@ int fa_fwd_doc(const void *q, const void *k, const void *v, void *o, float *lse,
 
 /*
  * fa_fwd / fa_fwd_varlen with a learned attention sink per query head
- * ("Sliding windows and local:global layers": gpt-oss's learned sink per
+ * ("Sliding windows and local:global layers": gpt-oss builds one into every
  * head).  sinks [Hq] fp32, device, in units of scaled scores: z_h joins every
  * row's softmax denominator as the score of one extra key whose value is
  * zero, so O_i = sum_j e^(s_ij) V_j / (e^(z_h) + sum_j e^(s_ij)) and LSE
