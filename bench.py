@@ -243,7 +243,8 @@ def oracle_sample(inp, target_s, cores, name=PREFILL):
     full = prefill_flops(B, Hq, N, d, True, inp.window)
     stride = max(1, int(math.ceil(full / max(rate * target_s, 1.0))))
     fl, dt, nrows = run(stride, stride - 1)
-    desc = (f"{nrows} query rows (every {stride}th, all {Hq} heads) of the {name} workload, "
+    which = "every row" if stride == 1 else f"every {stride}th row"
+    desc = (f"{nrows} query rows ({which}, all {Hq} heads) of the {name} workload, "
             f"{fl / 1e9:.1f} GFLOP in {dt:.1f} s")
     return fl / dt / 1e12, desc, dt
 
