@@ -89,6 +89,10 @@ def lib():
             _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, _i64p, ctypes.c_int64, _f64p]
         L.oracle_attn_bwd_dq_rows.restype = ctypes.c_int
+        L.oracle_attn_bwd_dkv_rows.argtypes = [
+            _u16p, _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, _i64p, ctypes.c_int64, _f64p, _f64p]
+        L.oracle_attn_bwd_dkv_rows.restype = ctypes.c_int
         L.oracle_attn_varlen_rows_sink_tokens.argtypes = [
             _u16p, _u16p, _u16p, _i32p] + [ctypes.c_int] * 6 + [
             ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, _f64p, _f64p]
@@ -283,6 +287,25 @@ def attn_bwd_dq_rows(q, k, v, dout, cu_seqlens, rows, causal=False, window=0, sc
                                          int(causal), int(window), float(scale), r, r.size, dq),
            "attn_bwd_dq_rows")
     return dq
+
+
+def attn_bwd_dkv_rows(q, k, v, dout, cu_seqlens, rows, causal=False, window=0, scale=None):
+    """dK and dV of the packed key tokens ``rows`` only (all KV heads)
+    -> ([R, Hkv, d], [R, Hkv, d]): the sums over the query rows that see each
+    key, from every row's LSE and D = rowsum(P * dP) taken first."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    T, Hq, d = qb.shape
+    Hkv = kb.shape[1]
+    cu = _i32(cu_seqlens)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dk = np.empty((r.size, Hkv, d), np.float64)
+    dv = np.empty((r.size, Hkv, d), np.float64)
+    _check(lib().oracle_attn_bwd_dkv_rows(qb, kb, vb, db, cu, len(cu) - 1, Hq, Hkv, d,
+                                          int(causal), int(window), float(scale), r, r.size,
+                                          dk, dv), "attn_bwd_dkv_rows")
+    return dk, dv
 
 
 def attn_varlen_sinks(q, k, v, cu_seqlens, sinks, causal=False, window=0, scale=None, rows=None):

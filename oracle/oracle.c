@@ -37,7 +37,7 @@
  *   O = sum_s w_s O_s / sum_s w_s.
  *
  * Further functions, each with its reading stated where it is defined:
- *   - oracle_attn_bwd_varlen (+ _sinks, _dq_rows): the gradients dQ, dK, dV
+ *   - oracle_attn_bwd_varlen (+ _sinks, _dq_rows, _dkv_rows): the gradients dQ, dK, dV
  *     (and of the sink logits) by the chain rule through the definition;
  *   - the learned sink logit per head (the _sinks variants): one more score
  *     in the denominator with a zero value;
@@ -695,6 +695,126 @@ int oracle_attn_bwd_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t
         free(kp); free(vp); free(vis);
     }
     return bad ? -2 : 0;
+}
+
+/*
+ * dK and dV of selected key tokens only (every KV head): rows[r] is a packed
+ * token index; dk, dv [nrows, Hkv, d].  The same chain rule as the full
+ * backward, summed per key instead of scattered per query:
+ *   dV_j = sum_{h in group} sum_{i : j in A(i)} P_ij dO_i,
+ *   dK_j = scale sum_{h in group} sum_{i : j in A(i)} dS_ij Q_i,
+ *   P_ij = exp(S_ij - LSE_i),  dS_ij = P_ij (dO_i . V_j - D_i),
+ * with LSE_i and D_i = sum_j P_ij (dO_i . V_j) of every query row (token,
+ * query head) taken first from bwd_row over the row's whole allowed set.
+ * The second pass sums over query heads, then query rows, in ascending order.
+ */
+int oracle_attn_bwd_dkv_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *dout, const int32_t *cu_seqlens, int num_seqs,
+                             int Hq, int Hkv, int d, int causal, int window, double scale,
+                             const int64_t *rows, int64_t nrows, double *dk, double *dv)
+{
+    if (Hq <= 0 || Hkv <= 0 || d <= 0 || Hq % Hkv != 0 || num_seqs < 0 || nrows < 0) return -1;
+    const int group = Hq / Hkv;
+    const int64_t total = cu_seqlens[num_seqs];
+    int64_t maxlen = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t L = (int64_t)cu_seqlens[s + 1] - cu_seqlens[s];
+        if (L < 0) return -1;
+        if (L > maxlen) maxlen = L;
+    }
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return -1;
+    /* row statistics of every (token, query head) */
+    double *lse = (double *)malloc(sizeof(double) * (size_t)(total > 0 ? total : 1) * Hq);
+    double *Dr = (double *)malloc(sizeof(double) * (size_t)(total > 0 ? total : 1) * Hq);
+    if (!lse || !Dr) {
+        free(lse); free(Dr);
+        return -2;
+    }
+    int bad = 0;
+#pragma omp parallel
+    {
+        size_t n = (size_t)(maxlen > 0 ? maxlen : 1);
+        double *sc = (double *)malloc(sizeof(double) * n);
+        double *p = (double *)malloc(sizeof(double) * n);
+        double *dp = (double *)malloc(sizeof(double) * n);
+        double *ds = (double *)malloc(sizeof(double) * n);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dod = (double *)malloc(sizeof(double) * (size_t)d);
+        double *orow = (double *)malloc(sizeof(double) * (size_t)d);
+        double *dqs = (double *)malloc(sizeof(double) * (size_t)d);
+        const uint16_t **kp = (const uint16_t **)malloc(sizeof(void *) * n);
+        const uint16_t **vp = (const uint16_t **)malloc(sizeof(void *) * n);
+        unsigned char *vis = (unsigned char *)malloc(n);
+        if (!sc || !p || !dp || !ds || !qd || !dod || !orow || !dqs || !kp || !vp || !vis) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t task = 0; task < total * (int64_t)Hq; ++task) {
+                int64_t t = task / Hq;
+                int h = (int)(task % Hq), g = h / group;
+                int seq = 0;
+                while (seq < num_seqs && cu_seqlens[seq + 1] <= t) ++seq;
+                int64_t start = cu_seqlens[seq];
+                int64_t L = (int64_t)cu_seqlens[seq + 1] - start, i = t - start;
+                const int64_t row = (t * Hq + h) * (int64_t)d;
+                for (int c = 0; c < d; ++c) {
+                    qd[c] = widen(q[row + c]);
+                    dod[c] = widen(dout[row + c]);
+                }
+                for (int64_t j = 0; j < L; ++j) {
+                    kp[j] = k + ((start + j) * Hkv + g) * (int64_t)d;
+                    vp[j] = v + ((start + j) * Hkv + g) * (int64_t)d;
+                    vis[j] = (unsigned char)allowed(i, j, causal, window);
+                }
+                bwd_row(qd, dod, d, L, kp, vp, vis, scale, -INFINITY, sc, p, dp, ds, orow,
+                        dqs, lse + task, Dr + task);
+            }
+        }
+        free(sc); free(p); free(dp); free(ds); free(qd); free(dod); free(orow); free(dqs);
+        free(kp); free(vp); free(vis);
+    }
+    if (bad) {
+        free(lse); free(Dr);
+        return -2;
+    }
+    /* per selected key token and KV head: the sums over the rows that see it */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t task = 0; task < nrows * (int64_t)Hkv; ++task) {
+        int64_t r = task / Hkv, t = rows[r];
+        int g = (int)(task % Hkv);
+        int seq = 0;
+        while (seq < num_seqs && cu_seqlens[seq + 1] <= t) ++seq;
+        int64_t start = cu_seqlens[seq];
+        int64_t L = (int64_t)cu_seqlens[seq + 1] - start, j = t - start;
+        const uint16_t *kj = k + (t * Hkv + g) * (int64_t)d;
+        const uint16_t *vj = v + (t * Hkv + g) * (int64_t)d;
+        double *dkr = dk + (r * Hkv + g) * (int64_t)d;
+        double *dvr = dv + (r * Hkv + g) * (int64_t)d;
+        for (int c = 0; c < d; ++c) dkr[c] = dvr[c] = 0.0;
+        for (int h = g * group; h < (g + 1) * group; ++h) {
+            for (int64_t i = 0; i < L; ++i) {
+                if (!allowed(i, j, causal, window)) continue;
+                const int64_t ti = start + i;
+                const uint16_t *qi = q + (ti * Hq + h) * (int64_t)d;
+                const uint16_t *doi = dout + (ti * Hq + h) * (int64_t)d;
+                double s_ij = 0.0, dp_ij = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    s_ij += widen(qi[c]) * widen(kj[c]);
+                    dp_ij += widen(doi[c]) * widen(vj[c]);
+                }
+                const double p_ij = exp(scale * s_ij - lse[ti * Hq + h]);
+                const double ds_ij = p_ij * (dp_ij - Dr[ti * Hq + h]);
+                for (int c = 0; c < d; ++c) {
+                    dvr[c] += p_ij * widen(doi[c]);
+                    dkr[c] += scale * ds_ij * widen(qi[c]);
+                }
+            }
+        }
+    }
+    free(lse); free(Dr);
+    return 0;
 }
 
 /*

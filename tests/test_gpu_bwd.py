@@ -125,8 +125,9 @@ def test_dk_dv_deterministic(fa):
 
 def test_gqa4k_full_size(fa):
     """The full 4k GQA shape (B=1, Hq=32, Hkv=8, N=4096, d=128, causal, seed 0):
-    sampled dQ rows (every head) against the oracle's row gradient, and for
-    dK, dV the properties the exact gradient has at any size, per KV head:
+    sampled dQ rows (every query head) and sampled dK, dV key rows (every KV
+    head) element by element against the oracle's row gradients, plus the
+    properties the exact gradient has at any size, per KV head:
     sum_j dK_j = 0, and sum_j dV_j = the group's dO summed over all rows."""
     inp = workloads.make("gqa4k", seed=0)
     B, N, Hq, d = inp.q.shape
@@ -140,6 +141,13 @@ def test_gqa4k_full_size(fa):
     rq = oracle.attn_bwd_dq_rows(inp.q[0], inp.k[0], inp.v[0], do[0], cu, rows, True, 0,
                                  inp.scale)
     check("dQ rows", dq[0, rows], rq, "gqa4k")
+    g = torch.Generator("cpu").manual_seed(2)
+    krows = sorted(set([0, 1, 127, 128, 129, 2048, 4094, 4095] +
+                       torch.randint(0, N, (24,), generator=g).tolist()))
+    rk, rv = oracle.attn_bwd_dkv_rows(inp.q[0], inp.k[0], inp.v[0], do[0], cu, krows, True, 0,
+                                      inp.scale)
+    check("dK rows", dk[0, krows], rk, "gqa4k")
+    check("dV rows", dv[0, krows], rv, "gqa4k")
     dk64 = dk.double().cpu()[0]                        # [N, Hkv, d]
     assert (dk64.sum(0).abs() <= 1e-3 * dk64.abs().sum(0) + 1e-3).all()
     dv64 = dv.double().cpu()[0]

@@ -154,6 +154,16 @@ def test_full_size_dense_sampled(fa, name, n_random):
     compare(o_s, o_ref, l_s, lse_ref, name)
 
 
+def test_gqa4k_every_row(fa):
+    """The headline workload (B=1, Hq=32, Hkv=8, N=4096, d=128, causal, seed 0)
+    in the bench's launch configuration: every row and head of O and LSE
+    against the fp64 oracle (the whole score matrix, about 4 s on 16 cores)."""
+    inp = workloads.make("gqa4k", seed=0)
+    o, lse = run_dense(fa, inp)
+    o_ref, lse_ref = oracle.attn(inp.q, inp.k, inp.v, True, 0, inp.scale)
+    compare(o, o_ref, lse, lse_ref, "gqa4k every row")
+
+
 def test_full_size_varlen_sampled(fa):
     inp = workloads.make("varlen16", seed=0)
     q, k, v, cu = inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.cu_seqlens.cuda()

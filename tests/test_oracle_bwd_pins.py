@@ -209,3 +209,43 @@ def test_minus_inf_sinks_backward_is_plain():
     for x, y in zip(a, b[:3]):
         assert np.array_equal(x, y)
     assert np.all(b[3] == 0.0)
+
+
+
+def test_dkv_rows_match_full_backward():
+    """The key-row dK, dV (row statistics first, then per-key sums over the
+    rows that see the key) equal the pinned full backward's rows, which
+    scatters each query row's terms into every key it sees."""
+    lens = [40, 0, 77]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv, d = int(cu[-1]), 4, 2, 32
+    q, k, v = rnd((T, Hq, d), 51), rnd((T, Hkv, d), 52), rnd((T, Hkv, d), 53)
+    do = rnd((T, Hq, d), 54)
+    rows = [0, 5, 39, 40, 41, 100, 116]
+    for causal, window in ((0, 0), (1, 0), (1, 9), (1, 1)):
+        _, dk, dv = oracle.attn_bwd_varlen(q, k, v, do, cu, causal, window, 0.3)
+        gk, gv = oracle.attn_bwd_dkv_rows(q, k, v, do, cu, rows, causal, window, 0.3)
+        for got, ref in ((gk, dk[rows]), (gv, dv[rows])):
+            assert np.allclose(got, ref, rtol=1e-12, atol=1e-13 * np.abs(ref).max())
+    # a window of one key: each key is seen only by its own row, whose softmax
+    # is that key alone, so dS = 0 (dK = 0) and dV_j sums dO_j over the
+    # group's query heads
+    gk, gv = oracle.attn_bwd_dkv_rows(q, k, v, do, cu, rows, 1, 1, 0.3)
+    assert np.abs(gk).max() == 0.0
+    dod = do.double().numpy().reshape(T, Hkv, Hq // Hkv, d).sum(axis=2)
+    assert np.allclose(gv, dod[rows], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,window", [(0, 0), (1, 0), (1, 5)])
+def test_dkv_rows_match_autograd(causal, window):
+    """Independent of the oracle's other backward: fp64 autograd of the
+    forward definition, on a dense GQA batch, at chosen key rows."""
+    B, N, Hq, Hkv, d = 1, 33, 4, 2, 16
+    q, k, v = rnd((B, N, Hq, d), 61), rnd((B, N, Hkv, d), 62), rnd((B, N, Hkv, d), 63)
+    do = rnd((B, N, Hq, d), 64)
+    _, dk_ref, dv_ref = autograd_grads(q, k, v, do, causal, window, 0.25)
+    rows = [0, 1, 16, 31, 32]
+    cu = np.array([0, N], dtype=np.int32)
+    gk, gv = oracle.attn_bwd_dkv_rows(q[0], k[0], v[0], do[0], cu, rows, causal, window, 0.25)
+    assert np.allclose(gk, dk_ref[0, rows], rtol=1e-10, atol=1e-12)
+    assert np.allclose(gv, dv_ref[0, rows], rtol=1e-10, atol=1e-12)
