@@ -57,13 +57,18 @@ def parse():
     ap.add_argument("--no-next", action="store_true",
                     help="skip the extension rows (backward, FP8-cache decode)")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "bwd", "decode_fp8",
-                                       "prefill_paged", "prefill_fp8"],
+                                       "prefill_paged", "prefill_fp8", "prefill_configs"],
                     default="all",
                     help="time one kernel family only (for profiler captures)")
     ap.add_argument("--prefill-workload", default=PREFILL,
                     choices=["gqa4k", "long32k", "long32k_w4096"])
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="number of decode sequences (64 = the decode64 workload)")
+    ap.add_argument("--configs", default="long32k,long32k_w4096,varlen16",
+                    help="prefill workloads timed as extension rows (comma list)")
+    ap.add_argument("--rescale-stats", action="store_true",
+                    help="count the conditional rescales of one gqa4k prefill with the "
+                         "counter build (libfa_sm100_counters.so) and print them")
     return ap.parse_args()
 
 
@@ -112,6 +117,23 @@ def prefill_flops(B, Hq, N, d, causal=True, window=0):
         pairs = window * (window + 1) // 2 + (N - window) * window
         return 4.0 * B * Hq * d * pairs
     return 4.0 * B * Hq * N * N * d / (2.0 if causal else 1.0)
+
+
+def timing_stats(ms, dev=None):
+    """Mean, median, min and 90th percentile of per-call times in ms (each the
+    max over ranks)."""
+    xs = sorted(float(x) for x in ms)
+    n = len(xs)
+    p90 = xs[min(n - 1, max(0, int(math.ceil(0.9 * n)) - 1))]
+    mean, med, mn, p90 = max_over_ranks([statistics.mean(xs), statistics.median(xs), xs[0], p90],
+                                        dev)
+    return {"mean_ms": round(mean, 5), "median_ms": round(med, 5), "min_ms": round(mn, 5),
+            "p90_ms": round(p90, 5), "calls": n}
+
+
+def fp64_sums(**tensors):
+    """fp64 sum of every element of each input (a checksum of the draw)."""
+    return {k: float(torch.sum(t, dtype=torch.float64).item()) for k, t in tensors.items()}
 
 
 def kernel_source_hash():
@@ -231,8 +253,8 @@ def oracle_sample(inp, target_s, cores, name=PREFILL):
     def run(stride, offset):
         rows = list(range(offset, N, stride))
         t0 = time.perf_counter()
-        oracle.attn_rows(inp.q, inp.k, inp.v, [(0, r) for r in rows], True, inp.window,
-                         inp.scale)
+        run.last = oracle.attn_rows(inp.q, inp.k, inp.v, [(0, r) for r in rows], True,
+                                    inp.window, inp.scale)
         dt = time.perf_counter() - t0
         W = inp.window if inp.window else N + 1
         fl = sum(4.0 * Hq * d * min(r + 1, W) for r in rows)
@@ -246,7 +268,23 @@ def oracle_sample(inp, target_s, cores, name=PREFILL):
     which = "every row" if stride == 1 else f"every {stride}th row"
     desc = (f"{nrows} query rows ({which}, all {Hq} heads) of the {name} workload, "
             f"{fl / 1e9:.1f} GFLOP in {dt:.1f} s")
+    oracle_sample.last = (list(range(stride - 1, N, stride)), run.last)
     return fl / dt / 1e12, desc, dt
+
+
+def oracle_parity(o, lse, rows, ref):
+    """The kernel's O [1,N,Hq,d] and LSE [1,Hq,N] against the oracle's rows."""
+    import numpy as np
+    o_ref, lse_ref = ref
+    og = o[0, rows].float().cpu().double().numpy()
+    lg = lse[0][:, rows].T.cpu().double().numpy()
+    eo = np.abs(og - o_ref)
+    el = np.abs(lg - lse_ref)
+    res = {"rows": len(rows), "o_max_abs": float(eo.max()), "o_mean_abs": float(eo.mean()),
+           "lse_max_abs": float(el.max())}
+    res["within_tolerance"] = bool(res["o_max_abs"] <= 2e-2 and res["o_mean_abs"] <= 2e-3 and
+                                   res["lse_max_abs"] <= 1e-3)
+    return res
 
 
 # --------------------------------------------------------------------- ours
@@ -267,7 +305,7 @@ def bench_ours(args):
     # ---- inputs (seeded per rank; resident in HBM before timing)
     do_p = args.only in ("all", "prefill", "bwd", "prefill_fp8")
     do_d = args.only in ("all", "decode", "decode_fp8")
-    if args.only in ("bwd", "decode_fp8", "prefill_paged", "prefill_fp8"):
+    if args.only in ("bwd", "decode_fp8", "prefill_paged", "prefill_fp8", "prefill_configs"):
         return bench_only_next(fa_import(), args, do_p, do_d)
     pname = args.prefill_workload
     seed = rank_seed(args.seed, rank)
@@ -337,9 +375,26 @@ def bench_ours(args):
     d_ms = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
     p_tot, d_tot = sum(p_ms), sum(d_ms)
     p_tot, d_tot = max_over_ranks([p_tot, d_tot], dev)
+    p_stats, d_stats = timing_stats(p_ms, dev), timing_stats(d_ms, dev)
     err = fa.check_device_error()
     if err:
         raise RuntimeError(f"device error in timed region: {fa.status_string(err)}")
+
+    # ---- the prefill again, back to back without the L2 flush (its inputs,
+    # 50 MB, then stay in the 126 MB L2 between calls)
+    nf_stats = None
+    if do_p:
+        for _ in range(3):
+            prefill()
+        nf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in nf:
+            a.record(stream)
+            prefill()
+            b.record(stream)
+        torch.cuda.synchronize()
+        nf_stats = timing_stats([a.elapsed_time(b) for a, b in nf], dev)
+        nf_stats["tflops_median"] = round(flops / (nf_stats["median_ms"] * 1e-3) / 1e12, 2)
 
     # ---- extension rows, timed on their own after the step (same inputs):
     # the backward of the prefill and the decode over an FP8 copy of the cache
@@ -389,7 +444,7 @@ def bench_ours(args):
     e2e_steps(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    n_e2e = max(3, min(args.steps, 10))
+    n_e2e = max(3, args.steps)
     e0.record(s_in)
     e2e_steps(n_e2e)
     e1.record(s_out)                               # after the last download, which waits on all
@@ -429,7 +484,14 @@ def bench_ours(args):
                    "decode": {"num_seqs": S, "Hq": dq.shape[1], "Hkv": Hkv_d, "d": dd,
                               "kv_tokens": int(din.seq_lens.sum()), "kv_bytes": kv_bytes},
                    "l2": "flushed before every timed kernel (256 MiB write)",
-                   "parallelism": f"{world} independent replica(s), one per GPU"},
+                   "parallelism": f"{world} independent replica(s), one per GPU",
+                   "input_fp64_sums": {
+                       "prefill": fp64_sums(q=pin.q, k=pin.k, v=pin.v) if do_p else None,
+                       "decode": fp64_sums(q=din.q, k_cache=din.k_cache, v_cache=din.v_cache,
+                                           seq_lens=din.seq_lens) if do_d else None}},
+        "timing": {"prefill": p_stats, "decode": d_stats,
+                   "prefill_no_flush": nf_stats,
+                   "value_from": "mean over the timed steps"},
         "roofline": {"bound": "tensor", "achieved": round(ach_tf, 2),
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(ach_tf / pk["bf16_tflops"], 4),
@@ -462,6 +524,12 @@ def bench_ours(args):
         val, desc, _ = oracle_sample(pin, args.cpu_seconds, cores, pname)
         line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
+        # the kernel's output on the same rows (a fresh call: the extension
+        # rows reuse the output buffers)
+        fa.fwd(q, k, v, True, pin.window, pin.scale, out=o, lse=lse)
+        torch.cuda.synchronize()
+        rows, ref = oracle_sample.last
+        line["cpu_baseline"]["parity"] = oracle_parity(o, lse, rows, ref)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -533,7 +601,9 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
             fn()
             b.record(stream)
         torch.cuda.synchronize()
-        return max_over_ranks([sum(a.elapsed_time(b) for a, b in evs)], dev)[0] / K
+        ms = [a.elapsed_time(b) for a, b in evs]
+        timed.stats = timing_stats(ms, dev)
+        return max_over_ranks([sum(ms)], dev)[0] / K
 
     if which in ("all", "bwd"):
         bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, flops, out)
@@ -545,6 +615,8 @@ def bench_next(fa, args, dev, stream, flush, pk, traffic_all, pin, q, k, v, o, l
     if which in ("all", "prefill_fp8"):
         bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse,
                                flops, out)
+    if which in ("all", "prefill_configs"):
+        bench_next_prefill_configs(fa, args, dev, timed, pk, traffic_all, out)
     err = fa.check_device_error()
     if err:
         raise RuntimeError(f"device error in the extension rows: {fa.status_string(err)}")
@@ -559,9 +631,11 @@ def bench_next_bwd(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, o, lse, 
     B, N, Hq, d = q.shape
     wsb = torch.empty(fa.bwd_workspace_bytes(B * N, Hq, d), dtype=torch.uint8, device=dev)
     ms = timed(lambda: fa.bwd(q, k, v, o, g, lse, True, pin.window, pin.scale, gq, gk, gv, wsb))
+    st = timed.stats
     bflops = 2.5 * flops
     ach = bflops / (ms * 1e-3) / 1e12
     out["bwd"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+                  "timing": st,
                   "flop_per_call": bflops, "launches_per_call": 3,
                   "workload": "backward of the prefill workload (dQ, dK, dV), causal",
                   "roofline": {"bound": "tensor", "achieved": round(ach, 2),
@@ -580,7 +654,9 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
     ws = torch.empty(max(fa.fp8_workspace_bytes(B, N, Hkv), 4), dtype=torch.uint8, device=dev)
     prep = fa.fp8_prepare(q, k, v, signs, workspace=ws)
     ms_prep = timed(lambda: fa.fp8_prepare(q, k, v, signs, out=prep, workspace=ws))
+    st_prep = timed.stats
     ms = timed(lambda: fa.fwd_fp8(prep, True, pin.window, pin.scale, out=o, lse=lse))
+    st = timed.stats
     ach = flops / (ms * 1e-3) / 1e12
     peak8 = 2.0 * pk["bf16_tflops"]          # FP8 dense = 2 x bf16 (nominal ratio)
     # preparation: bf16 Q, K, V read, E4M3 codes written (V read twice: its
@@ -590,7 +666,7 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
     prep_gbs = prep_bytes / (ms_prep * 1e-3) / 1e9
     out["prefill_fp8"] = {
         "value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
-        "flop_per_call": flops, "launches_per_call": 1,
+        "timing": st, "flop_per_call": flops, "launches_per_call": 1,
         "with_prepare": {"value": round(flops / ((ms + ms_prep) * 1e-3) / 1e12, 2),
                          "unit": "TFLOP/s", "ms_per_call": round(ms + ms_prep, 4),
                          "launches_per_call": 3},
@@ -601,7 +677,8 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
                      "peak_source": "measured bf16 burst x 2 (nominal FP8:bf16 ratio)",
                      "kernel": "prefill_kernel<128> (FP8 mode)",
                      "traffic": traffic_all.get("prefill_fp8_gqa4k")},
-        "prepare": {"ms_per_call": round(ms_prep, 4), "bytes_per_call": prep_bytes,
+        "prepare": {"ms_per_call": round(ms_prep, 4), "timing": st_prep,
+                    "bytes_per_call": prep_bytes,
                     "launches_per_call": 2,
                     "roofline": {"bound": "hbm", "achieved": round(prep_gbs, 1),
                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -609,6 +686,63 @@ def bench_next_prefill_fp8(fa, args, dev, timed, pk, traffic_all, pin, q, k, v, 
                                  "kernel": "fp8_rot_kernel + fp8_quant_vt_kernel",
                                  "traffic": traffic_all.get("fp8_prepare_gqa4k")}}}
     del prep, ws
+
+
+def bench_next_prefill_configs(fa, args, dev, timed, pk, traffic_all, out):
+    """The other prefill workloads, each its own row with its own roofline:
+    long32k (N = 32768, causal), long32k_w4096 (the same inputs with a
+    4,096-key sliding window: FLOPs of the exact visible pairs), varlen16
+    (16 packed sequences, sum over sequences of 4*Hq*d*L^2/2)."""
+    names = [n for n in args.configs.split(",") if n]
+    cache = {}
+    for name in names:
+        cfg = workloads.CONFIGS[name]
+        if cfg["kind"] == "dense":
+            key = ("dense", cfg["N"])
+            if key not in cache:
+                cache.clear()
+                torch.cuda.empty_cache()
+                inp = workloads.make(name, seed=args.seed)
+                qq, kk, vv = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+                cache[key] = (inp, qq, kk, vv, torch.empty_like(qq),
+                              torch.empty((qq.shape[0], qq.shape[2], qq.shape[1]),
+                                          dtype=torch.float32, device=dev))
+            inp, qq, kk, vv, oo, ll = cache[key]
+            W = cfg["window"]
+            B, N, Hq, d = qq.shape
+            flop = prefill_flops(B, Hq, N, d, True, W)
+            ms = timed(lambda: fa.fwd(qq, kk, vv, True, W, inp.scale, out=oo, lse=ll))
+            shape = f"B={B} Hq={Hq} Hkv={kk.shape[2]} N={N} d={d} causal" + \
+                    (f" window={W}" if W else "")
+            sums = fp64_sums(q=inp.q, k=inp.k, v=inp.v)
+        else:
+            cache.clear()
+            torch.cuda.empty_cache()
+            inp = workloads.make(name, seed=args.seed)
+            qq, kk, vv = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+            cu = inp.cu_seqlens.to(dev)
+            oo = torch.empty_like(qq)
+            ll = torch.empty((qq.shape[1], qq.shape[0]), dtype=torch.float32, device=dev)
+            T, Hq, d = qq.shape
+            flop = sum(4.0 * Hq * d * L * L / 2.0 for L in inp.lens)
+            ms = timed(lambda: fa.fwd_varlen(qq, kk, vv, cu, inp.max_seqlen, True, 0, inp.scale,
+                                             out=oo, lse=ll))
+            shape = (f"{len(inp.lens)} packed sequences, lengths {inp.lens} (total {T}), "
+                     f"Hq={Hq} Hkv={kk.shape[2]} d={d} causal")
+            sums = fp64_sums(q=inp.q, k=inp.k, v=inp.v)
+        st = timed.stats
+        ach = flop / (ms * 1e-3) / 1e12
+        out["prefill_" + name] = {
+            "value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+            "timing": st, "flop_per_call": flop, "launches_per_call": 1,
+            "workload": f"{name}: {shape}", "input_fp64_sums": sums,
+            "roofline": {"bound": "tensor", "achieved": round(ach, 2),
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(ach / pk["bf16_tflops"], 4),
+                         "kernel": "prefill_kernel<128>",
+                         "traffic": traffic_all.get("prefill_" + name)}}
+    cache.clear()
+    torch.cuda.empty_cache()
 
 
 def paged_prefill_workload(seed):
@@ -628,6 +762,7 @@ def bench_next_paged(fa, args, dev, timed, pk, traffic_all, out):
     lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=dev)
     ms = timed(lambda: fa.fwd_paged(q, kc, vc, bt, cu, sl, w.max_seqlen_q, True, 0, w.scale,
                                     out=o, lse=lse))
+    st = timed.stats
     Hq, d = q.shape[1], q.shape[2]
     pairs = 0.0
     for Lq, Lk in zip(w.lens_q, w.seq_lens_k.tolist()):
@@ -635,6 +770,7 @@ def bench_next_paged(fa, args, dev, timed, pk, traffic_all, out):
     flop = 4.0 * Hq * d * pairs
     ach = flop / (ms * 1e-3) / 1e12
     out["prefill_paged"] = {"value": round(ach, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4),
+                            "timing": st,
                             "flop_per_call": flop, "launches_per_call": 1,
                             "workload": "chunked prefill over a 16-token paged cache: 8 sequences, "
                                         f"chunks {w.lens_q}, context+chunk {w.seq_lens_k.tolist()}",
@@ -661,10 +797,12 @@ def bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, 
     vc8, vs8 = quant(dv)
     ms = timed(lambda: fa.decode_paged_fp8(dq, kc8, vc8, ks8, vs8, dbt, dsl, din.scale,
                                            out=dout, lse=dlse, workspace=ws))
+    st = timed.stats
     tokens = float(din.seq_lens.sum().item())
     kv8 = tokens * dk.shape[2] * dk.shape[3] * 1 * 2
     ach = kv8 / (ms * 1e-3) / 1e9
     out["decode_fp8"] = {"value": round(ach, 1), "unit": "GB/s", "ms_per_call": round(ms, 4),
+                         "timing": st,
                          "kv_bytes": kv8, "tokens_per_s": round(tokens / (ms * 1e-3), 1),
                          "launches_per_call": 2,
                          "workload": "decode workload with its cache as FP8 E4M3 + scales",
@@ -716,9 +854,49 @@ def bench_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def rescale_stats(args):
+    """Conditional-rescale counts of one causal prefill on the prefill
+    workload, from the counter build of the library (never the product
+    library, which counts nothing)."""
+    import ctypes
+    path = os.path.join(ROOT, "exact_io_aware_75_b200", "libfa_sm100_counters.so")
+    if not os.path.exists(path):
+        raise SystemExit("build it first: python exact_io_aware_75_b200/build.py --counters")
+    lib = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_rescale_counters.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), vp]
+    lib.fa_rescale_counters.restype = i
+    torch.cuda.set_device(0)
+    inp = workloads.make(args.prefill_workload, seed=args.seed)
+    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
+    B, N, Hq, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    cnt = (ctypes.c_ulonglong * 3)()
+    s = torch.cuda.current_stream().cuda_stream
+    lib.fa_rescale_counters(cnt, s)                 # zero
+    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B,
+                    Hq, k.shape[2], N, d, 1, inp.window, inp.scale, 0, s)
+    if rc != 0 or lib.fa_rescale_counters(cnt, s) != 0:
+        raise SystemExit(f"counter build failed: fa_fwd {rc}")
+    dec, grew, done = (int(x) for x in cnt)
+    print(json.dumps({
+        "workload": args.prefill_workload, "threshold_log2": 8,
+        "decisions": dec, "max_grew": grew, "rescaled": done,
+        "skipped_fraction": round(1.0 - done / max(dec, 1), 5),
+        "rescales_vs_unconditional": round(grew / max(done, 1), 2),
+        "what": "per (warp of 32 query rows, key block after a tile's first): decisions; "
+                "max_grew = some row's running max grew (an online softmax without the "
+                "threshold rescales there); rescaled = it grew by more than 2^8"}), flush=True)
+
+
 def main():
     args = parse()
-    if args.impl == "reference":
+    if args.rescale_stats:
+        rescale_stats(args)
+    elif args.impl == "reference":
         bench_reference(args)
     else:
         bench_ours(args)

@@ -10,14 +10,23 @@ sys.path.insert(0, ROOT)
 import bench  # noqa: E402
 
 
-def test_every_recorded_line_matches_the_current_sources():
+def test_recorded_lines_count_only_while_current():
+    """Every committed line names a known kernel family, a 12-digit source
+    hash and a positive byte count; the bench uses exactly the lines whose
+    family still hashes as at the capture (a stale line reads as null)."""
     got = bench.recorded_traffic()
     lines = [ln.split() for ln in open(os.path.join(ROOT, "profiles", "dram_traffic.txt"))
              if ln.strip() and not ln.startswith("#")]
-    assert {p[0] for p in lines} == set(got)
-    for key in ("prefill_gqa4k", "decode_decode64", "bwd_gqa4k", "prefill_fp8_gqa4k",
-                "fp8_prepare_gqa4k"):
-        assert got[key] > 0
+    assert lines
+    current = set()
+    for p in lines:
+        fam = bench.family_of(p[0])
+        assert fam is not None, p[0]
+        assert len(p[1]) == 12 and all(c in "0123456789abcdef" for c in p[1]), p
+        assert float(p[3]) > 0, p
+        if p[1] == bench.family_hash(fam):
+            current.add(p[0])
+    assert set(got) == current
 
 
 def test_families_and_stale_lines(tmp_path):
