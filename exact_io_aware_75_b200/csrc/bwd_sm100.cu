@@ -93,7 +93,7 @@ struct Params {
     float *dq_acc;      // [total, Hq, d] fp32
     void *dk, *dv;      // [total, Hkv, d] bf16
     const int *cu_seqlens;
-    int num_seqs, seqlen, total_tokens;
+    int num_seqs, seqlen, total_tokens, max_seqlen;
     int Hq, Hkv, group;
     int causal, window;
     float scale, scale_log2;
@@ -116,6 +116,12 @@ __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     if (p.cu_seqlens) {
         w.tok0 = __ldg(p.cu_seqlens + w.seq);
         w.L = __ldg(p.cu_seqlens + w.seq + 1) - w.tok0;
+        // A sequence outside [0, total_tokens) or longer than max_seqlen is
+        // skipped by every role alike and reported.
+        if (w.tok0 < 0 || w.L < 0 || w.L > p.max_seqlen || w.tok0 > p.total_tokens - w.L) {
+            report_error(kDevErrInput);
+            return false;
+        }
     } else {
         w.tok0 = w.seq * p.seqlen;
         w.L = p.seqlen;
@@ -706,6 +712,7 @@ int launch_bwd(const BwdArgs &a, cudaStream_t stream) {
     p.num_seqs = a.num_seqs;
     p.seqlen = a.seqlen;
     p.total_tokens = (int)total;
+    p.max_seqlen = a.max_seqlen;
     p.Hq = a.Hq;
     p.Hkv = a.Hkv;
     p.group = a.Hq / a.Hkv;

@@ -90,9 +90,12 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
  *   cu_seqlens [num_seqs + 1] int32, device: 0 = cu[0] <= cu[1] <= ... =
  *              total_tokens (prefix sums of the lengths).  Empty sequences are
  *              allowed and write nothing.
- *   max_seqlen >= every sequence length (sizes the launch).  A longer sequence
- *              is reported through fa_check_device_error (FA_ERR_INVALID_ARG)
- *              and its rows past max_seqlen are left unwritten.
+ *   max_seqlen >= every sequence length (sizes the launch).
+ * Device-side input errors: a sequence longer than max_seqlen, or one that
+ * does not lie inside [0, total_tokens) (offsets not ascending, or past the
+ * end), is skipped -- none of its rows is read or written -- and reported
+ * through fa_check_device_error as FA_ERR_INVALID_ARG.  The other sequences
+ * are computed as usual.
  */
 int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
                   const int *cu_seqlens, int num_seqs, int total_tokens,
@@ -222,6 +225,9 @@ int fa_bwd_varlen_sinks(const void *q, const void *k, const void *v, const void 
  * Backward of packed variable-length prefill (fa_fwd_varlen's layouts: q, o,
  * dout, dq [total, Hq, d]; k, v, dk, dv [total, Hkv, d]; lse [Hq, total];
  * cu_seqlens as there).  Workspace: fa_bwd_workspace_bytes(total_tokens, Hq, d).
+ * A sequence longer than max_seqlen or outside [0, total_tokens) is skipped
+ * (its dK, dV rows unwritten, no dQ contribution) and reported through
+ * fa_check_device_error as FA_ERR_INVALID_ARG, as for fa_fwd_varlen.
  */
 int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o,
                   const void *dout, const float *lse, void *dq, void *dk, void *dv,
@@ -375,10 +381,13 @@ int fa_fwd_fp8(const void *q8, const void *k8, const void *vt8, const float *q_s
  *
  * The split-KV scratch comes from a fixed 32 MiB array in the library's own
  * device memory, which every GPU that loads the library holds until the
- * process exits.  Sizes whose workspace (fa_decode_workspace_bytes) exceeds
- * 32 MiB are refused with FA_ERR_WORKSPACE before any CUDA call.  The first
- * call on each device looks up the array's device address (with that device
- * current); make that first call before any stream capture.  All calls share
+ * process exits.  The arguments are checked as by fa_decode_paged; then
+ * sizes whose workspace (fa_decode_workspace_bytes) exceeds 32 MiB are
+ * refused with FA_ERR_WORKSPACE, before any CUDA call.  The first call on
+ * each device looks up the array's device address (with that device current),
+ * and a call looks it up again when the device's current context has changed
+ * since (for example after cudaDeviceReset); make that first call before any
+ * stream capture.  All calls share
  * the array and it keeps the last call's contents (nothing in it needs to
  * start at zero); calls that may overlap on the GPU race on it, so the caller
  * must order them.  Allocates nothing.  Other arguments, results and errors
@@ -411,6 +420,23 @@ int fa_check_device_error(void *stream);
 int fa_selftest_watchdog(void *stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
+/*
+ * Conditional-rescale statistics of the prefill kernels ("FlashAttention-4"
+ * in samanvya.dev's "Attention Is the Bottleneck": the output is rescaled
+ * only when the running maximum grows enough to threaten the fp32 range).
+ * Counted only in a library built with FA_COUNT_RESCALES=1
+ * (exact_io_aware_75_b200/build.py --counters writes libfa_sm100_counters.so);
+ * the regular build returns FA_ERR_UNSUPPORTED and counts nothing.
+ * Synchronises `stream`, copies three counters to out3 (host) and zeroes them:
+ *   out3[0]  decisions: every key block after a tile's first, per warp of 32
+ *            query rows;
+ *   out3[1]  decisions where some row's running maximum grew (an online
+ *            softmax without the threshold rescales there);
+ *   out3[2]  decisions where it grew by more than the threshold (the kernel
+ *            rescaled).
+ */
+int fa_rescale_counters(unsigned long long *out3, void *stream);
+
 int fa_version(void);
 
 #ifdef __cplusplus

@@ -314,3 +314,18 @@ def test_binding_fails_loudly_without_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import exact_io_aware_75_b200"],
                        cwd=tmp_path, capture_output=True, text=True)
     assert r.returncode != 0 and "missing" in r.stderr
+
+
+def test_noalloc_checks_arguments_before_size(fa):
+    """fa_decode_paged_noalloc: an oversized request (64 sequences x 2048
+    pages) with another bad argument reports that argument, as
+    fa_decode_paged would, not the size; with valid arguments, the size."""
+    lib = fa.library()
+
+    def call(q=P, Hq=32, page=16):
+        return lib.fa_decode_paged_noalloc(q, P, P, P, P, P, 0, 64, 100, Hq, 8, 128, page,
+                                           2048, 0.1, None)
+    assert call(Hq=30) == fa.FA_ERR_INVALID_ARG        # Hq not a multiple of Hkv
+    assert call(page=32) == fa.FA_ERR_UNSUPPORTED       # page size other than 16
+    assert call(q=P + 2) == fa.FA_ERR_ALIGNMENT         # misaligned query pointer
+    assert call() == fa.FA_ERR_WORKSPACE                # valid, but needs > 32 MiB

@@ -55,3 +55,33 @@ def test_noalloc_refuses_oversize(fa):
     rc = fa.library().fa_decode_paged_noalloc(P, P, P, P, P, P, 0, 64, 100, 32, 8, 128, 16,
                                               2048, 0.1, None)
     assert rc == fa.FA_ERR_WORKSPACE
+
+
+def test_noalloc_near_limit_matches_oracle(fa):
+    """64 sequences x 32 query heads, d = 128, 496 pages per block-table row:
+    the split-KV scratch takes 31.5 of the array's 32 MiB, and the two full-
+    length sequences (first and last) write its first and last partials.
+    Every row of O and LSE is compared with the fp64 oracle, on two calls in
+    a row."""
+    import numpy as np
+
+    import oracle
+    from parity import compare
+
+    g = torch.Generator("cpu").manual_seed(23)
+    lens = torch.randint(1, 2049, (64,), generator=g).tolist()
+    lens[0] = lens[63] = 496 * 16
+    inp = workloads.paged(lens=lens, Hq=32, Hkv=8, d=128, seed=23, poison=True)
+    assert inp.block_table.shape[1] == 496
+    need = fa.decode_workspace_bytes(64, 32, 128, 16, 496)
+    assert (31 << 20) < need <= 32 << 20
+    args = (inp.q.cuda(), inp.k_cache.cuda(), inp.v_cache.cuda(),
+            inp.block_table.cuda(), inp.seq_lens.cuda())
+    o_ref, lse_ref = oracle.decode_paged(inp.q, inp.k_cache, inp.v_cache, inp.block_table,
+                                         inp.seq_lens, inp.scale)
+    for _ in range(2):
+        o, lse = fa.decode_paged_noalloc(*args, inp.scale)
+        assert fa.check_device_error() == 0
+        compare(o, o_ref, lse, lse_ref, "noalloc near the limit")
+    assert np.isfinite(o_ref).all()
+
