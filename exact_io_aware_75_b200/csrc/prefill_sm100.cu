@@ -59,20 +59,6 @@ constexpr int kRegsControl = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchRegs,
               "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Exponential-phase token between the two softmax warpgroups (see softmax_wg):
-// 0 = none; 1 = the token is taken before the first exponentials, which start
-// against the running maximum while the block maximum is still being formed;
-// 2 = the block maximum and the rescale decision come first, then the token,
-// then the exponentials.
-#ifndef FA_PINGPONG
-#define FA_PINGPONG 0
-#endif
-constexpr int kPingPong = FA_PINGPONG;
-// P to bf16: 1 = integer rounding (pack_bf16_rna), 0 = the cvt instruction.
-#ifndef FA_P_ALU
-#define FA_P_ALU 0
-#endif
-constexpr bool kPackAlu = FA_P_ALU != 0;
 #ifndef FA_POLY_PERIOD
 #define FA_POLY_PERIOD 0
 #endif
@@ -83,11 +69,6 @@ constexpr int kPolyPeriod = FA_POLY_PERIOD;
 #endif
 // FP8 kernel: one group of four scores in kPolyPeriodF8 takes it (0 = none).
 constexpr int kPolyPeriodF8 = FA_POLY_F8;
-// FP8 kernel, P to E4M3: 1 = integer rounding (pack_e4m3x4_rna), 0 = cvt.
-#ifndef FA_P8_ALU
-#define FA_P8_ALU 0
-#endif
-constexpr bool kPack8Alu = FA_P8_ALU != 0;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPageRows = 16;                 // tokens per cache page (paged mode)
 constexpr int kPagesPerTile = 128 / kPageRows;
@@ -153,14 +134,10 @@ struct Unit {
     int ns[2], A;
 };
 
-#ifndef FA_PAGED_ORDER
-#define FA_PAGED_ORDER 1
-#endif
-
 template <bool PAGED, bool SINK = false>
 __device__ __forceinline__ bool get_unit(int u, const Params &p, Unit &w) {
     int mb;
-    if (PAGED && FA_PAGED_ORDER) {
+    if (PAGED) {
         // Chunked prefill: every row block of a chunk reads (nearly) the
         // sequence's whole cached context, which is far larger than the
         // chunk.  Units of one (sequence, KV head) -- all row blocks, all
@@ -243,37 +220,6 @@ __device__ __forceinline__ int unit_next(const Unit &w, int j) {
     return (j + 1 == w.A) ? w.lo_all : j + 1;
 }
 
-// Whether tile t of the unit takes key block j.
-template <bool SINK>
-__device__ __forceinline__ bool unit_in(const Unit &w, int t, int j) {
-    const int lo = t ? w.lo[1] : w.lo[0], hi = t ? w.hi[1] : w.hi[0];
-    if (SINK && j < (t ? w.ns[1] : w.ns[0])) return true;
-    return j >= lo && j < hi;
-}
-
-// The unit's (block, tile) phases run in the MMA warp's order: for each key
-// block, tile 0's then tile 1's.  Every block in the walk is taken by at
-// least one tile (the tiles' ranges overlap or touch, and sink blocks below
-// A belong to the tile with the larger ns).  For tile t's phase at block j:
-// does the phase just before it belong to the other tile (wait for its
-// token), and does the one just after it (pass the token)?
-template <bool SINK>
-__device__ __forceinline__ void phase_links(const Unit &w, int t, int j, bool &wait_other,
-                                            bool &pass_other) {
-    const int first = SINK ? unit_first(w) : w.lo_all;
-    const bool has_prev = j != first;
-    const int jp = (SINK && j == w.lo_all && w.A > 0) ? w.A - 1 : j - 1;
-    const int jn = SINK ? unit_next(w, j) : j + 1;
-    const bool has_next = jn < w.hi_all;
-    if (t == 0) {
-        wait_other = has_prev && unit_in<SINK>(w, 1, jp);
-        pass_other = unit_in<SINK>(w, 1, j) || (has_next && !unit_in<SINK>(w, 0, jn));
-    } else {
-        wait_other = unit_in<SINK>(w, 0, j) || (has_prev && !unit_in<SINK>(w, 1, jp));
-        pass_other = has_next && unit_in<SINK>(w, 0, jn);
-    }
-}
-
 // Unit `it` of this CTA: rows of G = gridDim.x units are walked in
 // alternating directions (snake order), so with units sorted by decreasing
 // cost every CTA gets a similar total.
@@ -290,10 +236,6 @@ struct Shared {
     uint64_t q_full[2], q_empty[2];
     uint64_t kv_full[8], kv_empty[8];
     uint64_t s_full[2], p_lo[2], p_hi[2], o_full[2], o_empty[2];
-    // tok[t][w]: warp w of softmax warpgroup t has finished the exponentials
-    // of a block whose successor, in the unit's order of (block, tile)
-    // phases, belongs to the other warpgroup.
-    uint64_t tok[2][4];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -630,7 +572,7 @@ __device__ __forceinline__ void exp_half(const float (&v)[kHalf], float sl2, flo
             p1 = ex2(x1);
         }
         a2[c & 1] = f2add(a2[c & 1], f2pack(p0, p1));
-        pk[c] = kPackAlu ? pack_bf16_rna(p0, p1) : pack_bf16(p0, p1);
+        pk[c] = pack_bf16(p0, p1);
     }
     acc = f2add(a2[0], a2[1]);
 }
@@ -661,7 +603,7 @@ __device__ __forceinline__ void exp_half_f8(const float (&v)[kHalf], float sl2, 
         }
         a2[0] = f2add(a2[0], f2pack(p0, p1));
         a2[1] = f2add(a2[1], f2pack(p2, p3));
-        pk[c] = kPack8Alu ? pack_e4m3x4_rna(p0, p1, p2, p3) : pack_e4m3x4(p0, p1, p2, p3);
+        pk[c] = pack_e4m3x4(p0, p1, p2, p3);
     }
     acc = f2add(a2[0], a2[1]);
 }
@@ -677,7 +619,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
     const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = sh.tmem_base + lanes + t * kBlockN;
     const uint32_t tO = sh.tmem_base + lanes + C::kColO + t * D;
-    uint32_t s_cnt = 0, pv_cnt = 0, tok_cnt = 0;
+    uint32_t s_cnt = 0, pv_cnt = 0;
 
     FOR_EACH_UNIT(u) {
         Unit w;
@@ -767,25 +709,9 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                         sA[c] = -INFINITY;
             }
             const float mA = row_max64(sA);
-            // Exponential-phase token.  Warp w of tile 0 and warp w + 4 of
-            // tile 1 share an SM sub-partition and its exp2 unit; their
-            // exponentials alternate in the unit's (block, tile) order instead
-            // of overlapping, so each phase runs at the unit's full rate while
-            // the tensor core works on the other tile ("FlashAttention-3":
-            // ping-pong of two warpgroups).
-            bool tok_wait = false, tok_pass = false, took = false;
-            if constexpr (kPingPong > 0) phase_links<SINK>(w, t, j, tok_wait, tok_pass);
-            auto take_token = [&]() -> bool {
-                took = true;
-                if (!tok_wait) return true;
-                if (!mbar_wait_warp(&sh.tok[t ^ 1][warp & 3], tok_cnt & 1, abort)) return false;
-                ++tok_cnt;
-                return true;
-            };
             // With the reference max unchanged (the common case under the
             // conditional rescale) the first half's P needs no block max:
-            // without the token in between, start its exponentials while the
-            // block max is still unknown.
+            // start its exponentials while the block max is still unknown.
             float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
             uint32_t pkA[F8 ? kHalf / 4 : kHalf / 2];
             uint64_t accA = f2pack(0.f, 0.f);
@@ -796,10 +722,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                 else
                     exp_half(v, sl2, mb, pk, acc);
             };
-            if (kPingPong != 2 && !first) {
-                if (kPingPong == 1 && !take_token()) return;
-                exp_any(sA, pkA, accA);
-            }
+            if (!first) exp_any(sA, pkA, accA);
             tmem_wait_ld();
             #pragma unroll
             for (int c = 0; c < kHalf; ++c) sB[c] = __uint_as_float(rawB[c]);
@@ -811,7 +734,7 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                         sB[c] = -INFINITY;
             }
             const float m_blk = fmaxf(mA, row_max64(sB)) * sl2;
-            bool redo = first || kPingPong == 2;
+            bool redo = first;
             if (first) {
                 m_ref = m_blk;
             } else {
@@ -848,7 +771,6 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                     redo = true;
                 }
             }
-            if (kPingPong > 0 && !took && !take_token()) return;
             if (redo) {
                 mb = (m_ref == -INFINITY) ? 0.f : m_ref;
                 accA = f2pack(0.f, 0.f);
@@ -868,10 +790,6 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
             uint32_t pkB[F8 ? kHalf / 4 : kHalf / 2];
             uint64_t accB = f2pack(0.f, 0.f);
             exp_any(sB, pkB, accB);
-            if (kPingPong > 0 && tok_pass) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sh.tok[t][warp & 3]);
-            }
             if constexpr (F8)
                 tmem_st16(tS + kHalf / 4, pkB);
             else
@@ -974,7 +892,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mbar_init(&sh.p_hi[t], 4);
             mbar_init(&sh.o_full[t], 1);
             mbar_init(&sh.o_empty[t], 4);
-            for (int x = 0; x < 4; ++x) mbar_init(&sh.tok[t][x], 1);
         }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&sh.kv_full[s], PAGED ? 2 : 1);

@@ -495,36 +495,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
-// The same pair conversion on the integer pipe, for finite inputs: adding
-// half a bf16 unit in the last place to the bit pattern and keeping the upper
-// 16 bits rounds the magnitude to nearest, ties away from zero (a carry into
-// the exponent field is the correct rounding up to the next binade; the sign
-// bit is never reached).  The cvt instruction above runs on the same unit as
-// ex2, which the softmax keeps busy; these two adds and one byte permute do not.
-__device__ __forceinline__ uint32_t pack_bf16_rna(float lo, float hi) {
-    const uint32_t a = __float_as_uint(lo) + 0x8000u;
-    const uint32_t b = __float_as_uint(hi) + 0x8000u;
-    return __byte_perm(a, b, 0x7632);
-}
-
-// Four non-negative fp32 values of at most 256 (softmax weights under the
-// conditional rescale) to E4M3 codes, rounded to nearest with ties away from
-// zero, without the conversion instruction.  Multiplying by 2^-120 lines the
-// fp32 exponent field up with E4M3's (bias 127 against 7): an E4M3 normal
-// becomes an fp32 normal whose bits 20-26 are the code's exponent and three
-// mantissa bits, and an E4M3 subnormal (below 2^-6) an fp32 subnormal whose
-// bits 20-22 are its three mantissa bits (scalar multiplies, which keep
-// subnormals).  Adding 2^19 rounds the dropped bits; a shift by 4 puts each
-// code in its word's top byte, and byte permutes gather them, p0 in bits 0-7.
-__device__ __forceinline__ uint32_t pack_e4m3x4_rna(float p0, float p1, float p2, float p3) {
-    constexpr float kAlign = 7.52316384526264005e-37f;   // 2^-120
-    const uint32_t b0 = (__float_as_uint(__fmul_rn(p0, kAlign)) + 0x80000u) << 4;
-    const uint32_t b1 = (__float_as_uint(__fmul_rn(p1, kAlign)) + 0x80000u) << 4;
-    const uint32_t b2 = (__float_as_uint(__fmul_rn(p2, kAlign)) + 0x80000u) << 4;
-    const uint32_t b3 = (__float_as_uint(__fmul_rn(p3, kAlign)) + 0x80000u) << 4;
-    return __byte_perm(__byte_perm(b0, b1, 0x0073), __byte_perm(b2, b3, 0x0073), 0x5410);
-}
-
 // Four fp32 values to E4M3 codes (round to nearest even, saturating at
 // +-448), packed with p0 in bits 0-7 (the lowest K index) up to p3 in 24-31.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {

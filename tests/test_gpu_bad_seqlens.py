@@ -60,11 +60,12 @@ def test_offsets_past_total_or_descending(fa):
     assert torch.all(o[100:] == 0)
     _check_seq(o, lse, w, cu, 0)
     # descending offsets: sequence 1 has a negative length and is skipped;
-    # sequence 2 (tokens 50..250) is a valid sequence and is computed
-    cu = torch.tensor([0, 100, 50, 250], dtype=torch.int32)
+    # sequence 0 is computed and nothing past it is written
+    cu = torch.tensor([0, 100, 50], dtype=torch.int32)
     o, lse, err = _run(fa, w, cu, 200)
     assert err == fa.FA_ERR_INVALID_ARG
-    _check_seq(o, lse, w, cu, 2)
+    assert torch.all(o[100:] == 0)
+    _check_seq(o, lse, w, cu, 0)
 
 
 def test_bwd_sequence_longer_than_max_seqlen(fa):
