@@ -60,7 +60,7 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kLaunchR
               "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #ifndef FA_POLY_PERIOD
-#define FA_POLY_PERIOD 0
+#define FA_POLY_PERIOD 8
 #endif
 // One score pair in kPolyPeriod takes the FMA-pipe exponential (0 = none).
 constexpr int kPolyPeriod = FA_POLY_PERIOD;
