@@ -150,7 +150,7 @@ def kernel_source_hash():
 # wrappers, and for the FP8 preparation the argument struct it takes).
 TRAFFIC_FAMILIES = {
     "prefill": ("prefill_sm100.cu", "sm100.cuh"),
-    "decode": ("decode_sm100.cu", "sm100.cuh"),
+    "decode": ("decode_sm100.cu", "decode_tc_sm100.cu", "sm100.cuh"),
     "bwd": ("bwd_sm100.cu", "sm100.cuh"),
     "fp8_prepare": ("fp8_prep.cu", "sm100.cuh", "fa_internal.h"),
 }
@@ -809,7 +809,7 @@ def bench_next_fp8(fa, args, dev, timed, pk, traffic_all, din, dq, dk, dv, dbt, 
                          "roofline": {"bound": "hbm", "achieved": round(ach, 1),
                                       "peak": pk["hbm_gbs"], "unit": "GB/s",
                                       "frac": round(ach / pk["hbm_gbs"], 4),
-                                      "kernel": "decode_split_kernel<128,4,fp8> + combine",
+                                      "kernel": "decode_tc_kernel<128,4> + combine",
                                       "traffic": traffic_all.get("decode_fp8_decode64")}}
     del kc8, vc8, ks8, vs8
 

@@ -665,7 +665,9 @@ int launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     p.k_scale = a.k_scale;
     p.v_scale = a.v_scale;
     int rc;
-    if (a.fp8)
+    if (decode_tc_supported(a))
+        rc = launch_decode_split_tc(a, p.part_o, p.part_lse, pl.max_chunks, stream);
+    else if (a.fp8)
         rc = launch_split_d<true>(a.d, pl.QPW, tk, tv, p, stream);
     else
         rc = launch_split_d<false>(a.d, pl.QPW, tk, tv, p, stream);

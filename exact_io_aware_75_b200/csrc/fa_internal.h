@@ -69,6 +69,13 @@ struct DecodeArgs {
 size_t decode_workspace_bytes(int num_seqs, int Hq, int d, int page_size, int max_pages);
 int launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
+// Split-KV decode of an FP8 cache on the tensor core (decode_tc_sm100.cu):
+// group sizes 1, 2, 4, 8 and d = 128; writes the same chunk partials as the
+// CUDA-core split kernel.
+bool decode_tc_supported(const DecodeArgs &a);
+int launch_decode_split_tc(const DecodeArgs &a, float *part_o, float *part_lse, int max_chunks,
+                           cudaStream_t stream);
+
 // Sizes the backward launch needs; validated by the public entry points.
 struct BwdArgs {
     const void *q, *k, *v, *o, *dout;

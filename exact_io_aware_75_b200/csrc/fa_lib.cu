@@ -2,6 +2,7 @@
 // kernel shares the device error word without relocatable device code.
 #include "fa_api.cu"
 #include "prefill_sm100.cu"
+#include "decode_tc_sm100.cu"
 #include "decode_sm100.cu"
 #include "decode_noalloc.cu"
 #include "bwd_sm100.cu"

@@ -33,8 +33,11 @@ def run(fa, w, sinks=None):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 2), (6, 3)])
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 8), (16, 2), (6, 3), (16, 4), (12, 4), (32, 1)])
 def test_fp8_shapes(fa, d, Hq, Hkv):
+    """Group sizes 1, 2, 4 and 8 run on the tensor-core kernel with 1, 2, 4 or 8
+    pages per tile (eight, four, two or one KV heads per unit); 3 and 32 on the
+    CUDA-core kernel."""
     w = workloads.paged_fp8(lens=[1, 15, 16, 17, 255, 256, 257, 1000], Hq=Hq, Hkv=Hkv, d=d,
                             seed=Hq + d, poison=True, spare_pages=3)
     o, lse = run(fa, w)
