@@ -65,7 +65,7 @@ constexpr int kRegsWork = 216, kRegsControl = 72;
 static_assert(2 * 128 * kRegsWork + 128 * kRegsControl <= kThreads * 168, "register split");
 constexpr int kScaleSlots = 4;     // scales ring (tiles ahead of the softmax)
 constexpr float kRescaleThreshold = 8.0f;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 constexpr int kSmemLimit = 227 * 1024;
 
 struct TcParams {
@@ -163,7 +163,8 @@ struct TcShared {
 //   stages  nst x [V codes | K codes], kRows x 128 bytes each (128-byte
 //           swizzled rows, pages of the tile consecutive); the V codes are
 //           the A operand of P·V
-//   P       2 x [hi | lo]  P^T as E4M3, K-major B operand (N rows x 128 bytes)
+//   P       2 x [hi | lo]  P^T as E4M3, K-major B operand: 2N rows x 128 bytes,
+//           the hi rows then the lo rows (one MMA chain with N' = 2N)
 //   Q       2 x (2 x N x 128)  Q in f16, K-major B operand (64-column boxes)
 template <int D, int G>
 struct Layout {
@@ -177,8 +178,9 @@ struct Layout {
     static constexpr uint32_t kFixed = 2 * kPBytes + 2 * kQBytes;
     __host__ __device__ static uint32_t pbuf(int nst) { return nst * kStage; }
     __host__ __device__ static uint32_t qbuf(int nst) { return pbuf(nst) + 2 * kPBytes; }
-    // TMEM columns: S (2 x N, per tile), O^T (2 x N, per unit), K in f16 (2 x D/2)
-    static constexpr uint32_t kColS = 0, kColO = 2 * N, kColK = 4 * N;
+    // TMEM columns: S (2 x N, per tile), O^T (2 x 2N, per unit: the hi and the
+    // lo products side by side), K in f16 (2 x D/2)
+    static constexpr uint32_t kColS = 0, kColO = 2 * N, kColK = 6 * N;
     static_assert(kColK + D <= kTmemCols, "TMEM columns");
 };
 
@@ -473,7 +475,7 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
     const uint32_t idS = idesc_f32d(kRows, N, false);
-    const uint32_t idPV = idesc_f32d(kRows, N, true);
+    const uint32_t idPV = idesc_f32d(kRows, 2 * N, true);
     const uint32_t stage0 = smem_u32(smem);
     const uint32_t pb = smem_u32(smem + Ly::pbuf(p.nst));
     const uint32_t qb = smem_u32(smem + Ly::qbuf(p.nst));
@@ -497,11 +499,11 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
         if (w.unit_last(p)) tc_commit(&sh.q_empty[ub]);
         return true;
     };
-    // O^T[unit] (+)= V^T (P_hi^T + P_lo^T), kind::f8f6f4, 32 rows per MMA:
-    // A = the V codes of the stage (MN-major, d on M, 128-byte swizzle, 32
-    // rows = 4096 bytes per step), B = P^T (K-major, 32 bytes per step).  The
-    // unit's first tile starts the accumulator; the stage is released when
-    // the MMAs have read it.
+    // [O_hi^T | O_lo^T][unit] (+)= V^T [P_hi^T | P_lo^T], kind::f8f6f4, 32 rows
+    // per MMA: A = the V codes of the stage (MN-major, d on M, 128-byte
+    // swizzle, 32 rows = 4096 bytes per step), B = the 2N rows of P^T
+    // (K-major, 32 bytes per step).  The unit's first tile starts the
+    // accumulator; the stage is released when the MMAs have read it.
     auto issue_pv = [&](bool first, int ub, uint32_t uuse, uint32_t i, int st, uint32_t ph) -> bool {
         const int b = i & 1;
         if (!wait1(&sh.full[st], ph, abort)) return false;
@@ -511,13 +513,9 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
         const uint32_t v_lo = desc_lo(stage0 + st * Ly::kStage, 16);
         const uint32_t p_lo = desc_lo(pb + b * Ly::kPBytes, 16);
         #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            #pragma unroll
-            for (int ks = 0; ks < kRows / 32; ++ks)
-                mma_ss_lo_f8(tmem + Ly::kColO + ub * N, v_lo + ((ks * 4096) >> 4),
-                             p_lo + ((t * Ly::kPTerm + ks * 32) >> 4), idPV,
-                             (t > 0 || ks > 0 || !first) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kRows / 32; ++ks)
+            mma_ss_lo_f8(tmem + Ly::kColO + ub * 2 * N, v_lo + ((ks * 4096) >> 4),
+                         p_lo + ((ks * 32) >> 4), idPV, (ks > 0 || !first) ? 1u : 0u);
         tc_commit(&sh.pv_done[b]);
         tc_commit(&sh.empty[st]);
         return true;
@@ -525,21 +523,27 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
 
     int pst = 0;
     uint32_t pph = 0;
-    Walk cur;
-    cur.start(p);
-    if (cur.valid) {
-        Walk nxt = cur;
-        nxt.next(p);
-        if (!issue_s(cur, 0)) goto out;
-        for (uint32_t i = 0; cur.valid; ++i) {
-            if (nxt.valid && !issue_s(nxt, i + 1)) goto out;
-            if (!issue_pv(cur.unit_first(), cur.ub(), cur.uuse(), i, pst, pph)) goto out;
+    // w runs one tile ahead: S of tile i+1 is issued before P·V of tile i
+    Walk w;
+    w.start(p);
+    if (w.valid) {
+        if (!issue_s(w, 0)) goto out;
+        bool f0 = w.unit_first();
+        int ub0 = w.ub();
+        uint32_t uu0 = w.uuse();
+        w.next(p);
+        for (uint32_t i = 0;; ++i) {
+            if (w.valid && !issue_s(w, i + 1)) goto out;
+            if (!issue_pv(f0, ub0, uu0, i, pst, pph)) goto out;
             if (++pst == p.nst) {
                 pst = 0;
                 pph ^= 1;
             }
-            cur = nxt;
-            if (nxt.valid) nxt.next(p);
+            if (!w.valid) break;
+            f0 = w.unit_first();
+            ub0 = w.ub();
+            uu0 = w.uuse();
+            w.next(p);
         }
     }
 out:
@@ -548,33 +552,37 @@ out:
 }
 
 // ----------------------------------------------------------- softmax warps
-// In-place rescale of this warp's 32 lanes of O^T: column n times alpha[n].
+// In-place rescale of this warp's 32 lanes of [O_hi^T | O_lo^T]: columns n
+// and N + n times alpha[n].
 template <int N>
 __device__ __forceinline__ void rescale_o(uint32_t to, const float *alpha) {
     #pragma unroll 1
-    for (int c = 0; c < N; c += 16) {
+    for (int c = 0; c < 2 * N; c += 16) {
         uint32_t ov[16];
         tmem_ld16(to + c, ov);
         tmem_wait_ld();
         #pragma unroll
         for (int k = 0; k < 16; ++k)
-            ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha[c + k]);
+            ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha[(c + k) & (N - 1)]);
         tmem_st16(to + c, ov);
     }
     tmem_wait_st();
 }
 
-// A unit's normalised partial O: thread = d lane of O^T, columns n < nrows.
+// A unit's normalised partial O = (O_hi + O_lo) / l: thread = d lane of O^T,
+// columns n < nrows.
 template <int N, int D>
 __device__ __forceinline__ void write_o(uint32_t to, const float *inv_l, float *dst, int nrows, int r) {
-    uint32_t ov[N];
+    uint32_t ov[2 * N];
     #pragma unroll
-    for (int c = 0; c < N; c += 16) tmem_ld16(to + c, ov + c);
+    for (int c = 0; c < 2 * N; c += 16) tmem_ld16(to + c, ov + c);
     tmem_wait_ld();
     if (r < D) {
         #pragma unroll
         for (int n = 0; n < N; ++n)
-            if (n < nrows) dst[(size_t)n * D + r] = __uint_as_float(ov[n]) * inv_l[n];
+            if (n < nrows)
+                dst[(size_t)n * D + r] =
+                    (__uint_as_float(ov[n]) + __uint_as_float(ov[N + n])) * inv_l[n];
     }
 }
 
@@ -738,7 +746,7 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
             // rescale O^T in place: P·V of tile i-1 must have completed
             if (!waitw(&sh.pv_done[b ^ 1], ((i - 1) >> 1) & 1, abort)) return;
             tc_fence_after();
-            rescale_o<N>(tmem + Ly::kColO + ub * N, sh.alpha[b]);
+            rescale_o<N>(tmem + Ly::kColO + ub * 2 * N, sh.alpha[b]);
         }
         tc_fence_before();
         __syncwarp();
@@ -800,7 +808,7 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
             const int nrows = HG * G;
             const size_t row0 = ((size_t)w.seq * p.max_chunks + w.chunk) * p.Hq +
                                 (size_t)w.hg * nrows;
-            write_o<N, D>(tmem + Ly::kColO + ub * N, sh.inv_l[ub], p.part_o + row0 * D, nrows, r);
+            write_o<N, D>(tmem + Ly::kColO + ub * 2 * N, sh.inv_l[ub], p.part_o + row0 * D, nrows, r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.o_free[ub]);
