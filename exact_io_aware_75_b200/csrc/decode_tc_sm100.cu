@@ -262,14 +262,23 @@ __host__ __device__ constexpr uint32_t idesc_f32d(int M, int N, bool a_mn_major)
            ((uint32_t)(M >> 4) << 24);
 }
 
-// Bounded waits (warp-collective form: every lane waits).
-__device__ __forceinline__ bool wait1(uint64_t *bar, uint32_t parity, volatile int *abort) {
+// Bounded waits: the first test inline, the rest out of line (one copy per
+// role R, since the roles run under different register budgets), so that
+// the per-tile loops stay short in the instruction cache.
+template <int R>
+__device__ __noinline__ bool wait_rest(uint64_t *bar, uint32_t parity, volatile int *abort) {
     return mbar_wait(bar, parity, abort);
 }
+template <int R>
+__device__ __forceinline__ bool wait1(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    return mbar_try_wait(smem_u32(bar), parity) || wait_rest<R>(bar, parity, abort);
+}
+template <int R>
 __device__ __forceinline__ bool waitw(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    const bool ok = wait1(bar, parity, abort);
+    const bool ok = wait1<R>(bar, parity, abort);
     return __all_sync(0xffffffffu, ok);
 }
+enum : int { kRoleSoftmax = 0, kRoleConvert = 1, kRoleControl = 2 };
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
@@ -305,7 +314,7 @@ __device__ void producer(const CUtensorMap *tmK, const CUtensorMap *tmV, const T
                 }
             }
         }
-        if (!waitw(&sh.empty[st], ph ^ 1, abort)) goto drain;
+        if (!waitw<kRoleControl>(&sh.empty[st], ph ^ 1, abort)) goto drain;
         {
             const int npg = w.npg(p);
             uint8_t *sV = smem + (size_t)st * Ly::kStage;
@@ -384,7 +393,7 @@ __device__ void scales_warp(const TcParams &p, TcShared &sh) {
                 }
             }
         }
-        if (!waitw(&sh.scl_empty[sl], ph ^ 1, abort)) return;
+        if (!waitw<kRoleControl>(&sh.scl_empty[sl], ph ^ 1, abort)) return;
         if (tl == (w.first - w.pg0) / p.ppt) {
             #pragma unroll
             for (int q = 0; q < 8; ++q) sh.scl[sl][kind * 8 + q] = v[q];
@@ -416,7 +425,7 @@ __device__ void q_warp(const TcParams &p, TcShared &sh, uint8_t *smem) {
     w.start(p);
     for (; w.valid; w.next_unit(p)) {
         const int ub = w.ub();
-        if (!waitw(&sh.q_empty[ub], (w.uuse() & 1) ^ 1, abort)) return;
+        if (!waitw<kRoleControl>(&sh.q_empty[ub], (w.uuse() & 1) ^ 1, abort)) return;
         const uint32_t qb = smem_u32(smem + Ly::qbuf(p.nst) + ub * Ly::kQBytes);
         const int hq0 = w.hg * nrows;
         #pragma unroll 1
@@ -484,9 +493,9 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
     // 64-column boxes of N rows).
     auto issue_s = [&](const Walk &w, uint32_t i) -> bool {
         const int b = i & 1, ub = w.ub();
-        if (w.unit_first() && !wait1(&sh.q_full[ub], w.uuse() & 1, abort)) return false;
-        if (!wait1(&sh.k_ready[b], (i >> 1) & 1, abort)) return false;
-        if (i >= 2 && !wait1(&sh.s_free[b], ((i >> 1) - 1) & 1, abort)) return false;
+        if (w.unit_first() && !wait1<kRoleControl>(&sh.q_full[ub], w.uuse() & 1, abort)) return false;
+        if (!wait1<kRoleControl>(&sh.k_ready[b], (i >> 1) & 1, abort)) return false;
+        if (i >= 2 && !wait1<kRoleControl>(&sh.s_free[b], ((i >> 1) - 1) & 1, abort)) return false;
         tc_fence_after();
         const uint32_t q_lo = desc_lo(qb + ub * Ly::kQBytes, 16);
         #pragma unroll
@@ -506,9 +515,9 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
     // accumulator; the stage is released when the MMAs have read it.
     auto issue_pv = [&](bool first, int ub, uint32_t uuse, uint32_t i, int st, uint32_t ph) -> bool {
         const int b = i & 1;
-        if (!wait1(&sh.full[st], ph, abort)) return false;
-        if (!wait1(&sh.o_ok[b], (i >> 1) & 1, abort)) return false;
-        if (first && !wait1(&sh.o_free[ub], (uuse & 1) ^ 1, abort)) return false;
+        if (!wait1<kRoleControl>(&sh.full[st], ph, abort)) return false;
+        if (!wait1<kRoleControl>(&sh.o_ok[b], (i >> 1) & 1, abort)) return false;
+        if (first && !wait1<kRoleControl>(&sh.o_free[ub], (uuse & 1) ^ 1, abort)) return false;
         tc_fence_after();
         const uint32_t v_lo = desc_lo(stage0 + st * Ly::kStage, 16);
         const uint32_t p_lo = desc_lo(pb + b * Ly::kPBytes, 16);
@@ -555,7 +564,7 @@ out:
 // In-place rescale of this warp's 32 lanes of [O_hi^T | O_lo^T]: columns n
 // and N + n times alpha[n].
 template <int N>
-__device__ __forceinline__ void rescale_o(uint32_t to, const float *alpha) {
+__device__ __noinline__ void rescale_o(uint32_t to, const float *alpha) {
     #pragma unroll 1
     for (int c = 0; c < 2 * N; c += 16) {
         uint32_t ov[16];
@@ -572,7 +581,7 @@ __device__ __forceinline__ void rescale_o(uint32_t to, const float *alpha) {
 // A unit's normalised partial O = (O_hi + O_lo) / l: thread = d lane of O^T,
 // columns n < nrows.
 template <int N, int D>
-__device__ __forceinline__ void write_o(uint32_t to, const float *inv_l, float *dst, int nrows, int r) {
+__device__ __noinline__ void write_o(uint32_t to, const float *inv_l, float *dst, int nrows, int r) {
     uint32_t ov[2 * N];
     #pragma unroll
     for (int c = 0; c < 2 * N; c += 16) tmem_ld16(to + c, ov + c);
@@ -625,21 +634,21 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
         const int b = i & 1, ub = w.ub();
         const bool first = w.unit_first(), last = w.unit_last(p);
         if (first) {
-            if (!waitw(&sh.q_full[ub], w.uuse() & 1, abort)) return;
+            if (!waitw<kRoleSoftmax>(&sh.q_full[ub], w.uuse() & 1, abort)) return;
             #pragma unroll
             for (int j = 0; j < G; ++j) cq[j] = sh.qc[ub][h * G + j];
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.q_empty[ub]);
         }
         // this tile's scales
-        if (!waitw(&sh.scl_full[sl], sph, abort)) return;
+        if (!waitw<kRoleSoftmax>(&sh.scl_full[sl], sph, abort)) return;
         const bool valid = pi < w.npg(p) && (w.first + pi) * kPage + t < w.L;
         const float ks = sh.scl[sl][pi * HG + h], vr = sh.scl[sl][8 + pi * HG + h];
         const float vref = sh.scl[sl][16 + h];
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.scl_empty[sl]);
 
-        if (!waitw(&sh.s_full[b], (i >> 1) & 1, abort)) return;
+        if (!waitw<kRoleSoftmax>(&sh.s_full[b], (i >> 1) & 1, abort)) return;
         tc_fence_after();
         uint32_t v[2 * G];
         tmem_ld_cols<2 * G>(tmem + Ly::kColS + b * N + cb, v);
@@ -673,7 +682,7 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.red_bar[b]);
-            if (!waitw(&sh.red_bar[b], (i >> 1) & 1, abort)) return;
+            if (!waitw<kRoleSoftmax>(&sh.red_bar[b], (i >> 1) & 1, abort)) return;
             #pragma unroll
             for (int j = 0; j < G; ++j) {
                 float x = -INFINITY;
@@ -705,7 +714,7 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
             pv[j] = pr * vr;
         }
         // P^T[b] is free once P·V of tile i-2 has completed
-        if (i >= 2 && !waitw(&sh.pv_done[b], ((i >> 1) - 1) & 1, abort)) return;
+        if (i >= 2 && !waitw<kRoleSoftmax>(&sh.pv_done[b], ((i >> 1) - 1) & 1, abort)) return;
         {
             // P = hi + lo, both E4M3: hi rounds P, lo rounds the remainder
             uint32_t hi[G], lo[G];
@@ -741,10 +750,10 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.p_ready[b]);
         // every warp's P and rescale flags of this tile are published
-        if (!waitw(&sh.p_ready[b], (i >> 1) & 1, abort)) return;
+        if (!waitw<kRoleSoftmax>(&sh.p_ready[b], (i >> 1) & 1, abort)) return;
         if (!first && sh.resc[b] == (int)i) {
             // rescale O^T in place: P·V of tile i-1 must have completed
-            if (!waitw(&sh.pv_done[b ^ 1], ((i - 1) >> 1) & 1, abort)) return;
+            if (!waitw<kRoleSoftmax>(&sh.pv_done[b ^ 1], ((i - 1) >> 1) & 1, abort)) return;
             tc_fence_after();
             rescale_o<N>(tmem + Ly::kColO + ub * 2 * N, sh.alpha[b]);
         }
@@ -773,7 +782,7 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sh.lred_bar[ub]);
-                if (!waitw(&sh.lred_bar[ub], w.uuse() & 1, abort)) return;
+                if (!waitw<kRoleSoftmax>(&sh.lred_bar[ub], w.uuse() & 1, abort)) return;
                 #pragma unroll
                 for (int j = 0; j < G; ++j) {
                     // rows of head h in the other pages: every HG-th half-warp;
@@ -802,8 +811,8 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
                 l[j] = 0.f;
             }
             // the unit's partial O: wait for its last P·V and for every l
-            if (!waitw(&sh.pv_done[b], (i >> 1) & 1, abort)) return;
-            if (!waitw(&sh.l_ready[ub], w.uuse() & 1, abort)) return;
+            if (!waitw<kRoleSoftmax>(&sh.pv_done[b], (i >> 1) & 1, abort)) return;
+            if (!waitw<kRoleSoftmax>(&sh.l_ready[ub], w.uuse() & 1, abort)) return;
             tc_fence_after();
             const int nrows = HG * G;
             const size_t row0 = ((size_t)w.seq * p.max_chunks + w.chunk) * p.Hq +
@@ -836,8 +845,8 @@ __device__ void convert_k_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
     uint32_t ph = 0;
     for (uint32_t i = 0; w.valid; w.next(p), ++i, (++st == p.nst ? (st = 0, ph ^= 1) : 0)) {
         const int b = i & 1;
-        if (!waitw(&sh.full[st], ph, abort)) return;
-        if (i >= 2 && !waitw(&sh.s_full[b], ((i >> 1) - 1) & 1, abort)) return;
+        if (!waitw<kRoleConvert>(&sh.full[st], ph, abort)) return;
+        if (i >= 2 && !waitw<kRoleConvert>(&sh.s_full[b], ((i >> 1) - 1) & 1, abort)) return;
         tc_fence_after();
         const uint32_t sK = stage0 + st * Ly::kStage + Ly::kRegion;
         const uint32_t tk = tmem + Ly::kColK + b * (D / 2);
