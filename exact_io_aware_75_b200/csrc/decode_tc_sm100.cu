@@ -5,9 +5,8 @@
 // ("Prefill and decode are different problems"), so its target is the HBM
 // copy rate.  With an FP8 cache the CUDA-core kernel (decode_sm100.cu) is
 // bound by its own instruction issue: per (token, KV head) it converts 2·d
-// codes and runs 2·d·group fused multiply-adds.  Here the CUDA cores only
-// convert codes (E4M3 -> f16 is exact: every E4M3 value is an f16 normal)
-// and the 5th-generation tensor core does the rest:
+// codes and runs 2·d·group fused multiply-adds.  Here both products run in
+// kind::f8f6f4 on the codes exactly as the TMA copy left them:
 //
 //   * A tile is 128 rows = (pages of the tile) x (KV heads of the unit) x
 //     16 tokens, head-major inside a page: rows 16h..16h+15 of a page are
@@ -16,33 +15,33 @@
 //   * S = K·Q^T for all the unit's query heads at once (N = 16 or 32
 //     columns; M = 128 rows): each row only keeps the columns of its own
 //     KV head's query heads, so the product is block diagonal and the rest
-//     is discarded.  K (f16) sits in TMEM, Q (f16) in shared memory.
-//   * P·V as O^T = V^T · P^T with kind::f8f6f4: V^T is the raw V codes as
-//     the TMA copy left them (an MN-major 8-bit operand, d on M), P^T a
+//     is discarded.  K is the K-major A operand; Q is carried as two E4M3
+//     terms (q1 = E4M3(q 2^e), q2 = E4M3(q 2^e - q1), 2^e a power of two per
+//     row) stacked along N, which together hold every bf16 value exactly
+//     unless its remainder falls below E4M3's normal range (2^-10 of the
+//     row's largest magnitude); the softmax adds the two column groups.
+//   * P·V as O^T = V^T · P^T: V^T is the MN-major A operand (d on M), P^T a
 //     K-major E4M3 operand; P is zero outside the block diagonal, so one
 //     chain of MMAs serves every KV head of the tile.  P is carried as two
-//     E4M3 terms, P ~ hi + lo with lo = E4M3(P - hi), and both are
-//     multiplied by the same codes: relative error about 2^-8 per weight,
-//     the order of the bf16 P of the prefill.
+//     E4M3 terms, P ~ hi + lo with lo = E4M3(P - hi), stacked along N:
+//     relative error about 2^-8 per weight, the order of the bf16 P of the
+//     prefill.
 //   * Softmax: one thread per row with the tile's per-query-head maximum
 //     and the conditional rescale of the prefill (threshold 8 in log2
 //     units): O^T accumulates in TMEM over a unit's tiles and is rescaled
 //     in place only when a query head's maximum grows past the threshold.
 //
-// Numerics.  Q is carried in f16 with a per-row power of two (the row's
-// largest |q| brought to [2^14, 2^15)): the bf16 mantissa fits f16's, so
-// this is exact except for elements below 2^-14 of the scaled range, whose
-// error is at most 2^-25 times the row's scale.  FP8 scales: the k scale of
-// a row's page multiplies its scores; P is multiplied by v_scale / vref
-// (vref = the largest v scale of that KV head over the unit's pages) before
-// it is split, and the unit's O is multiplied by vref / l at the end.
+// FP8 scales: the k scale of a row's page multiplies its scores; P is
+// multiplied by v_scale / vref (vref = the largest v scale of that KV head
+// over the unit's pages) before it is split, and the unit's O is
+// multiplied by vref / l at the end.
 //
-// Roles (384 threads, one CTA per SM, persistent over (sequence, head group,
+// Roles (256 threads, one CTA per SM, persistent over (sequence, head group,
 // chunk) units): warps 0-3 softmax, the in-place O rescale and the unit's
-// output, warps 4-7 K conversion (to TMEM), warp 8 TMA producer, warp 9 MMA
-// issuer (one thread), warp 10 FP8 scales (a ring of its own), warp 11 Q
-// preparation.  The stages, the scales and every TMEM/shared buffer are
-// handed over by mbarriers; every wait is bounded.
+// output, warp 4 TMA producer, warp 5 MMA issuer (one thread), warp 6 FP8
+// scales (a ring of its own), warp 7 Q preparation.  The stages, the scales
+// and every TMEM/shared buffer are handed over by mbarriers; every wait is
+// bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -57,15 +56,11 @@ constexpr int kPage = 16;          // tokens per page
 constexpr int kChunkPages = 16;    // pages per split-KV chunk (the combine's layout)
 constexpr int kRows = 128;         // rows per tile
 constexpr int kMaxStages = 8;
-constexpr int kThreads = 384;
-constexpr int kWarpProducer = 8, kWarpMma = 9, kWarpScales = 10, kWarpQ = 11;
-// Registers: 168 per thread at launch; the softmax and the conversion
-// warpgroups take 216, the control warpgroup keeps 72.
-constexpr int kRegsWork = 216, kRegsControl = 72;
-static_assert(2 * 128 * kRegsWork + 128 * kRegsControl <= kThreads * 168, "register split");
+constexpr int kThreads = 256;
+constexpr int kWarpProducer = 4, kWarpMma = 5, kWarpScales = 6, kWarpQ = 7;
 constexpr int kScaleSlots = 4;     // scales ring (tiles ahead of the softmax)
 constexpr float kRescaleThreshold = 8.0f;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 256;
 constexpr int kSmemLimit = 227 * 1024;
 
 struct TcParams {
@@ -141,7 +136,7 @@ struct Walk {
 
 struct TcShared {
     uint64_t full[kMaxStages], empty[kMaxStages];
-    uint64_t k_ready[2], s_full[2], s_free[2], p_ready[2], o_ok[2], pv_done[2];
+    uint64_t s_full[2], s_free[2], p_ready[2], o_ok[2], pv_done[2];
     uint64_t o_free[2];          // per unit buffer: O^T read out by the unit's epilogue
     uint64_t red_bar[2];
     uint64_t scl_full[kScaleSlots], scl_empty[kScaleSlots];
@@ -165,7 +160,8 @@ struct TcShared {
 //           the A operand of P·V
 //   P       2 x [hi | lo]  P^T as E4M3, K-major B operand: 2N rows x 128 bytes,
 //           the hi rows then the lo rows (one MMA chain with N' = 2N)
-//   Q       2 x (2 x N x 128)  Q in f16, K-major B operand (64-column boxes)
+//   Q       2 x [q1 | q2]  Q as two E4M3 terms, K-major B operand: 2N rows x
+//           128 bytes, the q1 rows then the q2 rows
 template <int D, int G>
 struct Layout {
     static_assert(D == 128, "d = 128");
@@ -174,14 +170,14 @@ struct Layout {
     static constexpr uint32_t kStage = 2 * kRegion;
     static constexpr uint32_t kPTerm = N * 128;                 // one E4M3 term of P^T
     static constexpr uint32_t kPBytes = 2 * kPTerm;
-    static constexpr uint32_t kQBytes = (D / 64) * N * 128;
+    static constexpr uint32_t kQBytes = 2 * N * 128;
     static constexpr uint32_t kFixed = 2 * kPBytes + 2 * kQBytes;
     __host__ __device__ static uint32_t pbuf(int nst) { return nst * kStage; }
     __host__ __device__ static uint32_t qbuf(int nst) { return pbuf(nst) + 2 * kPBytes; }
-    // TMEM columns: S (2 x N, per tile), O^T (2 x 2N, per unit: the hi and the
-    // lo products side by side), K in f16 (2 x D/2)
-    static constexpr uint32_t kColS = 0, kColO = 2 * N, kColK = 6 * N;
-    static_assert(kColK + D <= kTmemCols, "TMEM columns");
+    // TMEM columns: S (2 x 2N, per tile: the q1 and the q2 products side by
+    // side), O^T (2 x 2N, per unit: the hi and the lo products side by side)
+    static constexpr uint32_t kColS = 0, kColO = 4 * N;
+    static_assert(kColO + 4 * N <= kTmemCols, "TMEM columns");
 };
 
 // Byte offset of 16-byte chunk c of code row r in a K or V region.
@@ -278,7 +274,7 @@ __device__ __forceinline__ bool waitw(uint64_t *bar, uint32_t parity, volatile i
     const bool ok = wait1<R>(bar, parity, abort);
     return __all_sync(0xffffffffu, ok);
 }
-enum : int { kRoleSoftmax = 0, kRoleConvert = 1, kRoleControl = 2 };
+enum : int { kRoleSoftmax = 0, kRoleControl = 2 };
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
@@ -408,9 +404,10 @@ __device__ void scales_warp(const TcParams &p, TcShared &sh) {
 }
 
 // ------------------------------------------------------------ Q preparation
-// Per unit: the unit's query heads (rows n < HG*G; the rest zero) as f16
-// with a power-of-two row scale, written K-major with the 128-byte swizzle,
-// and the score multiplier scale*log2(e)*2^e of every row.
+// Per unit: the unit's query heads (rows n < HG*G; the rest zero) as two
+// E4M3 terms with a power-of-two row scale, written K-major with the
+// 128-byte swizzle (q1 rows, then q2 rows), and the score multiplier
+// scale*log2(e)*2^-e of every row.
 template <int D, int G>
 __device__ void q_warp(const TcParams &p, TcShared &sh, uint8_t *smem) {
     using Ly = Layout<D, G>;
@@ -454,18 +451,29 @@ __device__ void q_warp(const TcParams &p, TcShared &sh, uint8_t *smem) {
                 #pragma unroll
                 for (int m = LPR / 2; m >= 1; m >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-                // e: the row's largest magnitude times 2^-e lies in [2^14, 2^15)
+                // 2^e: the power of two that brings the row's largest magnitude
+                // into [128, 256); q = (q1 + q2) 2^-e with q1 = E4M3(q 2^e) and
+                // q2 = E4M3(q 2^e - q1): exact for every bf16 value whose
+                // remainder is not an E4M3 subnormal (below 2^-10 of the row's max)
                 int e = 0;
-                if (amax > 0.f) e = min(max((int)((__float_as_uint(amax) >> 23) & 0xff) - 127 - 14, -100), 100);
-                const float down = __uint_as_float((uint32_t)(127 - e) << 23);
-                uint32_t h[4];
+                if (amax > 0.f) e = min(max(127 + 7 - (int)((__float_as_uint(amax) >> 23) & 0xff), -100), 100);
+                const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+                uint32_t c1[4], c2[4];
                 #pragma unroll
-                for (int i = 0; i < 4; ++i) h[i] = pack_f16(f[2 * i] * down, f[2 * i + 1] * down);
+                for (int i = 0; i < 4; ++i) {
+                    const float x0 = f[2 * i] * up, x1 = f[2 * i + 1] * up;
+                    c1[i] = e4m3x2(x0, x1);
+                    float h0, h1;
+                    e4m3x2_val(c1[i], h0, h1);
+                    c2[i] = e4m3x2(x0 - h0, x1 - h1);
+                }
                 const int d0 = sub * 8;
-                const uint32_t addr = qb + (d0 >> 6) * (N * 128) + n * 128 +
-                                      ((((d0 & 63) >> 3) ^ (n & 7)) << 4);
-                sts128(addr, h[0], h[1], h[2], h[3]);
-                if (sub == 0) sh.qc[ub][n] = p.scale_log2 * __uint_as_float((uint32_t)(127 + e) << 23);
+                const uint32_t row = qb + n * 128 + ((((d0 >> 4) ^ (n & 7))) << 4) + (d0 & 15);
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};"
+                             ::"r"(row), "r"(c1[0] | (c1[1] << 16)), "r"(c1[2] | (c1[3] << 16)) : "memory");
+                asm volatile("st.shared.v2.b32 [%0], {%1, %2};"
+                             ::"r"(row + N * 128), "r"(c2[0] | (c2[1] << 16)), "r"(c2[2] | (c2[3] << 16)) : "memory");
+                if (sub == 0) sh.qc[ub][n] = p.scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23);
             }
         }
         fence_proxy_async_smem();
@@ -483,27 +491,27 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
     constexpr int N = Ly::N;
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
-    const uint32_t idS = idesc_f32d(kRows, N, false);
+    const uint32_t idS = idesc_f32d(kRows, 2 * N, false);
     const uint32_t idPV = idesc_f32d(kRows, 2 * N, true);
     const uint32_t stage0 = smem_u32(smem);
     const uint32_t pb = smem_u32(smem + Ly::pbuf(p.nst));
     const uint32_t qb = smem_u32(smem + Ly::qbuf(p.nst));
 
-    // S = K Q^T: A = K (f16 in TMEM, 8 columns per 16 d), B = Q (K-major,
-    // 64-column boxes of N rows).
-    auto issue_s = [&](const Walk &w, uint32_t i) -> bool {
+    // [S1 | S2] = K [Q1 | Q2]^T, kind::f8f6f4, 32 d per MMA: A = the K codes
+    // of the stage (K-major, 128-byte swizzle, 32 bytes per step), B = the 2N
+    // rows of the two E4M3 terms of Q.
+    auto issue_s = [&](const Walk &w, uint32_t i, int st, uint32_t ph) -> bool {
         const int b = i & 1, ub = w.ub();
         if (w.unit_first() && !wait1<kRoleControl>(&sh.q_full[ub], w.uuse() & 1, abort)) return false;
-        if (!wait1<kRoleControl>(&sh.k_ready[b], (i >> 1) & 1, abort)) return false;
+        if (!wait1<kRoleControl>(&sh.full[st], ph, abort)) return false;
         if (i >= 2 && !wait1<kRoleControl>(&sh.s_free[b], ((i >> 1) - 1) & 1, abort)) return false;
         tc_fence_after();
+        const uint32_t k_lo = desc_lo(stage0 + st * Ly::kStage + Ly::kRegion, 16);
         const uint32_t q_lo = desc_lo(qb + ub * Ly::kQBytes, 16);
         #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = ((ks >> 2) * (N * 128) + (ks & 3) * 32) >> 4;
-            mma_ts_lo(tmem + Ly::kColS + b * N, tmem + Ly::kColK + b * (D / 2) + ks * 8,
-                      q_lo + off, idS, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 32; ++ks)
+            mma_ss_lo_f8(tmem + Ly::kColS + b * 2 * N, k_lo + ((ks * 32) >> 4),
+                         q_lo + ((ks * 32) >> 4), idS, ks > 0 ? 1u : 0u);
         tc_commit(&sh.s_full[b]);
         if (w.unit_last(p)) tc_commit(&sh.q_empty[ub]);
         return true;
@@ -513,9 +521,8 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
     // swizzle, 32 rows = 4096 bytes per step), B = the 2N rows of P^T
     // (K-major, 32 bytes per step).  The unit's first tile starts the
     // accumulator; the stage is released when the MMAs have read it.
-    auto issue_pv = [&](bool first, int ub, uint32_t uuse, uint32_t i, int st, uint32_t ph) -> bool {
+    auto issue_pv = [&](bool first, int ub, uint32_t uuse, uint32_t i, int st) -> bool {
         const int b = i & 1;
-        if (!wait1<kRoleControl>(&sh.full[st], ph, abort)) return false;
         if (!wait1<kRoleControl>(&sh.o_ok[b], (i >> 1) & 1, abort)) return false;
         if (first && !wait1<kRoleControl>(&sh.o_free[ub], (uuse & 1) ^ 1, abort)) return false;
         tc_fence_after();
@@ -530,24 +537,31 @@ __device__ void mma_issuer(const TcParams &p, TcShared &sh, uint8_t *smem) {
         return true;
     };
 
-    int pst = 0;
-    uint32_t pph = 0;
+    int pst = 0, sst = 0;
+    uint32_t sph = 0;
     // w runs one tile ahead: S of tile i+1 is issued before P·V of tile i
     Walk w;
     w.start(p);
     if (w.valid) {
-        if (!issue_s(w, 0)) goto out;
+        if (!issue_s(w, 0, sst, sph)) goto out;
+        if (++sst == p.nst) {
+            sst = 0;
+            sph ^= 1;
+        }
         bool f0 = w.unit_first();
         int ub0 = w.ub();
         uint32_t uu0 = w.uuse();
         w.next(p);
         for (uint32_t i = 0;; ++i) {
-            if (w.valid && !issue_s(w, i + 1)) goto out;
-            if (!issue_pv(f0, ub0, uu0, i, pst, pph)) goto out;
-            if (++pst == p.nst) {
-                pst = 0;
-                pph ^= 1;
+            if (w.valid) {
+                if (!issue_s(w, i + 1, sst, sph)) goto out;
+                if (++sst == p.nst) {
+                    sst = 0;
+                    sph ^= 1;
+                }
             }
+            if (!issue_pv(f0, ub0, uu0, i, pst)) goto out;
+            if (++pst == p.nst) pst = 0;
             if (!w.valid) break;
             f0 = w.unit_first();
             ub0 = w.ub();
@@ -628,9 +642,10 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
     }
     Walk w;
     w.start(p);
-    int sl = 0;
-    uint32_t sph = 0;
-    for (uint32_t i = 0; w.valid; w.next(p), ++i, (++sl == kScaleSlots ? (sl = 0, sph ^= 1) : 0)) {
+    int sl = 0, st = 0;
+    uint32_t sph = 0, ph = 0;
+    for (uint32_t i = 0; w.valid; w.next(p), ++i, (++sl == kScaleSlots ? (sl = 0, sph ^= 1) : 0),
+                                  (++st == p.nst ? (st = 0, ph ^= 1) : 0)) {
         const int b = i & 1, ub = w.ub();
         const bool first = w.unit_first(), last = w.unit_last(p);
         if (first) {
@@ -650,8 +665,9 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
 
         if (!waitw<kRoleSoftmax>(&sh.s_full[b], (i >> 1) & 1, abort)) return;
         tc_fence_after();
-        uint32_t v[2 * G];
-        tmem_ld_cols<2 * G>(tmem + Ly::kColS + b * N + cb, v);
+        uint32_t v[2 * G], v2[2 * G];
+        tmem_ld_cols<2 * G>(tmem + Ly::kColS + b * 2 * N + cb, v);
+        tmem_ld_cols<2 * G>(tmem + Ly::kColS + b * 2 * N + N + cb, v2);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -660,7 +676,8 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
         float s[G], mx[G];
         #pragma unroll
         for (int j = 0; j < G; ++j) {
-            const float sv = __uint_as_float(upper ? v[G + j] : v[j]);
+            const float sv = upper ? __uint_as_float(v[G + j]) + __uint_as_float(v2[G + j])
+                                   : __uint_as_float(v[j]) + __uint_as_float(v2[j]);
             s[j] = valid ? sv * (cq[j] * ks) : -INFINITY;
             mx[j] = s[j];
         }
@@ -746,6 +763,16 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
             for (int j = 0; j < G; ++j) sh.alpha[b][h * G + j] = alpha[j];
             if (resc) sh.resc[b] = (int)i;
         }
+        // V codes of rows past the sequence are zeroed in the stage: P is zero
+        // there, and 0 * NaN would poison O (P·V reads the codes as they are)
+        if (__any_sync(0xffffffffu, !valid)) {
+            if (!waitw<kRoleSoftmax>(&sh.full[st], ph, abort)) return;
+            if (!valid) {
+                const uint32_t vrow = smem_u32(smem) + st * Ly::kStage + r * 128;
+                #pragma unroll
+                for (int c = 0; c < 8; ++c) sts128(vrow + c * 16, 0, 0, 0, 0);
+            }
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.p_ready[b]);
@@ -825,59 +852,6 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
     }
 }
 
-// ---------------------------------------------------------- convert warps
-// K warps: per tile, the K codes of row r -> f16 pairs in TMEM lane r (the A
-// operand of S), once S of tile i-2 has released that buffer.  The MMA
-// issues P·V of a tile only after S of that tile, so the V rows zeroed here
-// are in place before P·V reads them.
-template <int D, int G>
-__device__ void convert_k_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
-    using Ly = Layout<D, G>;
-    volatile int *abort = &sh.abort;
-    const int warp = warp_id(), lane = lane_id();
-    const int r = (warp & 3) * 32 + lane;
-    const int pi = r / (kPage * p.HG), t = r & 15;
-    const uint32_t tmem = sh.tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t stage0 = smem_u32(smem);
-    Walk w;
-    w.start(p);
-    int st = 0;
-    uint32_t ph = 0;
-    for (uint32_t i = 0; w.valid; w.next(p), ++i, (++st == p.nst ? (st = 0, ph ^= 1) : 0)) {
-        const int b = i & 1;
-        if (!waitw<kRoleConvert>(&sh.full[st], ph, abort)) return;
-        if (i >= 2 && !waitw<kRoleConvert>(&sh.s_full[b], ((i >> 1) - 1) & 1, abort)) return;
-        tc_fence_after();
-        const uint32_t sK = stage0 + st * Ly::kStage + Ly::kRegion;
-        const uint32_t tk = tmem + Ly::kColK + b * (D / 2);
-        #pragma unroll 2
-        for (int c = 0; c < D / 16; ++c) {
-            const uint4 a = lds128(sK + code_off<D>(r, c));
-            uint32_t wd[8];
-            e4m3x4_to_f16x4(a.x, wd[0], wd[1]);
-            e4m3x4_to_f16x4(a.y, wd[2], wd[3]);
-            e4m3x4_to_f16x4(a.z, wd[4], wd[5]);
-            e4m3x4_to_f16x4(a.w, wd[6], wd[7]);
-            tmem_st8(tk + c * 8, wd);
-        }
-        // V codes of rows past the sequence are zeroed in the stage: P is zero
-        // there, and 0 * NaN would poison O (P·V reads the codes as they are)
-        if (!(pi < w.npg(p) && (w.first + pi) * kPage + t < w.L)) {
-            const uint32_t vrow = stage0 + st * Ly::kStage + r * 128;
-            #pragma unroll
-            for (int c = 0; c < 8; ++c) sts128(vrow + c * 16, 0, 0, 0, 0);
-            fence_proxy_async_smem();
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-            mbar_arrive(&sh.k_ready[b]);
-            mbar_arrive(&sh.empty[st]);
-        }
-    }
-}
-
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -892,14 +866,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.nst; ++s) {
             mbar_init(&sh.full[s], 1);       // TMA bytes
-            mbar_init(&sh.empty[s], 5);      // the four K warps and the P·V commit
+            mbar_init(&sh.empty[s], 1);      // the P·V commit
         }
         for (int s = 0; s < kScaleSlots; ++s) {
             mbar_init(&sh.scl_full[s], 1);
             mbar_init(&sh.scl_empty[s], 4);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh.k_ready[b], 4);
             mbar_init(&sh.s_full[b], 1);
             mbar_init(&sh.s_free[b], 4);
             mbar_init(&sh.p_ready[b], 4);
@@ -933,14 +906,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     __syncthreads();
     tc_fence_after();
 
-    if (warp < 8) {
-        regs_increase<kRegsWork>();
-        if (warp < 4)
-            softmax_wg<D, G>(p, sh, smem);
-        else
-            convert_k_wg<D, G>(p, sh, smem);
+    if (warp < 4) {
+        softmax_wg<D, G>(p, sh, smem);
     } else {
-        regs_decrease<kRegsControl>();
         if (warp == kWarpProducer)
             producer<D, G>(&tmK, &tmV, p, sh, smem);
         else if (warp == kWarpMma) {
