@@ -150,14 +150,15 @@ def kernel_source_hash():
 # wrappers, and for the FP8 preparation the argument struct it takes).
 TRAFFIC_FAMILIES = {
     "prefill": ("prefill_sm100.cu", "sm100.cuh"),
-    "decode": ("decode_sm100.cu", "decode_tc_sm100.cu", "sm100.cuh"),
+    "decode": ("decode_sm100.cu", "sm100.cuh"),
+    "decode_fp8": ("decode_tc_sm100.cu", "decode_sm100.cu", "sm100.cuh"),
     "bwd": ("bwd_sm100.cu", "sm100.cuh"),
     "fp8_prepare": ("fp8_prep.cu", "sm100.cuh", "fa_internal.h"),
 }
 
 
 def family_of(key):
-    for fam in ("fp8_prepare", "prefill", "decode", "bwd"):
+    for fam in ("fp8_prepare", "prefill", "decode_fp8", "decode", "bwd"):
         if key.startswith(fam):
             return fam
     return None

@@ -36,8 +36,11 @@
 //     happen in L2, 16 KB per operation); bwd_convert_kernel rounds the
 //     accumulator to bf16 at the end.
 //   * Warp 12 loads K_j, V_j once per unit and Q_t, dO_t per tile by TMA into
-//     a 3-slot ring, with the tile's LSE (in log2 units) and D beside them;
-//     warp 13 (one thread) issues every MMA and owns the TMEM allocation.
+//     a 3-slot ring, with the tile's LSE (in log2 units) and D beside them.
+//     Two threads issue the MMAs: warp 13 S^T and dP^T (and owns the TMEM
+//     allocation), warp 14 the three gradient GEMMs, so that a tile's S^T
+//     never waits behind the previous tile's gradients (which wait for that
+//     tile's softmax) and the two issue streams overlap.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -54,7 +57,8 @@ constexpr int kBlockQ = 64;    // queries per tile
 constexpr int kThreads = 512;
 constexpr int kWarpDrain = 8;  // warps 8..11
 constexpr int kWarpTma = 12;
-constexpr int kWarpMma = 13;
+constexpr int kWarpMma = 13;       // S^T, dP^T; TMEM allocation
+constexpr int kWarpMmaGrad = 14;   // dV, dK, dQ^T
 constexpr int kStages = 3;
 // Register split (launched with 512 x 128 = 65,536): the two elementwise
 // warpgroups hold a whole 64-column row of Sᵀ and dPᵀ each.
@@ -165,7 +169,7 @@ struct Shared {
     uint64_t qd_full[kStages], qd_empty[kStages];
     uint64_t s_full[2], p_full[2], dq_full[2], dq_free[2];
     uint64_t acc_full, acc_free;
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -230,68 +234,19 @@ out:
     }
 }
 
-// ------------------------------------------------------------ MMA issuer
-__device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
+// ----------------------------------------------------------- MMA issuers
+// S^T(b) = K Q^T and dP^T(b) = V dO^T: K-major operands, d/16 steps; a step
+// moves 32 bytes inside a 64-column box, 4 steps cross to the next box.  S^T
+// of tile n overwrites the P^T that dV of tile n-2 reads, so it waits for
+// that tile's gradient MMAs to complete; dP^T overwrites the dQ^T of tile
+// n-2, so it waits until that is drained.
+__device__ void mma_issuer_s(const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
     const uint32_t idS = idesc_bf16_f32_ab(kBlockK, kBlockQ, false, false);
-    const uint32_t idAcc = idesc_bf16_f32_ab(kBlockK, kD, false, true);
-    const uint32_t idDQ = idesc_bf16_f32_ab(kD, kBlockQ, true, true);
     const uint32_t aK = smem_u32(smem + kOffK), aV = smem_u32(smem + kOffV);
-    const uint32_t aStage = smem_u32(smem + kOffStage), aDS = smem_u32(smem + kOffDS);
+    const uint32_t aStage = smem_u32(smem + kOffStage);
     uint32_t uc = 0, n = 0;
-
-    // S^T(b) = K Q^T and dP^T(b) = V dO^T: K-major operands, d/16 steps; a
-    // step moves 32 bytes inside a 64-column box, 4 steps cross to the next box.
-    auto issue_s = [&](int b, int s) {
-        const uint32_t q = aStage + s * kStageBytes;
-        #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
-            const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
-            mma_ss(tmem + kColS + b * kBlockQ, smem_desc_sw128(aK + okv, 16, 1024),
-                   smem_desc_sw128(q + oq, 16, 1024), idS, ks > 0);
-        }
-    };
-    auto issue_dp = [&](int b, int s) {
-        const uint32_t dO = aStage + s * kStageBytes + kQTile;
-        #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
-            const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
-            mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aV + okv, 16, 1024),
-                   smem_desc_sw128(dO + oq, 16, 1024), idS, ks > 0);
-        }
-    };
-    // dV += P^T dO, dK += dS^T Q (K = 64 queries), then dQ^T = K^T dS^T (K = 128 keys).
-    // dO and Q are MN-major B operands (d contiguous; 16 query rows per step,
-    // boxes of 64 columns LBO apart); dS^T sits in shared memory as 128 key rows
-    // of 64 queries, 128-byte swizzled: K-major A for dK, MN-major B for dQ^T.
-    auto issue_grads = [&](int m, bool first) -> bool {
-        const int b = m & 1, s = m % kStages;
-        if (!mbar_wait(&sh.p_full[b], (m >> 1) & 1, abort)) return false;
-        if (first && uc > 1)
-            if (!mbar_wait(&sh.acc_free, (uc - 2) & 1, abort)) return false;
-        tc_fence_after();
-        const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
-        const uint32_t ds = aDS + b * kDSBytes;
-        #pragma unroll
-        for (int ks = 0; ks < kBlockQ / 16; ++ks)
-            mma_ts(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
-                   smem_desc_sw128(dO + ks * 2048, kQBox, 1024), idAcc, (ks > 0 || !first) ? 1u : 0u);
-        #pragma unroll
-        for (int ks = 0; ks < kBlockQ / 16; ++ks)
-            mma_ss(tmem + kColDK, smem_desc_sw128(ds + ks * 32, 16, 1024),
-                   smem_desc_sw128(q + ks * 2048, kQBox, 1024), idAcc, (ks > 0 || !first) ? 1u : 0u);
-        tc_commit(&sh.qd_empty[s]);
-        #pragma unroll
-        for (int ks = 0; ks < kBlockK / 16; ++ks)
-            mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aK + ks * 2048, kKVBox, 1024),
-                   smem_desc_sw128(ds + ks * 2048, kDSBytes, 1024), idDQ, ks > 0);
-        tc_commit(&sh.dq_full[b]);
-        return true;
-    };
-
     FOR_EACH_UNIT(u) {
         Unit w;
         if (!get_unit(u, p, w)) continue;
@@ -300,22 +255,84 @@ __device__ void mma_issuer(const Params &p, Shared &sh, uint8_t *smem) {
         for (int k = 0; k < w.ntiles; ++k, ++n) {
             const int b = n & 1, s = n % kStages;
             if (!mbar_wait(&sh.qd_full[s], (n / kStages) & 1, abort)) goto out;
+            if (n >= 2 && !mbar_wait(&sh.dq_full[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
-            issue_s(b, s);
-            // dPᵀ(b) overwrites the dQᵀ of tile n-2: wait until it is drained
+            const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+            #pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
+                const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
+                mma_ss(tmem + kColS + b * kBlockQ, smem_desc_sw128(aK + okv, 16, 1024),
+                       smem_desc_sw128(q + oq, 16, 1024), idS, ks > 0);
+            }
             if (n >= 2 && !mbar_wait(&sh.dq_free[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
-            issue_dp(b, s);
+            #pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
+                const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
+                mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aV + okv, 16, 1024),
+                       smem_desc_sw128(dO + oq, 16, 1024), idS, ks > 0);
+            }
             tc_commit(&sh.s_full[b]);
-            if (k > 0 && !issue_grads(n - 1, k == 1)) goto out;
         }
-        if (!issue_grads(n - 1, w.ntiles == 1)) goto out;
-        tc_commit(&sh.kv_empty);
+        tc_commit(&sh.kv_empty);      // K_j, V_j read by this thread's MMAs
+    }
+out:
+    tc_commit(&sh.drain[0]);
+    mbar_drain_wait(&sh.drain[0], 0);
+}
+
+// dV += P^T dO, dK += dS^T Q (K = 64 queries), then dQ^T = K^T dS^T (K = 128
+// keys), once the tile's softmax has published P^T (TMEM) and dS^T (shared
+// memory).  dO and Q are MN-major B operands (d contiguous; 16 query rows
+// per step, boxes of 64 columns LBO apart); dS^T sits in shared memory as 128
+// key rows of 64 queries, 128-byte swizzled: K-major A for dK, MN-major B
+// for dQ^T.
+__device__ void mma_issuer_grad(const Params &p, Shared &sh, uint8_t *smem) {
+    volatile int *abort = &sh.abort;
+    const uint32_t tmem = sh.tmem_base;
+    const uint32_t idAcc = idesc_bf16_f32_ab(kBlockK, kD, false, true);
+    const uint32_t idDQ = idesc_bf16_f32_ab(kD, kBlockQ, true, true);
+    const uint32_t aK = smem_u32(smem + kOffK);
+    const uint32_t aStage = smem_u32(smem + kOffStage), aDS = smem_u32(smem + kOffDS);
+    uint32_t uc = 0, m = 0;
+    FOR_EACH_UNIT(u) {
+        Unit w;
+        if (!get_unit(u, p, w)) continue;
+        if (!mbar_wait(&sh.kv_full, uc & 1, abort)) goto out;
+        ++uc;
+        for (int k = 0; k < w.ntiles; ++k, ++m) {
+            const bool first = k == 0;
+            const int b = m & 1, s = m % kStages;
+            if (!mbar_wait(&sh.p_full[b], (m >> 1) & 1, abort)) goto out;
+            if (first && uc > 1 && !mbar_wait(&sh.acc_free, (uc - 2) & 1, abort)) goto out;
+            tc_fence_after();
+            const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+            const uint32_t ds = aDS + b * kDSBytes;
+            #pragma unroll
+            for (int ks = 0; ks < kBlockQ / 16; ++ks)
+                mma_ts(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
+                       smem_desc_sw128(dO + ks * 2048, kQBox, 1024), idAcc,
+                       (ks > 0 || !first) ? 1u : 0u);
+            #pragma unroll
+            for (int ks = 0; ks < kBlockQ / 16; ++ks)
+                mma_ss(tmem + kColDK, smem_desc_sw128(ds + ks * 32, 16, 1024),
+                       smem_desc_sw128(q + ks * 2048, kQBox, 1024), idAcc,
+                       (ks > 0 || !first) ? 1u : 0u);
+            tc_commit(&sh.qd_empty[s]);
+            #pragma unroll
+            for (int ks = 0; ks < kBlockK / 16; ++ks)
+                mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aK + ks * 2048, kKVBox, 1024),
+                       smem_desc_sw128(ds + ks * 2048, kDSBytes, 1024), idDQ, ks > 0);
+            tc_commit(&sh.dq_full[b]);
+        }
+        tc_commit(&sh.kv_empty);      // K_j read by dQ^T
         tc_commit(&sh.acc_full);
     }
 out:
-    tc_commit(&sh.drain);
-    mbar_drain_wait(&sh.drain, 0);
+    tc_commit(&sh.drain[1]);
+    mbar_drain_wait(&sh.drain[1], 0);
 }
 
 // ---------------------------------------------------- softmax-gradient warps
@@ -512,7 +529,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     if (threadIdx.x == 0) {
         mbar_init(&sh.kv_full, 1);
-        mbar_init(&sh.kv_empty, 1);
+        mbar_init(&sh.kv_empty, 2);     // one commit from each MMA issuer
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sh.qd_full[s], 2);   // TMA bytes + the LSE/D rows
             mbar_init(&sh.qd_empty[s], 1);
@@ -525,7 +542,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         mbar_init(&sh.acc_full, 1);
         mbar_init(&sh.acc_free, 8);
-        mbar_init(&sh.drain, 1);
+        mbar_init(&sh.drain[0], 1);
+        mbar_init(&sh.drain[1], 1);
         sh.abort = 0;
         fence_barrier_init();
     }
@@ -552,7 +570,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (warp == kWarpTma) {
             producer(&tmQ, &tmK, &tmV, &tmdO, p, sh, smem);
         } else if (warp == kWarpMma) {
-            if (lane_id() == 0) mma_issuer(p, sh, smem);
+            if (lane_id() == 0) mma_issuer_s(p, sh, smem);
+        } else if (warp == kWarpMmaGrad) {
+            if (lane_id() == 0) mma_issuer_grad(p, sh, smem);
         }
     }
     __syncwarp();
