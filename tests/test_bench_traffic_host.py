@@ -31,7 +31,8 @@ def test_recorded_lines_count_only_while_current():
 
 def test_families_and_stale_lines(tmp_path):
     assert bench.family_of("prefill_paged_chunks8") == "prefill"
-    assert bench.family_of("decode_fp8_decode64") == "decode"
+    assert bench.family_of("decode_fp8_decode64") == "decode_fp8"
+    assert bench.family_of("decode_decode64") == "decode"
     assert bench.family_of("fp8_prepare_gqa4k") == "fp8_prepare"
     assert bench.family_of("bwd_gqa4k") == "bwd"
     assert bench.family_of("something_else") is None
