@@ -54,6 +54,7 @@ namespace bwd_impl {
 constexpr int kD = 128;          // tile width in d; a head dim of 64 is zero-padded to it
 constexpr int kBlockK = 128;   // keys per unit
 constexpr int kBlockQ = 64;    // queries per tile
+constexpr int kHalfQ = 32;     // queries per half of the elementwise pass
 constexpr int kThreads = 512;
 constexpr int kWarpDrain = 8;  // warps 8..11
 constexpr int kWarpTma = 12;
@@ -61,7 +62,8 @@ constexpr int kWarpMma = 13;       // S^T, dP^T; TMEM allocation
 constexpr int kWarpMmaGrad = 14;   // dV, dK, dQ^T
 constexpr int kStages = 3;
 // Register split (launched with 512 x 128 = 65,536): the two elementwise
-// warpgroups hold a whole 64-column row of Sᵀ and dPᵀ each.
+// warpgroups hold half a row (32 columns) of Sᵀ and dPᵀ at a time, with room
+// to overlap the exponentials of several column groups.
 constexpr int kRegsSoftmax = 176;
 constexpr int kRegsDrain = 88;
 constexpr int kRegsControl = 72;
@@ -244,7 +246,8 @@ __device__ void mma_issuer_s(const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
     const uint32_t idS = idesc_bf16_f32_ab(kBlockK, kBlockQ, false, false);
-    const uint32_t aK = smem_u32(smem + kOffK), aV = smem_u32(smem + kOffV);
+    const uint32_t kLo = desc_lo(smem_u32(smem + kOffK), 16);
+    const uint32_t vLo = desc_lo(smem_u32(smem + kOffV), 16);
     const uint32_t aStage = smem_u32(smem + kOffStage);
     uint32_t uc = 0, n = 0;
     FOR_EACH_UNIT(u) {
@@ -257,22 +260,21 @@ __device__ void mma_issuer_s(const Params &p, Shared &sh, uint8_t *smem) {
             if (!mbar_wait(&sh.qd_full[s], (n / kStages) & 1, abort)) goto out;
             if (n >= 2 && !mbar_wait(&sh.dq_full[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
-            const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
+            const uint32_t qLo = desc_lo(aStage + s * kStageBytes, 16);
+            const uint32_t dLo = qLo + (kQTile >> 4);
             #pragma unroll
             for (int ks = 0; ks < kD / 16; ++ks) {
-                const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
-                const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
-                mma_ss(tmem + kColS + b * kBlockQ, smem_desc_sw128(aK + okv, 16, 1024),
-                       smem_desc_sw128(q + oq, 16, 1024), idS, ks > 0);
+                const uint32_t okv = ((ks >> 2) * kKVBox + (ks & 3) * 32) >> 4;
+                const uint32_t oq = ((ks >> 2) * kQBox + (ks & 3) * 32) >> 4;
+                mma_ss_lo(tmem + kColS + b * kBlockQ, kLo + okv, qLo + oq, idS, ks > 0);
             }
             if (n >= 2 && !mbar_wait(&sh.dq_free[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
             #pragma unroll
             for (int ks = 0; ks < kD / 16; ++ks) {
-                const uint32_t okv = (ks >> 2) * kKVBox + (ks & 3) * 32;
-                const uint32_t oq = (ks >> 2) * kQBox + (ks & 3) * 32;
-                mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aV + okv, 16, 1024),
-                       smem_desc_sw128(dO + oq, 16, 1024), idS, ks > 0);
+                const uint32_t okv = ((ks >> 2) * kKVBox + (ks & 3) * 32) >> 4;
+                const uint32_t oq = ((ks >> 2) * kQBox + (ks & 3) * 32) >> 4;
+                mma_ss_lo(tmem + kColDP + b * kBlockQ, vLo + okv, dLo + oq, idS, ks > 0);
             }
             tc_commit(&sh.s_full[b]);
         }
@@ -294,7 +296,7 @@ __device__ void mma_issuer_grad(const Params &p, Shared &sh, uint8_t *smem) {
     const uint32_t tmem = sh.tmem_base;
     const uint32_t idAcc = idesc_bf16_f32_ab(kBlockK, kD, false, true);
     const uint32_t idDQ = idesc_bf16_f32_ab(kD, kBlockQ, true, true);
-    const uint32_t aK = smem_u32(smem + kOffK);
+    const uint32_t kLoMN = desc_lo(smem_u32(smem + kOffK), kKVBox);
     const uint32_t aStage = smem_u32(smem + kOffStage), aDS = smem_u32(smem + kOffDS);
     uint32_t uc = 0, m = 0;
     FOR_EACH_UNIT(u) {
@@ -310,21 +312,21 @@ __device__ void mma_issuer_grad(const Params &p, Shared &sh, uint8_t *smem) {
             tc_fence_after();
             const uint32_t q = aStage + s * kStageBytes, dO = q + kQTile;
             const uint32_t ds = aDS + b * kDSBytes;
+            const uint32_t qLoMN = desc_lo(q, kQBox), dLoMN = desc_lo(dO, kQBox);
+            const uint32_t dsLoK = desc_lo(ds, 16), dsLoMN = desc_lo(ds, kDSBytes);
             #pragma unroll
             for (int ks = 0; ks < kBlockQ / 16; ++ks)
-                mma_ts(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
-                       smem_desc_sw128(dO + ks * 2048, kQBox, 1024), idAcc,
-                       (ks > 0 || !first) ? 1u : 0u);
+                mma_ts_lo(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
+                          dLoMN + ((ks * 2048) >> 4), idAcc, (ks > 0 || !first) ? 1u : 0u);
             #pragma unroll
             for (int ks = 0; ks < kBlockQ / 16; ++ks)
-                mma_ss(tmem + kColDK, smem_desc_sw128(ds + ks * 32, 16, 1024),
-                       smem_desc_sw128(q + ks * 2048, kQBox, 1024), idAcc,
-                       (ks > 0 || !first) ? 1u : 0u);
+                mma_ss_lo(tmem + kColDK, dsLoK + ((ks * 32) >> 4), qLoMN + ((ks * 2048) >> 4), idAcc,
+                          (ks > 0 || !first) ? 1u : 0u);
             tc_commit(&sh.qd_empty[s]);
             #pragma unroll
             for (int ks = 0; ks < kBlockK / 16; ++ks)
-                mma_ss(tmem + kColDP + b * kBlockQ, smem_desc_sw128(aK + ks * 2048, kKVBox, 1024),
-                       smem_desc_sw128(ds + ks * 2048, kDSBytes, 1024), idDQ, ks > 0);
+                mma_ss_lo(tmem + kColDP + b * kBlockQ, kLoMN + ((ks * 2048) >> 4),
+                          dsLoMN + ((ks * 2048) >> 4), idDQ, ks > 0);
             tc_commit(&sh.dq_full[b]);
         }
         tc_commit(&sh.kv_empty);      // K_j read by dQ^T
@@ -336,6 +338,45 @@ out:
 }
 
 // ---------------------------------------------------- softmax-gradient warps
+// One half row (32 queries) of the elementwise pass for one key:
+//   P = 2^(s * scale * log2e - LSE * log2e),  dS = P * (dP - D),
+// with -LSE*log2e and -D read as broadcast float4 rows, packed f32x2 math, and
+// P, dS rounded to bf16 pairs.  EDGE: queries outside [lo_c, hi_c) (columns of
+// this half) take P = 0.
+template <bool EDGE>
+__device__ __forceinline__ void grad_half(const uint32_t (&sr)[kHalfQ], const uint32_t (&dr)[kHalfQ],
+                                          const float4 *nl4, const float4 *nd4, uint64_t c2,
+                                          int lo_c, int hi_c, uint32_t (&pk)[kHalfQ / 2],
+                                          uint32_t (&dk)[kHalfQ / 2]) {
+    #pragma unroll
+    for (int cc = 0; cc < kHalfQ; cc += 4) {
+        const float4 nl = nl4[cc >> 2], nd = nd4[cc >> 2];
+        float x0, x1, x2, x3;
+        f2unpack(f2fma(f2pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2,
+                       f2pack(nl.x, nl.y)), x0, x1);
+        f2unpack(f2fma(f2pack(__uint_as_float(sr[cc + 2]), __uint_as_float(sr[cc + 3])), c2,
+                       f2pack(nl.z, nl.w)), x2, x3);
+        float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+        if constexpr (EDGE) {
+            p0 = (cc + 0 >= lo_c && cc + 0 < hi_c) ? p0 : 0.f;
+            p1 = (cc + 1 >= lo_c && cc + 1 < hi_c) ? p1 : 0.f;
+            p2 = (cc + 2 >= lo_c && cc + 2 < hi_c) ? p2 : 0.f;
+            p3 = (cc + 3 >= lo_c && cc + 3 < hi_c) ? p3 : 0.f;
+        }
+        float d0, d1, d2, d3;
+        f2unpack(f2mul(f2pack(p0, p1),
+                       f2add(f2pack(__uint_as_float(dr[cc]), __uint_as_float(dr[cc + 1])),
+                             f2pack(nd.x, nd.y))), d0, d1);
+        f2unpack(f2mul(f2pack(p2, p3),
+                       f2add(f2pack(__uint_as_float(dr[cc + 2]), __uint_as_float(dr[cc + 3])),
+                             f2pack(nd.z, nd.w))), d2, d3);
+        pk[cc >> 1] = pack_bf16(p0, p1);
+        pk[(cc >> 1) + 1] = pack_bf16(p2, p3);
+        dk[cc >> 1] = pack_bf16(d0, d1);
+        dk[(cc >> 1) + 1] = pack_bf16(d2, d3);
+    }
+}
+
 template <int DH>
 __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
@@ -369,57 +410,41 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
             const int qmax = min(q0 + kBlockQ, w.L) - 1;
             const bool edge = (w.j0 + kBlockK > w.L) || (p.causal && w.jl > q0) ||
                               (p.window > 0 && w.j0 <= qmax - p.window);
-            // Sᵀ and dPᵀ rows of this key: all four loads in flight at once
-            uint32_t sr[kBlockQ], dr[kBlockQ];
-            tmem_ld32(tS, sr);
-            tmem_ld32(tS + 32, sr + 32);
-            tmem_ld32(tdP, dr);
-            tmem_ld32(tdP + 32, dr + 32);
-            tmem_wait_ld();
-            const uint64_t c2 = f2pack(sl2, sl2);
-            uint32_t pk[kBlockQ / 2], dk[kBlockQ / 2];
-            #pragma unroll
-            for (int c = 0; c < kBlockQ; c += 4) {
-                const float4 nl = nl4[c >> 2], nd = nd4[c >> 2];   // -LSE2, -D (broadcast)
-                float x0, x1, x2, x3;
-                f2unpack(f2fma(f2pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2,
-                               f2pack(nl.x, nl.y)), x0, x1);
-                f2unpack(f2fma(f2pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), c2,
-                               f2pack(nl.z, nl.w)), x2, x3);
-                float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-                if (edge) {
-                    const int i0 = q0 + c;
-                    bool v[4];
-                    #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        v[e] = key_ok;
-                        if (p.causal)
-                            v[e] = v[e] && kj <= i0 + e && (p.window <= 0 || kj > i0 + e - p.window);
-                    }
-                    p0 = v[0] ? p0 : 0.f;
-                    p1 = v[1] ? p1 : 0.f;
-                    p2 = v[2] ? p2 : 0.f;
-                    p3 = v[3] ? p3 : 0.f;
-                }
-                float d0, d1, d2, d3;
-                f2unpack(f2mul(f2pack(p0, p1),
-                               f2add(f2pack(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
-                                     f2pack(nd.x, nd.y))), d0, d1);
-                f2unpack(f2mul(f2pack(p2, p3),
-                               f2add(f2pack(__uint_as_float(dr[c + 2]), __uint_as_float(dr[c + 3])),
-                                     f2pack(nd.z, nd.w))), d2, d3);
-                pk[c >> 1] = pack_bf16(p0, p1);
-                pk[(c >> 1) + 1] = pack_bf16(p2, p3);
-                dk[c >> 1] = pack_bf16(d0, d1);
-                dk[(c >> 1) + 1] = pack_bf16(d2, d3);
+            // Sᵀ and dPᵀ rows of this key in two halves of 32 queries, each
+            // loaded, turned into Pᵀ (over Sᵀ columns the half has read) and
+            // dSᵀ, and stored before the next.  The mask of an edge tile is
+            // the column range [lo_c, hi_c) of this key's visible queries, a
+            // select per value, so the unrolled loop has no branches.
+            int lo_c = 0, hi_c = kBlockQ;
+            if (!key_ok) {
+                lo_c = kBlockQ;
+                hi_c = 0;
+            } else if (p.causal) {
+                lo_c = kj - q0;                                   // query >= key
+                if (p.window > 0) hi_c = min(kBlockQ, kj + p.window - q0);   // query < key + W
             }
-            tmem_st32(tS, pk);
-            // dSᵀ row r: eight 16-byte chunks of 8 queries, chunk index XOR
-            // (row & 7) (128-byte swizzle)
-            #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 v = make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
-                *reinterpret_cast<uint4 *>(dsb + ((ch ^ (r & 7)) << 4)) = v;
+            const uint64_t c2 = f2pack(sl2, sl2);
+            #pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sr[kHalfQ], dr[kHalfQ];
+                tmem_ld32(tS + hh * kHalfQ, sr);
+                tmem_ld32(tdP + hh * kHalfQ, dr);
+                tmem_wait_ld();
+                uint32_t pk[kHalfQ / 2], dk[kHalfQ / 2];
+                const float4 *nl = nl4 + hh * (kHalfQ / 4), *nd = nd4 + hh * (kHalfQ / 4);
+                if (edge)
+                    grad_half<true>(sr, dr, nl, nd, c2, lo_c - hh * kHalfQ, hi_c - hh * kHalfQ, pk, dk);
+                else
+                    grad_half<false>(sr, dr, nl, nd, c2, 0, 0, pk, dk);
+                tmem_st16(tS + hh * (kHalfQ / 2), pk);
+                // dSᵀ row r: eight 16-byte chunks of 8 queries, chunk index
+                // XOR (row & 7) (128-byte swizzle); this half holds four
+                #pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int ch = hh * 4 + c4;
+                    const uint4 v = make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
+                    *reinterpret_cast<uint4 *>(dsb + ((ch ^ (r & 7)) << 4)) = v;
+                }
             }
             tmem_wait_st();
             fence_proxy_async_smem();
