@@ -66,9 +66,6 @@ def parse():
                     help="number of decode sequences (64 = the decode64 workload)")
     ap.add_argument("--configs", default="long32k,long32k_w4096,varlen16",
                     help="prefill workloads timed as extension rows (comma list)")
-    ap.add_argument("--rescale-stats", action="store_true",
-                    help="count the conditional rescales of one gqa4k prefill with the "
-                         "counter build (libfa_sm100_counters.so) and print them")
     return ap.parse_args()
 
 
@@ -855,49 +852,9 @@ def bench_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def rescale_stats(args):
-    """Conditional-rescale counts of one causal prefill on the prefill
-    workload, from the counter build of the library (never the product
-    library, which counts nothing)."""
-    import ctypes
-    path = os.path.join(ROOT, "exact_io_aware_75_b200", "libfa_sm100_counters.so")
-    if not os.path.exists(path):
-        raise SystemExit("build it first: python exact_io_aware_75_b200/build.py --counters")
-    lib = ctypes.CDLL(path)
-    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-    lib.fa_fwd.argtypes = [vp] * 5 + [i] * 7 + [f, i, vp]
-    lib.fa_fwd.restype = i
-    lib.fa_rescale_counters.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), vp]
-    lib.fa_rescale_counters.restype = i
-    torch.cuda.set_device(0)
-    inp = workloads.make(args.prefill_workload, seed=args.seed)
-    q, k, v = inp.q.cuda(), inp.k.cuda(), inp.v.cuda()
-    B, N, Hq, d = q.shape
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
-    cnt = (ctypes.c_ulonglong * 3)()
-    s = torch.cuda.current_stream().cuda_stream
-    lib.fa_rescale_counters(cnt, s)                 # zero
-    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B,
-                    Hq, k.shape[2], N, d, 1, inp.window, inp.scale, 0, s)
-    if rc != 0 or lib.fa_rescale_counters(cnt, s) != 0:
-        raise SystemExit(f"counter build failed: fa_fwd {rc}")
-    dec, grew, done = (int(x) for x in cnt)
-    print(json.dumps({
-        "workload": args.prefill_workload, "threshold_log2": 8,
-        "decisions": dec, "max_grew": grew, "rescaled": done,
-        "skipped_fraction": round(1.0 - done / max(dec, 1), 5),
-        "rescales_vs_unconditional": round(grew / max(done, 1), 2),
-        "what": "per (warp of 32 query rows, key block after a tile's first): decisions; "
-                "max_grew = some row's running max grew (an online softmax without the "
-                "threshold rescales there); rescaled = it grew by more than 2^8"}), flush=True)
-
-
 def main():
     args = parse()
-    if args.rescale_stats:
-        rescale_stats(args)
-    elif args.impl == "reference":
+    if args.impl == "reference":
         bench_reference(args)
     else:
         bench_ours(args)

@@ -45,7 +45,7 @@ EXPORTS = ("fa_fwd", "fa_fwd_varlen", "fa_fwd_sinks", "fa_fwd_varlen_sinks", "fa
            "fa_decode_workspace_bytes", "fa_decode_paged", "fa_decode_paged_sinks",
            "fa_decode_paged_fp8", "fa_fp8_workspace_bytes", "fa_fp8_prepare", "fa_fwd_fp8",
            "fa_decode_paged_noalloc", "fa_status_string", "fa_check_device_error",
-           "fa_selftest_watchdog", "fa_rescale_counters", "fa_version")
+           "fa_selftest_watchdog", "fa_version")
 
 
 class FAError(RuntimeError):
@@ -109,8 +109,6 @@ def _load():
     lib.fa_check_device_error.restype = i
     lib.fa_selftest_watchdog.argtypes = [vp]
     lib.fa_selftest_watchdog.restype = i
-    lib.fa_rescale_counters.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), vp]
-    lib.fa_rescale_counters.restype = i
     lib.fa_version.argtypes = []
     lib.fa_version.restype = i
     return lib

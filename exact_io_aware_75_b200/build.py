@@ -1,10 +1,6 @@
 """Build the sm_100a library in place: exact_io_aware_75_b200/libfa_sm100.so.
 
-    python exact_io_aware_75_b200/build.py [--force] [--verbose-ptxas] [--counters]
-
---counters builds the same library with the prefill's conditional-rescale
-counters compiled in (FA_COUNT_RESCALES=1) as libfa_sm100_counters.so, for
-measurement only; the package always loads libfa_sm100.so.
+    python exact_io_aware_75_b200/build.py [--force] [--verbose-ptxas]
 
 Run by path: importing the package itself needs the built library.
 """
@@ -19,7 +15,6 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa_sm100.so")
-LIB_COUNTERS = os.path.join(PKG, "libfa_sm100_counters.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 
@@ -49,12 +44,5 @@ def build(force=False, ptxas_verbose=False, extra=(), out=LIB):
     return out
 
 
-def build_counters(force=False):
-    return build(force, extra=("-DFA_COUNT_RESCALES=1",), out=LIB_COUNTERS)
-
-
 if __name__ == "__main__":
-    if "--counters" in sys.argv:
-        print(build_counters(force="--force" in sys.argv))
-    else:
-        print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv))

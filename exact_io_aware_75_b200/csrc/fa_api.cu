@@ -634,23 +634,6 @@ int fa_selftest_watchdog(void *stream) {
     return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-int fa_rescale_counters(unsigned long long *out3, void *stream) {
-#if FA_COUNT_RESCALES
-    if (!out3) return FA_ERR_INVALID_ARG;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return FA_ERR_CUDA;
-    const unsigned long long zero[3] = {0, 0, 0};
-    if (cudaMemcpyFromSymbol(out3, fa::g_rescale_stats, sizeof zero) != cudaSuccess ||
-        cudaMemcpyToSymbol(fa::g_rescale_stats, zero, sizeof zero) != cudaSuccess)
-        return FA_ERR_CUDA;
-    return FA_OK;
-#else
-    (void)out3;
-    (void)stream;
-    return FA_ERR_UNSUPPORTED;
-#endif
-}
-
 int fa_version(void) { return 100; }
 
 }  // extern "C"

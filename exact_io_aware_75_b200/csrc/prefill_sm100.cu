@@ -739,15 +739,6 @@ __device__ void softmax_wg(const Params &p, Shared &sh, int *kdoc) {
                 m_ref = m_blk;
             } else {
                 const bool need = m_blk > m_ref + kRescaleThreshold;
-                if constexpr (FA_COUNT_RESCALES != 0) {
-                    const bool grew = __any_sync(0xffffffffu, m_blk > m_ref);
-                    const bool over = __any_sync(0xffffffffu, need);
-                    if (lane == 0) {
-                        atomicAdd(&g_rescale_stats[0], 1ull);
-                        if (grew) atomicAdd(&g_rescale_stats[1], 1ull);
-                        if (over) atomicAdd(&g_rescale_stats[2], 1ull);
-                    }
-                }
                 if (__any_sync(0xffffffffu, need)) {
                     const float m_new = fmaxf(m_ref, m_blk);
                     const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);

@@ -20,16 +20,6 @@ __device__ int g_device_error = 0;
 
 enum : int { kDevErrTimeout = 1, kDevErrInput = 2 };
 
-// Conditional-rescale statistics of the prefill softmax, counted only in a
-// build with FA_COUNT_RESCALES=1 (read by fa_rescale_counters): [0] warp-level
-// decisions (every key block after a tile's first, per warp of 32 rows),
-// [1] those where some row's maximum grew (an unconditional online softmax
-// rescales there), [2] those where it grew past the threshold (rescaled).
-#ifndef FA_COUNT_RESCALES
-#define FA_COUNT_RESCALES 0
-#endif
-__device__ unsigned long long g_rescale_stats[3] = {0, 0, 0};
-
 __device__ __forceinline__ void report_error(int code) {
     atomicCAS(&g_device_error, 0, code);
 }

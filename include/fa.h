@@ -420,23 +420,6 @@ int fa_check_device_error(void *stream);
 int fa_selftest_watchdog(void *stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
-/*
- * Conditional-rescale statistics of the prefill kernels ("FlashAttention-4"
- * in samanvya.dev's "Attention Is the Bottleneck": the output is rescaled
- * only when the running maximum grows enough to threaten the fp32 range).
- * Counted only in a library built with FA_COUNT_RESCALES=1
- * (exact_io_aware_75_b200/build.py --counters writes libfa_sm100_counters.so);
- * the regular build returns FA_ERR_UNSUPPORTED and counts nothing.
- * Synchronises `stream`, copies three counters to out3 (host) and zeroes them:
- *   out3[0]  decisions: every key block after a tile's first, per warp of 32
- *            query rows;
- *   out3[1]  decisions where some row's running maximum grew (an online
- *            softmax without the threshold rescales there);
- *   out3[2]  decisions where it grew by more than the threshold (the kernel
- *            rescaled).
- */
-int fa_rescale_counters(unsigned long long *out3, void *stream);
-
 int fa_version(void);
 
 #ifdef __cplusplus
