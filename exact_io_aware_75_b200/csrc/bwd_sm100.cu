@@ -170,6 +170,8 @@ struct Shared {
     uint64_t kv_full, kv_empty;
     uint64_t qd_full[kStages], qd_empty[kStages];
     uint64_t s_full[2], p_full[2], dq_full[2], dq_free[2];
+    uint64_t pt_free[2];     // dV of the buffer's tile done: Sᵀ's columns are free
+    uint64_t ds_free[2];     // dK of the buffer's tile done: its dSᵀ buffer is free
     uint64_t acc_full, acc_free;
     uint64_t drain[2];
     uint32_t tmem_base;
@@ -240,8 +242,8 @@ out:
 // S^T(b) = K Q^T and dP^T(b) = V dO^T: K-major operands, d/16 steps; a step
 // moves 32 bytes inside a 64-column box, 4 steps cross to the next box.  S^T
 // of tile n overwrites the P^T that dV of tile n-2 reads, so it waits for
-// that tile's gradient MMAs to complete; dP^T overwrites the dQ^T of tile
-// n-2, so it waits until that is drained.
+// that MMA to complete; dP^T overwrites the dQ^T of tile n-2, so it waits
+// until that is drained.
 __device__ void mma_issuer_s(const Params &p, Shared &sh, uint8_t *smem) {
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem_base;
@@ -258,7 +260,7 @@ __device__ void mma_issuer_s(const Params &p, Shared &sh, uint8_t *smem) {
         for (int k = 0; k < w.ntiles; ++k, ++n) {
             const int b = n & 1, s = n % kStages;
             if (!mbar_wait(&sh.qd_full[s], (n / kStages) & 1, abort)) goto out;
-            if (n >= 2 && !mbar_wait(&sh.dq_full[b], ((n - 2) >> 1) & 1, abort)) goto out;
+            if (n >= 2 && !mbar_wait(&sh.pt_free[b], ((n - 2) >> 1) & 1, abort)) goto out;
             tc_fence_after();
             const uint32_t qLo = desc_lo(aStage + s * kStageBytes, 16);
             const uint32_t dLo = qLo + (kQTile >> 4);
@@ -285,9 +287,12 @@ out:
     mbar_drain_wait(&sh.drain[0], 0);
 }
 
-// dV += P^T dO, dK += dS^T Q (K = 64 queries), then dQ^T = K^T dS^T (K = 128
-// keys), once the tile's softmax has published P^T (TMEM) and dS^T (shared
-// memory).  dO and Q are MN-major B operands (d contiguous; 16 query rows
+// dQ^T = K^T dS^T (K = 128 keys), then dV += P^T dO and dK += dS^T Q (K = 64
+// queries), once the tile's softmax has published P^T (TMEM) and dS^T (shared
+// memory).  dQ^T goes first so its drain, which the next dP^T on these
+// columns waits for, starts early; each step is committed on its own
+// barrier: dQ^T (drain may read), dV (S^T's columns free), dK (dS^T and the
+// Q/dO slot free).  dO and Q are MN-major B operands (d contiguous; 16 query rows
 // per step, boxes of 64 columns LBO apart); dS^T sits in shared memory as 128
 // key rows of 64 queries, 128-byte swizzled: K-major A for dK, MN-major B
 // for dQ^T.
@@ -315,19 +320,21 @@ __device__ void mma_issuer_grad(const Params &p, Shared &sh, uint8_t *smem) {
             const uint32_t qLoMN = desc_lo(q, kQBox), dLoMN = desc_lo(dO, kQBox);
             const uint32_t dsLoK = desc_lo(ds, 16), dsLoMN = desc_lo(ds, kDSBytes);
             #pragma unroll
+            for (int ks = 0; ks < kBlockK / 16; ++ks)
+                mma_ss_lo(tmem + kColDP + b * kBlockQ, kLoMN + ((ks * 2048) >> 4),
+                          dsLoMN + ((ks * 2048) >> 4), idDQ, ks > 0);
+            tc_commit(&sh.dq_full[b]);
+            #pragma unroll
             for (int ks = 0; ks < kBlockQ / 16; ++ks)
                 mma_ts_lo(tmem + kColDV, tmem + kColS + b * kBlockQ + ks * 8,
                           dLoMN + ((ks * 2048) >> 4), idAcc, (ks > 0 || !first) ? 1u : 0u);
+            tc_commit(&sh.pt_free[b]);
             #pragma unroll
             for (int ks = 0; ks < kBlockQ / 16; ++ks)
                 mma_ss_lo(tmem + kColDK, dsLoK + ((ks * 32) >> 4), qLoMN + ((ks * 2048) >> 4), idAcc,
                           (ks > 0 || !first) ? 1u : 0u);
             tc_commit(&sh.qd_empty[s]);
-            #pragma unroll
-            for (int ks = 0; ks < kBlockK / 16; ++ks)
-                mma_ss_lo(tmem + kColDP + b * kBlockQ, kLoMN + ((ks * 2048) >> 4),
-                          dsLoMN + ((ks * 2048) >> 4), idDQ, ks > 0);
-            tc_commit(&sh.dq_full[b]);
+            tc_commit(&sh.ds_free[b]);
         }
         tc_commit(&sh.kv_empty);      // K_j read by dQ^T
         tc_commit(&sh.acc_full);
@@ -437,6 +444,9 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
                 else
                     grad_half<false>(sr, dr, nl, nd, c2, 0, 0, pk, dk);
                 tmem_st16(tS + hh * (kHalfQ / 2), pk);
+                // dK and dQ^T of tile n-2 read this dSᵀ buffer
+                if (hh == 0 && n >= 2 &&
+                    !mbar_wait_warp(&sh.ds_free[wg], ((n - 2) >> 1) & 1, abort)) return;
                 // dSᵀ row r: eight 16-byte chunks of 8 queries, chunk index
                 // XOR (row & 7) (128-byte swizzle); this half holds four
                 #pragma unroll
@@ -564,6 +574,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mbar_init(&sh.p_full[b], 4);
             mbar_init(&sh.dq_full[b], 1);
             mbar_init(&sh.dq_free[b], 4);
+            mbar_init(&sh.pt_free[b], 1);
+            mbar_init(&sh.ds_free[b], 1);
         }
         mbar_init(&sh.acc_full, 1);
         mbar_init(&sh.acc_free, 8);
