@@ -54,7 +54,7 @@ namespace bwd_impl {
 constexpr int kD = 128;          // tile width in d; a head dim of 64 is zero-padded to it
 constexpr int kBlockK = 128;   // keys per unit
 constexpr int kBlockQ = 64;    // queries per tile
-constexpr int kHalfQ = 32;     // queries per half of the elementwise pass
+constexpr int kPartQ = 16;     // queries per step of the elementwise pass
 constexpr int kThreads = 512;
 constexpr int kWarpDrain = 8;  // warps 8..11
 constexpr int kWarpTma = 12;
@@ -62,8 +62,8 @@ constexpr int kWarpMma = 13;       // S^T, dP^T; TMEM allocation
 constexpr int kWarpMmaGrad = 14;   // dV, dK, dQ^T
 constexpr int kStages = 3;
 // Register split (launched with 512 x 128 = 65,536): the two elementwise
-// warpgroups hold half a row (32 columns) of Sᵀ and dPᵀ at a time, with room
-// to overlap the exponentials of several column groups.
+// warpgroups hold two 16-column steps of Sᵀ and dPᵀ at a time (one being
+// computed, the next in flight from TMEM).
 constexpr int kRegsSoftmax = 176;
 constexpr int kRegsDrain = 88;
 constexpr int kRegsControl = 72;
@@ -345,43 +345,75 @@ out:
 }
 
 // ---------------------------------------------------- softmax-gradient warps
-// One half row (32 queries) of the elementwise pass for one key:
+// The elementwise pass for one key row, in steps of 16 queries:
 //   P = 2^(s * scale * log2e - LSE * log2e),  dS = P * (dP - D),
 // with -LSE*log2e and -D read as broadcast float4 rows, packed f32x2 math, and
-// P, dS rounded to bf16 pairs.  EDGE: queries outside [lo_c, hi_c) (columns of
-// this half) take P = 0.
+// P, dS rounded to bf16 pairs.  Each step's Sᵀ and dPᵀ columns are loaded
+// while the previous step computes (two register sets of 16 + 16 values);
+// Pᵀ of a step goes over the Sᵀ columns of its own queries (already read),
+// dSᵀ into the step's two 16-byte chunks of the key's row (chunk index XOR
+// (row & 7), the 128-byte swizzle).  EDGE: queries outside [lo_c, hi_c)
+// take P = 0, as a select, so the unrolled code has no branches.
 template <bool EDGE>
-__device__ __forceinline__ void grad_half(const uint32_t (&sr)[kHalfQ], const uint32_t (&dr)[kHalfQ],
-                                          const float4 *nl4, const float4 *nd4, uint64_t c2,
-                                          int lo_c, int hi_c, uint32_t (&pk)[kHalfQ / 2],
-                                          uint32_t (&dk)[kHalfQ / 2]) {
+__device__ __forceinline__ bool grad_row(uint32_t tS, uint32_t tdP, const float4 *nl4,
+                                         const float4 *nd4, uint64_t c2, int lo_c, int hi_c,
+                                         uint8_t *dsb, int r, uint64_t *ds_free, uint32_t ds_par,
+                                         bool wait_ds, volatile int *abort) {
+    uint32_t sr[2][kPartQ], dr[2][kPartQ];
+    tmem_ld16(tS, sr[0]);
+    tmem_ld16(tdP, dr[0]);
+    tmem_wait_ld();
     #pragma unroll
-    for (int cc = 0; cc < kHalfQ; cc += 4) {
-        const float4 nl = nl4[cc >> 2], nd = nd4[cc >> 2];
-        float x0, x1, x2, x3;
-        f2unpack(f2fma(f2pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), c2,
-                       f2pack(nl.x, nl.y)), x0, x1);
-        f2unpack(f2fma(f2pack(__uint_as_float(sr[cc + 2]), __uint_as_float(sr[cc + 3])), c2,
-                       f2pack(nl.z, nl.w)), x2, x3);
-        float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-        if constexpr (EDGE) {
-            p0 = (cc + 0 >= lo_c && cc + 0 < hi_c) ? p0 : 0.f;
-            p1 = (cc + 1 >= lo_c && cc + 1 < hi_c) ? p1 : 0.f;
-            p2 = (cc + 2 >= lo_c && cc + 2 < hi_c) ? p2 : 0.f;
-            p3 = (cc + 3 >= lo_c && cc + 3 < hi_c) ? p3 : 0.f;
+    for (int qi = 0; qi < kBlockQ / kPartQ; ++qi) {
+        const int cur = qi & 1;
+        if (qi + 1 < kBlockQ / kPartQ) {
+            tmem_ld16(tS + (qi + 1) * kPartQ, sr[cur ^ 1]);
+            tmem_ld16(tdP + (qi + 1) * kPartQ, dr[cur ^ 1]);
         }
-        float d0, d1, d2, d3;
-        f2unpack(f2mul(f2pack(p0, p1),
-                       f2add(f2pack(__uint_as_float(dr[cc]), __uint_as_float(dr[cc + 1])),
-                             f2pack(nd.x, nd.y))), d0, d1);
-        f2unpack(f2mul(f2pack(p2, p3),
-                       f2add(f2pack(__uint_as_float(dr[cc + 2]), __uint_as_float(dr[cc + 3])),
-                             f2pack(nd.z, nd.w))), d2, d3);
-        pk[cc >> 1] = pack_bf16(p0, p1);
-        pk[(cc >> 1) + 1] = pack_bf16(p2, p3);
-        dk[cc >> 1] = pack_bf16(d0, d1);
-        dk[(cc >> 1) + 1] = pack_bf16(d2, d3);
+        uint32_t pk[kPartQ / 2], dk[kPartQ / 2];
+        #pragma unroll
+        for (int cc = 0; cc < kPartQ; cc += 4) {
+            const int c = qi * kPartQ + cc;
+            const float4 nl = nl4[c >> 2], nd = nd4[c >> 2];
+            float x0, x1, x2, x3;
+            f2unpack(f2fma(f2pack(__uint_as_float(sr[cur][cc]), __uint_as_float(sr[cur][cc + 1])), c2,
+                           f2pack(nl.x, nl.y)), x0, x1);
+            f2unpack(f2fma(f2pack(__uint_as_float(sr[cur][cc + 2]), __uint_as_float(sr[cur][cc + 3])), c2,
+                           f2pack(nl.z, nl.w)), x2, x3);
+            float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            if constexpr (EDGE) {
+                p0 = (c + 0 >= lo_c && c + 0 < hi_c) ? p0 : 0.f;
+                p1 = (c + 1 >= lo_c && c + 1 < hi_c) ? p1 : 0.f;
+                p2 = (c + 2 >= lo_c && c + 2 < hi_c) ? p2 : 0.f;
+                p3 = (c + 3 >= lo_c && c + 3 < hi_c) ? p3 : 0.f;
+            }
+            float d0, d1, d2, d3;
+            f2unpack(f2mul(f2pack(p0, p1),
+                           f2add(f2pack(__uint_as_float(dr[cur][cc]), __uint_as_float(dr[cur][cc + 1])),
+                                 f2pack(nd.x, nd.y))), d0, d1);
+            f2unpack(f2mul(f2pack(p2, p3),
+                           f2add(f2pack(__uint_as_float(dr[cur][cc + 2]), __uint_as_float(dr[cur][cc + 3])),
+                                 f2pack(nd.z, nd.w))), d2, d3);
+            pk[cc >> 1] = pack_bf16(p0, p1);
+            pk[(cc >> 1) + 1] = pack_bf16(p2, p3);
+            dk[cc >> 1] = pack_bf16(d0, d1);
+            dk[(cc >> 1) + 1] = pack_bf16(d2, d3);
+        }
+        tmem_st8(tS + qi * (kPartQ / 2), pk);
+        // dK and dQ^T of tile n-2 read this dSᵀ buffer
+        if (qi == 0 && wait_ds && !mbar_wait_warp(ds_free, ds_par, abort)) {
+            tmem_wait_ld();     // the next step's load is in flight
+            return false;
+        }
+        #pragma unroll
+        for (int c2i = 0; c2i < 2; ++c2i) {
+            const int ch = qi * 2 + c2i;
+            const uint4 v = make_uint4(dk[4 * c2i], dk[4 * c2i + 1], dk[4 * c2i + 2], dk[4 * c2i + 3]);
+            *reinterpret_cast<uint4 *>(dsb + ((ch ^ (r & 7)) << 4)) = v;
+        }
+        if (qi + 1 < kBlockQ / kPartQ) tmem_wait_ld();
     }
+    return true;
 }
 
 template <int DH>
@@ -417,11 +449,8 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
             const int qmax = min(q0 + kBlockQ, w.L) - 1;
             const bool edge = (w.j0 + kBlockK > w.L) || (p.causal && w.jl > q0) ||
                               (p.window > 0 && w.j0 <= qmax - p.window);
-            // Sᵀ and dPᵀ rows of this key in two halves of 32 queries, each
-            // loaded, turned into Pᵀ (over Sᵀ columns the half has read) and
-            // dSᵀ, and stored before the next.  The mask of an edge tile is
-            // the column range [lo_c, hi_c) of this key's visible queries, a
-            // select per value, so the unrolled loop has no branches.
+            // The mask of an edge tile: the column range [lo_c, hi_c) of this
+            // key's visible queries.
             int lo_c = 0, hi_c = kBlockQ;
             if (!key_ok) {
                 lo_c = kBlockQ;
@@ -431,31 +460,12 @@ __device__ void softmax_wg(const Params &p, Shared &sh, uint8_t *smem) {
                 if (p.window > 0) hi_c = min(kBlockQ, kj + p.window - q0);   // query < key + W
             }
             const uint64_t c2 = f2pack(sl2, sl2);
-            #pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t sr[kHalfQ], dr[kHalfQ];
-                tmem_ld32(tS + hh * kHalfQ, sr);
-                tmem_ld32(tdP + hh * kHalfQ, dr);
-                tmem_wait_ld();
-                uint32_t pk[kHalfQ / 2], dk[kHalfQ / 2];
-                const float4 *nl = nl4 + hh * (kHalfQ / 4), *nd = nd4 + hh * (kHalfQ / 4);
-                if (edge)
-                    grad_half<true>(sr, dr, nl, nd, c2, lo_c - hh * kHalfQ, hi_c - hh * kHalfQ, pk, dk);
-                else
-                    grad_half<false>(sr, dr, nl, nd, c2, 0, 0, pk, dk);
-                tmem_st16(tS + hh * (kHalfQ / 2), pk);
-                // dK and dQ^T of tile n-2 read this dSᵀ buffer
-                if (hh == 0 && n >= 2 &&
-                    !mbar_wait_warp(&sh.ds_free[wg], ((n - 2) >> 1) & 1, abort)) return;
-                // dSᵀ row r: eight 16-byte chunks of 8 queries, chunk index
-                // XOR (row & 7) (128-byte swizzle); this half holds four
-                #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int ch = hh * 4 + c4;
-                    const uint4 v = make_uint4(dk[4 * c4], dk[4 * c4 + 1], dk[4 * c4 + 2], dk[4 * c4 + 3]);
-                    *reinterpret_cast<uint4 *>(dsb + ((ch ^ (r & 7)) << 4)) = v;
-                }
-            }
+            const bool ok = edge
+                ? grad_row<true>(tS, tdP, nl4, nd4, c2, lo_c, hi_c, dsb, r, &sh.ds_free[wg],
+                                 ((n - 2) >> 1) & 1, n >= 2, abort)
+                : grad_row<false>(tS, tdP, nl4, nd4, c2, 0, 0, dsb, r, &sh.ds_free[wg],
+                                  ((n - 2) >> 1) & 1, n >= 2, abort);
+            if (!ok) return;
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();

@@ -276,12 +276,6 @@ __device__ __forceinline__ bool waitw(uint64_t *bar, uint32_t parity, volatile i
 }
 enum : int { kRoleSoftmax = 0, kRoleControl = 2 };
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
-                   "r"(r[6]), "r"(r[7]) : "memory");
-}
-
 // ---------------------------------------------------------------- producer
 // Whole warp: a unit's block-table entries are read once, one per lane; lane
 // 0 issues one K and one V copy per page of each tile.
