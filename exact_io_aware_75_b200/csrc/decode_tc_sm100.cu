@@ -703,19 +703,17 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
         }
         // conditional rescale: the reference moves only when the tile's
         // maximum exceeds it by the threshold (P <= 2^8 otherwise)
+        // (selects, not branches: the G heads' exponentials overlap)
         float alpha[G];
         bool resc = false;
         #pragma unroll
         for (int j = 0; j < G; ++j) {
-            alpha[j] = 1.f;
-            if (first) {
-                m[j] = mx[j];
-            } else if (mx[j] > m[j] + kRescaleThreshold) {
-                alpha[j] = ex2(m[j] - mx[j]);
-                m[j] = mx[j];
-                l[j] *= alpha[j];
-                resc = true;
-            }
+            const bool up = !first && mx[j] > m[j] + kRescaleThreshold;
+            const float a = ex2(m[j] - mx[j]);
+            alpha[j] = up ? a : 1.f;
+            l[j] *= alpha[j];
+            m[j] = (first || up) ? mx[j] : m[j];
+            resc |= up;
         }
         float pv[G];
         #pragma unroll
@@ -752,11 +750,11 @@ __device__ void softmax_wg(const TcParams &p, TcShared &sh, uint8_t *smem) {
                 asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr + Ly::kPTerm), "r"(lo[j]) : "memory");
             }
         }
-        if (writer) {
-            #pragma unroll
-            for (int j = 0; j < G; ++j) sh.alpha[b][h * G + j] = alpha[j];
-            if (resc) sh.resc[b] = (int)i;
-        }
+        // every row of head h holds the same alpha: all lanes store it (one
+        // value per address, no divergent branch)
+        #pragma unroll
+        for (int j = 0; j < G; ++j) sh.alpha[b][h * G + j] = alpha[j];
+        if (resc) sh.resc[b] = (int)i;
         // V codes of rows past the sequence are zeroed in the stage: P is zero
         // there, and 0 * NaN would poison O (P·V reads the codes as they are)
         if (__any_sync(0xffffffffu, !valid)) {
