@@ -383,12 +383,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                 pmax[0] = pmax_own[0];
             }
             // ---- conditional rescale (uniform across the warp: every lane
-            // holds the same m_ref and page max for every head)
+            // holds the same m_ref and page max for every head); one branch
+            // for all heads, so the common path stays one block
+            bool any_up = false;
             #pragma unroll
-            for (int qh = 0; qh < QPW; ++qh) {
-                if (pmax[qh] > m_ref[qh] + kRescaleThreshold) {
-                    const float alpha = (m_ref[qh] == -INFINITY) ? 0.f : ex2(m_ref[qh] - pmax[qh]);
-                    m_ref[qh] = pmax[qh];
+            for (int qh = 0; qh < QPW; ++qh) any_up |= pmax[qh] > m_ref[qh] + kRescaleThreshold;
+            if (any_up) {
+                #pragma unroll
+                for (int qh = 0; qh < QPW; ++qh) {
+                    const bool up = pmax[qh] > m_ref[qh] + kRescaleThreshold;
+                    const float alpha = !up ? 1.f
+                                      : (m_ref[qh] == -INFINITY) ? 0.f : ex2(m_ref[qh] - pmax[qh]);
+                    m_ref[qh] = up ? pmax[qh] : m_ref[qh];
                     l_acc[qh] *= alpha;
                     const uint64_t a2 = f2pack(alpha, alpha);
                     #pragma unroll
@@ -419,31 +425,41 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                     pr[k][0] = __shfl_sync(0xffffffffu, p_own[0], (tg << 3) + 2 * k);
                 }
             }
-            // ---- P V over this lane's tokens
+            // ---- P V over this lane's tokens (a full page in one block; the
+            // sequence's last page checks each slot, since slots past
+            // seq_len may hold anything)
+            auto pv_slot = [&](int k) {
+                const int t = tg + 4 * k;
+                uint64_t vv2[DPL / 2];
+                if constexpr (FP8) {
+                    unpack_e4m3<DPL>(sV + (size_t)(t * p.HG + hl) * D + DPL * ds, vv2);
+                } else {
+                    const uint16_t *vr = reinterpret_cast<const uint16_t *>(sV) +
+                                         ((size_t)(t * p.HG + hl) * D + 8 * ds);
+                    #pragma unroll
+                    for (int b = 0; b < DPL / 8; ++b)
+                        unpack8x2(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv2[4 * b]);
+                }
+                #pragma unroll
+                for (int qh = 0; qh < QPW; ++qh) {
+                    const float pv = FP8 ? pr[k][qh] * vs_cur : pr[k][qh];
+                    const uint64_t pp = f2pack(pv, pv);
+                    #pragma unroll
+                    for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2fma(pp, vv2[i], o2[qh][i]);
+                }
+            };
             #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int t = tg + 4 * k;
                 #pragma unroll
                 for (int qh = 0; qh < QPW; ++qh) l_acc[qh] += pr[k][qh];
-                if (t < nvalid) {   // slots past seq_len may hold anything
-                    uint64_t vv2[DPL / 2];
-                    if constexpr (FP8) {
-                        unpack_e4m3<DPL>(sV + (size_t)(t * p.HG + hl) * D + DPL * ds, vv2);
-                    } else {
-                        const uint16_t *vr = reinterpret_cast<const uint16_t *>(sV) +
-                                             ((size_t)(t * p.HG + hl) * D + 8 * ds);
-                        #pragma unroll
-                        for (int b = 0; b < DPL / 8; ++b)
-                            unpack8x2(*reinterpret_cast<const uint4 *>(vr + 64 * b), &vv2[4 * b]);
-                    }
-                    #pragma unroll
-                    for (int qh = 0; qh < QPW; ++qh) {
-                        const float pv = FP8 ? pr[k][qh] * vs_cur : pr[k][qh];
-                        const uint64_t pp = f2pack(pv, pv);
-                        #pragma unroll
-                        for (int i = 0; i < DPL / 2; ++i) o2[qh][i] = f2fma(pp, vv2[i], o2[qh][i]);
-                    }
-                }
+            }
+            if (nvalid == kPage) {
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) pv_slot(k);
+            } else {
+                #pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (tg + 4 * k < nvalid) pv_slot(k);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.empty[st]);
